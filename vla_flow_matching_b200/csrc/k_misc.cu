@@ -1,0 +1,294 @@
+// Small per-call and per-step kernels of the pi0 denoising loop: prefix-mask
+// compaction, the batch-invariant half of the action-time MLP, state/action
+// input projections, RMSNorm, RoPE, gated GELU and the final norm + action
+// out-projection with the Euler update.
+//
+// Definitions follow the vllm-omni page "vllm_omni/diffusion/models/pi0/
+// modeling_pi0.py" (functions named at each kernel).
+#include "common.cuh"
+#include "kernels.cuh"
+
+namespace pi0x {
+
+// Count of valid prefix tokens n_b and their positions, in order
+// (`denoise_step`: position ids continue at sum(prefix_pad_masks)).
+__global__ void __launch_bounds__(256) k_prep_mask(const CallPtrs *cp, int P, int *nvalid, int *vidx) {
+  const int b = blockIdx.x;
+  const uint8_t *m = cp->mask + (size_t)b * P;
+  __shared__ int warp_tot[8];
+  __shared__ int base;
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  if (threadIdx.x == 0) base = 0;
+  __syncthreads();
+  for (int p0 = 0; p0 < P; p0 += 256) {
+    const int p = p0 + threadIdx.x;
+    const bool v = (p < P) && (m[p] != 0);
+    const unsigned bal = __ballot_sync(0xffffffffu, v);
+    if (lane == 0) warp_tot[w] = __popc(bal);
+    __syncthreads();
+    int off = base;
+    for (int i = 0; i < w; ++i) off += warp_tot[i];
+    if (v) vidx[(size_t)b * P + off + __popc(bal & ((1u << lane) - 1u))] = p;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      int t = 0;
+      for (int i = 0; i < 8; ++i) t += warp_tot[i];
+      base += t;
+    }
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) nvalid[b] = base;
+}
+
+void launch_prep_mask(const CallPtrs *cp, int B, int P, int *nvalid, int *vidx, cudaStream_t s) {
+  k_prep_mask<<<B, 256, 0, s>>>(cp, P, nvalid, vidx);
+}
+
+// tvec[k][n] = sum_i Wt[n][i] * temb_k[i] + b[n] for every Euler step k.
+// Wt is the time half of action_time_mlp_in (its input columns W..2W-1), temb_k the
+// float64 sinusoid of t_k = fp32(1 + k*(-1/N)) cast to fp32
+// (`create_sinusoidal_pos_embedding`, min period 4e-3, max period 4).  The result
+// is the same for every sample and action token, so it is formed once per call.
+template <typename TW>
+__global__ void __launch_bounds__(256) k_time_vec(const TW *wt, const float *bias, int num_steps, float *tvec) {
+  __shared__ float temb[kWidth];
+  const int k = blockIdx.x;
+  const double dt = -1.0 / (double)num_steps;
+  const float t = (float)(1.0 + (double)k * dt);
+  constexpr int half = kWidth / 2;
+  for (int i = threadIdx.x; i < half; i += blockDim.x) {
+    const double frac = (double)i / (double)(half - 1);
+    const double period = 4e-3 * pow(1000.0, frac);
+    const double ang = (2.0 * 3.141592653589793 / period) * (double)t;
+    temb[i] = (float)sin(ang);
+    temb[half + i] = (float)cos(ang);
+  }
+  __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int o = 0; o < 4; ++o) {
+    const int n = blockIdx.y * 32 + warp * 4 + o;
+    const TW *row = wt + (size_t)n * kWidth;
+    float acc = 0.f;
+    for (int i = lane; i < kWidth; i += 32) acc = fmaf(to_f32(row[i]), temb[i], acc);
+    acc = warp_sum(acc);
+    if (lane == 0) tvec[(size_t)k * kWidth + n] = acc + bias[n];
+  }
+}
+
+template <typename TW>
+void launch_time_vec(const TW *w_time, const float *bias, int num_steps, float *tvec, cudaStream_t s) {
+  k_time_vec<TW><<<dim3(num_steps, kWidth / 32), 256, 0, s>>>(w_time, bias, num_steps, tvec);
+}
+
+// State token: h[b] = state_proj(state[b]) (`embed_suffix`).
+template <typename TW>
+__global__ void __launch_bounds__(256) k_state_embed(const CallPtrs *cp, const TW *w, const float *bias, int S,
+                                                      float *h) {
+  __shared__ float sv[64];
+  const int b = blockIdx.x;
+  for (int i = threadIdx.x; i < S; i += blockDim.x) sv[i] = cp->state[(size_t)b * S + i];
+  __syncthreads();
+  for (int n = threadIdx.x; n < kWidth; n += blockDim.x) {
+    float acc = 0.f;
+    for (int i = 0; i < S; ++i) acc = fmaf(to_f32(w[(size_t)n * S + i]), sv[i], acc);
+    h[(size_t)b * kWidth + n] = acc + bias[n];
+  }
+}
+
+template <typename TW>
+void launch_state_embed(const CallPtrs *cp, const TW *w, const float *b, int B, int S, float *h, cudaStream_t s) {
+  k_state_embed<TW><<<B, 256, 0, s>>>(cp, w, b, S, h);
+}
+
+// Action tokens: out[i] = action_in_proj(x[i]) for every (sample, horizon) row.
+template <typename TW, typename T>
+__global__ void __launch_bounds__(256) k_action_in(const float *x, const TW *w, const float *bias, int A, T *out) {
+  __shared__ float xv[64];
+  const int r = blockIdx.x;
+  for (int i = threadIdx.x; i < A; i += blockDim.x) xv[i] = x[(size_t)r * A + i];
+  __syncthreads();
+  for (int n = threadIdx.x; n < kWidth; n += blockDim.x) {
+    float acc = 0.f;
+    for (int i = 0; i < A; ++i) acc = fmaf(to_f32(w[(size_t)n * A + i]), xv[i], acc);
+    out[(size_t)r * kWidth + n] = from_f32<T>(acc + bias[n]);
+  }
+}
+
+template <typename TW, typename T>
+void launch_action_in(const float *x, const TW *w, const float *b, int rows, int A, T *out, cudaStream_t s) {
+  k_action_in<TW, T><<<rows, 256, 0, s>>>(x, w, b, A, out);
+}
+
+// Gemma RMSNorm: out = h * (1/sqrt(mean(h^2) + 1e-6)) * (1 + gain), one warp per row.
+template <typename T>
+__global__ void __launch_bounds__(256) k_rmsnorm(const float *h, int row0, int rows, const float *gain, T *out) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int r = blockIdx.x * 8 + warp;
+  if (r >= rows) return;
+  const size_t row = (size_t)(row0 + r);
+  const float4 *src = reinterpret_cast<const float4 *>(h + row * kWidth);
+  float4 v[8];
+  float ss = 0.f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    v[i] = src[lane + 32 * i];
+    ss += v[i].x * v[i].x + v[i].y * v[i].y + v[i].z * v[i].z + v[i].w * v[i].w;
+  }
+  ss = warp_sum(ss);
+  const float inv = 1.0f / sqrtf(ss / (float)kWidth + kRmsEps);
+  const float4 *g4 = reinterpret_cast<const float4 *>(gain);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float4 g = g4[lane + 32 * i];
+    const int c = 4 * (lane + 32 * i);
+    T *o = out + row * kWidth + c;
+    o[0] = from_f32<T>((v[i].x * inv) * (1.0f + g.x));
+    o[1] = from_f32<T>((v[i].y * inv) * (1.0f + g.y));
+    o[2] = from_f32<T>((v[i].z * inv) * (1.0f + g.z));
+    o[3] = from_f32<T>((v[i].w * inv) * (1.0f + g.w));
+  }
+}
+
+template <typename T>
+void launch_rmsnorm(const float *h, int row0, int rows, const float *gain, T *out, cudaStream_t s) {
+  if (rows <= 0) return;
+  k_rmsnorm<T><<<(rows + 7) / 8, 256, 0, s>>>(h, row0, rows, gain, out);
+}
+
+// (b, j) of an activation row: state rows first, then b*H + (j-1).
+__device__ __forceinline__ void row_to_bj(int r, int B, int H, int &b, int &j) {
+  if (r < B) {
+    b = r;
+    j = 0;
+  } else {
+    b = (r - B) / H;
+    j = 1 + (r - B) % H;
+  }
+}
+
+// Rotate-half RoPE of q (8 heads) and k at position n_b + j, v copied through
+// (`_compute_layer_suffix_only` with HF `apply_rotary_pos_emb`).  Angles are fp32
+// products pos * inv_freq[i]; cos/sin are the accurate CUDA sincosf.
+template <typename T>
+__global__ void __launch_bounds__(256) k_rope_qkv(const float *raw, int row0, Geo g, const int *nvalid,
+                                                   const float *inv_freq, T *q, T *ks, T *vs) {
+  const int r = row0 + blockIdx.x;
+  int b, j;
+  row_to_bj(r, g.B, g.H, b, j);
+  const float pos = (float)(nvalid[b] + j);
+  const float *src = raw + (size_t)r * kQkvDim;
+  constexpr int half = kHeadDim / 2;
+  for (int p = threadIdx.x; p < (kHeads + 1) * half; p += blockDim.x) {
+    const int hd = p / half, i = p % half;
+    float sn, cs;
+    sincosf(pos * inv_freq[i], &sn, &cs);
+    const float a = src[hd * kHeadDim + i], bb = src[hd * kHeadDim + half + i];
+    const float lo = a * cs - bb * sn, hi = bb * cs + a * sn;
+    if (hd < kHeads) {
+      q[(size_t)r * kQDim + hd * kHeadDim + i] = from_f32<T>(lo);
+      q[(size_t)r * kQDim + hd * kHeadDim + half + i] = from_f32<T>(hi);
+    } else {
+      ks[(size_t)r * kHeadDim + i] = from_f32<T>(lo);
+      ks[(size_t)r * kHeadDim + half + i] = from_f32<T>(hi);
+    }
+  }
+  for (int d = threadIdx.x; d < kHeadDim; d += blockDim.x)
+    vs[(size_t)r * kHeadDim + d] = from_f32<T>(src[kQDim + kHeadDim + d]);
+}
+
+template <typename T>
+void launch_rope_qkv(const float *raw, int row0, int rows, const Geo &g, const int *nvalid, const float *inv_freq,
+                     T *q, T *ks, T *vs, cudaStream_t s) {
+  if (rows <= 0) return;
+  k_rope_qkv<T><<<rows, 256, 0, s>>>(raw, row0, g, nvalid, inv_freq, q, ks, vs);
+}
+
+// Gemma MLP activation: act = gelu_tanh(gate) * up, raw row = [gate(4096) | up(4096)].
+template <typename T>
+__global__ void __launch_bounds__(256) k_geglu(const float *raw, int row0, T *act) {
+  const size_t r = (size_t)(row0 + blockIdx.x);
+  for (int f = threadIdx.x; f < kMlp; f += blockDim.x) {
+    const float gt = raw[r * 2 * kMlp + f], up = raw[r * 2 * kMlp + kMlp + f];
+    act[r * kMlp + f] = from_f32<T>(gelu_tanh_f(gt) * up);
+  }
+}
+
+template <typename T>
+void launch_geglu(const float *raw, int row0, int rows, T *act, cudaStream_t s) {
+  if (rows <= 0) return;
+  k_geglu<T><<<rows, 256, 0, s>>>(raw, row0, act);
+}
+
+// Final RMSNorm of an action token, v = action_out_proj(.) in fp32, then the
+// Euler update x <- x + dt*v (`denoise_step` tail and `sample_actions`); the last
+// step also writes x_0.
+__global__ void __launch_bounds__(256) k_final_euler(const float *h, Geo g, const float *gain, const float *w_out,
+                                                      const float *b_out, float dt, float *x, const CallPtrs *cp,
+                                                      int last) {
+  __shared__ float y[kWidth];
+  __shared__ float red[8];
+  const int i = blockIdx.x;  // action row index b*H + (j-1)
+  const float *src = h + (size_t)(g.B + i) * kWidth;
+  float ss = 0.f;
+  for (int c = threadIdx.x; c < kWidth; c += blockDim.x) {
+    const float v = src[c];
+    y[c] = v;
+    ss += v * v;
+  }
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  ss = warp_sum(ss);
+  if (lane == 0) red[warp] = ss;
+  __syncthreads();
+  float tot = 0.f;
+  for (int w = 0; w < 8; ++w) tot += red[w];
+  const float inv = 1.0f / sqrtf(tot / (float)kWidth + kRmsEps);
+  for (int c = threadIdx.x; c < kWidth; c += blockDim.x) y[c] = (y[c] * inv) * (1.0f + gain[c]);
+  __syncthreads();
+  for (int a = warp; a < g.A; a += 8) {
+    const float *wr = w_out + (size_t)a * kWidth;
+    float acc = 0.f;
+    for (int c = lane; c < kWidth; c += 32) acc = fmaf(wr[c], y[c], acc);
+    acc = warp_sum(acc);
+    if (lane == 0) {
+      const float v = acc + b_out[a];
+      const size_t xi = (size_t)i * g.A + a;
+      const float xn = __fadd_rn(x[xi], __fmul_rn(dt, v));
+      x[xi] = xn;
+      if (last) cp->x0[xi] = xn;
+    }
+  }
+}
+
+void launch_final_euler(const float *h, const Geo &g, const float *gain, const float *w_out, const float *b_out,
+                        float dt, float *x, const CallPtrs *cp, int last, cudaStream_t s) {
+  k_final_euler<<<g.B * g.H, 256, 0, s>>>(h, g, gain, w_out, b_out, dt, x, cp, last);
+}
+
+__global__ void k_copy_x1(const CallPtrs *cp, int n, float *x) {
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) x[i] = cp->x1[i];
+}
+void launch_copy_x1(const CallPtrs *cp, int n, float *x, cudaStream_t s) {
+  k_copy_x1<<<(n + 255) / 256 < 1024 ? (n + 255) / 256 : 1024, 256, 0, s>>>(cp, n, x);
+}
+
+// ---- explicit instantiations ----
+template void launch_time_vec<float>(const float *, const float *, int, float *, cudaStream_t);
+template void launch_time_vec<bf16>(const bf16 *, const float *, int, float *, cudaStream_t);
+template void launch_state_embed<float>(const CallPtrs *, const float *, const float *, int, int, float *,
+                                        cudaStream_t);
+template void launch_state_embed<bf16>(const CallPtrs *, const bf16 *, const float *, int, int, float *,
+                                       cudaStream_t);
+template void launch_action_in<float, float>(const float *, const float *, const float *, int, int, float *,
+                                             cudaStream_t);
+template void launch_action_in<bf16, bf16>(const float *, const bf16 *, const float *, int, int, bf16 *,
+                                           cudaStream_t);
+template void launch_rmsnorm<float>(const float *, int, int, const float *, float *, cudaStream_t);
+template void launch_rmsnorm<bf16>(const float *, int, int, const float *, bf16 *, cudaStream_t);
+template void launch_rope_qkv<float>(const float *, int, int, const Geo &, const int *, const float *, float *,
+                                     float *, float *, cudaStream_t);
+template void launch_rope_qkv<bf16>(const float *, int, int, const Geo &, const int *, const float *, bf16 *,
+                                    bf16 *, bf16 *, cudaStream_t);
+template void launch_geglu<float>(const float *, int, int, float *, cudaStream_t);
+template void launch_geglu<bf16>(const float *, int, int, bf16 *, cudaStream_t);
+
+}  // namespace pi0x

@@ -1,0 +1,89 @@
+// Internal launch interface of the pi0x kernels (host side).  Not part of the ABI.
+//
+// Row layout of every per-token activation buffer for a batch of B samples with
+// horizon H (R = B + B*H rows): rows [0, B) hold the state token of sample b,
+// rows B + b*H + (j-1) hold action token j = 1..H of sample b.  The state rows
+// come first so that steps after the first one, which reuse the state token's
+// hidden states and K/V (they depend on neither x_t nor t), run on the
+// contiguous row range [B, R).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace pi0x {
+
+typedef __nv_bfloat16 bf16;
+
+// Pointers a call hands in; kept in device memory so that a captured CUDA graph
+// stays valid when the caller's buffers change between calls.
+constexpr int kMaxDepth = 32;
+struct CallPtrs {
+  const bf16 *prefix_k[kMaxDepth];
+  const bf16 *prefix_v[kMaxDepth];
+  const uint8_t *mask;
+  const float *state;
+  const float *x1;
+  float *x0;
+};
+
+// GEMM epilogues: D[m][n] = sum_k A[m][k] * Bw[n][k]
+enum Epi : int {
+  EPI_STORE_F32 = 0,   // out_f32[m][n] = D
+  EPI_BIAS_F32 = 1,    // out_f32[m][n] = D + vec[n]
+  EPI_VEC_SILU = 2,    // out_T[m][n] = silu(D + vec[n])
+  EPI_RESID_F32 = 3,   // out_f32[m][n] += D
+};
+
+struct GemmOut {
+  void *out;      // fp32 or activation type, row-major
+  int ldo;        // elements
+  int out_row0;   // output row of GEMM row 0
+  const float *vec;
+};
+
+// Batch geometry of one call.
+struct Geo {
+  int B, H, A, S, P, R;   // R = B + B*H
+};
+
+// ---- misc kernels (k_misc.cu) ----
+void launch_prep_mask(const CallPtrs *cp, int B, int P, int *nvalid, int *vidx, cudaStream_t s);
+template <typename TW>
+void launch_time_vec(const TW *w_time, const float *bias, int num_steps, float *tvec, cudaStream_t s);
+template <typename TW>
+void launch_state_embed(const CallPtrs *cp, const TW *w, const float *b, int B, int S, float *h, cudaStream_t s);
+template <typename TW, typename T>
+void launch_action_in(const float *x, const TW *w, const float *b, int rows, int A, T *out, cudaStream_t s);
+template <typename T>
+void launch_rmsnorm(const float *h, int row0, int rows, const float *gain, T *out, cudaStream_t s);
+template <typename T>
+void launch_rope_qkv(const float *raw, int row0, int rows, const Geo &g, const int *nvalid, const float *inv_freq,
+                     T *q, T *ks, T *vs, cudaStream_t s);
+template <typename T>
+void launch_geglu(const float *raw, int row0, int rows, T *act, cudaStream_t s);
+void launch_final_euler(const float *h, const Geo &g, const float *gain, const float *w_out, const float *b_out,
+                        float dt, float *x, const CallPtrs *cp, int last, cudaStream_t s);
+void launch_copy_x1(const CallPtrs *cp, int n, float *x, cudaStream_t s);
+
+// ---- attention (k_attn.cu) ----
+template <typename T>
+void launch_attention(const T *q, const T *ks, const T *vs, const CallPtrs *cp, int layer, const int *nvalid,
+                      const int *vidx, const Geo &g, int step0, T *out, cudaStream_t s);
+
+// ---- GEMMs ----
+template <typename OutT>
+void launch_gemm_simt(const float *A, int lda, const float *Bw, int ldb, int M, int N, int K, int epi,
+                      const GemmOut &o, cudaStream_t s);
+
+struct TcGemm {           // one tcgen05 GEMM with its tensor maps (built once)
+  CUtensorMap tmA, tmB;
+  int N, K, BN;
+};
+template <typename OutT>
+void launch_gemm_tc(const TcGemm &g, int a_row0, int M, int epi, const GemmOut &o, unsigned *err,
+                    cudaStream_t s);
+
+}  // namespace pi0x

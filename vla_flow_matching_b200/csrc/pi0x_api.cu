@@ -1,0 +1,667 @@
+// C ABI of libpi0x (include/pi0x.h): handle life cycle, weight repack, workspace,
+// tensor maps and the per-call kernel sequence of the pi0 Euler loop.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <string.h>
+
+#include <cmath>
+#include <new>
+#include <string>
+#include <vector>
+
+#include "../../include/pi0x.h"
+#include "../../include/pi0x_debug.h"
+#include "common.cuh"
+#include "kernels.cuh"
+
+using namespace pi0x;
+
+namespace {
+
+thread_local std::string g_last_error;
+
+int cuda_fail(cudaError_t e, const char *what) {
+  g_last_error = std::string(what) + ": " + cudaGetErrorString(e);
+  cudaGetLastError();
+  return e == cudaErrorMemoryAllocation ? PI0X_ENOMEM : PI0X_ECUDA;
+}
+#define CK(call)                                  \
+  do {                                            \
+    cudaError_t e_ = (call);                      \
+    if (e_ != cudaSuccess) return cuda_fail(e_, #call); \
+  } while (0)
+
+// ---- device arena: one cudaMalloc, 1 KiB aligned sub-allocations -------------
+struct Arena {
+  uint8_t *base = nullptr;
+  size_t size = 0, used = 0;
+  void *take(size_t bytes) {
+    size_t off = (used + 1023) & ~size_t(1023);
+    if (off + bytes > size) return nullptr;
+    used = off + bytes;
+    return base + off;
+  }
+};
+size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// ---- cuTensorMapEncodeTiled through the runtime's driver entry point ---------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn get_encode() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+// 2-D bf16 K-major map: `rows` x `cols` elements with row pitch `pitch` elements,
+// box = 64 columns x box_rows rows, 128-byte swizzle, zero fill out of bounds.
+bool make_map(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols, uint64_t pitch, uint32_t box_rows) {
+  EncodeTiledFn enc = get_encode();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {pitch * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+uint16_t f32_to_bf16_bits(float f) {
+  uint32_t u;
+  memcpy(&u, &f, 4);
+  if ((u & 0x7fffffffu) > 0x7f800000u) return 0x7fc0;  // NaN
+  u += 0x7fffu + ((u >> 16) & 1u);
+  return (uint16_t)(u >> 16);
+}
+float bf16_bits_to_f32(uint16_t b) {
+  uint32_t u = (uint32_t)b << 16;
+  float f;
+  memcpy(&f, &u, 4);
+  return f;
+}
+
+struct LayerW {
+  float *in_norm, *post_norm;
+  void *qkv, *o, *gu, *down;   // activation-type weights
+};
+
+struct Workspace {
+  int B = 0, P = 0, N = 0, R = 0;
+  Arena arena;
+  int *nvalid, *vidx;
+  float *tvec, *xw, *h, *raw;
+  void *xn, *q, *ks, *vs, *att, *act, *a_emb, *u_emb;
+  // host-input staging (device side), allocated lazily
+  Arena stage;
+  size_t stage_B = 0, stage_P = 0;
+  bf16 *st_k = nullptr, *st_v = nullptr;
+  uint8_t *st_mask = nullptr;
+  float *st_state = nullptr, *st_x = nullptr;
+  // tensor maps of the activation operands (bf16 mode)
+  CUtensorMap m_xn, m_att, m_act, m_aemb, m_uemb;
+};
+
+}  // namespace
+
+struct pi0x_handle {
+  pi0x_config cfg;
+  int device = 0;
+  bool bf16 = true;
+  size_t act_bytes = 2;  // element size of activation-type tensors
+  Arena warena;
+  // weights (device)
+  void *state_w, *ain_w, *tin_a, *tin_t, *tout_w;
+  float *state_b, *ain_b, *tin_b, *tout_b, *aout_w, *aout_b, *fnorm, *inv_freq;
+  LayerW layer[kMaxDepth];
+  // weight-side tensor maps + tile widths (bf16 mode)
+  TcGemm g_tin, g_tout, g_qkv[kMaxDepth], g_o[kMaxDepth], g_gu[kMaxDepth], g_down[kMaxDepth];
+  Workspace ws;
+  CallPtrs *d_ptrs = nullptr;
+  unsigned *d_err = nullptr;
+  cudaStream_t last_stream = nullptr;
+};
+
+namespace {
+
+int validate_config(const pi0x_config *c) {
+  if (!c) return PI0X_EINVAL;
+  if (c->width != kWidth || c->mlp_dim != kMlp || c->num_heads != kHeads || c->num_kv_heads != 1 ||
+      c->head_dim != kHeadDim)
+    return PI0X_EUNSUPPORTED;
+  if (c->depth < 1 || c->depth > kMaxDepth || c->horizon < 1 || c->horizon > 64 || c->action_dim < 1 ||
+      c->action_dim > 64 || c->state_dim < 1 || c->state_dim > 64)
+    return PI0X_EINVAL;
+  if (c->precision != PI0X_BF16 && c->precision != PI0X_FP32) return PI0X_EINVAL;
+  return PI0X_OK;
+}
+
+// Read `n` elements of a weight array (host or device memory) as fp32.
+int fetch(const void *p, size_t n, int dtype, std::vector<float> &out) {
+  if (!p) {
+    g_last_error = "null weight pointer";
+    return PI0X_EINVAL;
+  }
+  out.resize(n);
+  if (dtype == PI0X_DTYPE_F32) {
+    CK(cudaMemcpy(out.data(), p, n * 4, cudaMemcpyDefault));
+  } else {
+    std::vector<uint16_t> tmp(n);
+    CK(cudaMemcpy(tmp.data(), p, n * 2, cudaMemcpyDefault));
+    for (size_t i = 0; i < n; ++i) out[i] = bf16_bits_to_f32(tmp[i]);
+  }
+  return PI0X_OK;
+}
+
+// Upload fp32 values as fp32 or as the activation type.
+int upload(pi0x_handle *h, const std::vector<float> &v, bool as_act, void **dst) {
+  const size_t es = as_act ? h->act_bytes : 4;
+  void *d = h->warena.take(v.size() * es);
+  if (!d) return PI0X_ENOMEM;
+  if (as_act && h->bf16) {
+    std::vector<uint16_t> b(v.size());
+    for (size_t i = 0; i < v.size(); ++i) b[i] = f32_to_bf16_bits(v[i]);
+    CK(cudaMemcpy(d, b.data(), b.size() * 2, cudaMemcpyHostToDevice));
+  } else {
+    CK(cudaMemcpy(d, v.data(), v.size() * 4, cudaMemcpyHostToDevice));
+  }
+  *dst = d;
+  return PI0X_OK;
+}
+
+size_t weight_bytes(const pi0x_config &c, size_t es) {
+  const size_t W = kWidth;
+  size_t act = W * c.state_dim + W * c.action_dim + 2 * W * W + W * W +
+               (size_t)c.depth * ((size_t)kQkvDim * W + W * kQDim + 2 * (size_t)kMlp * W + W * kMlp);
+  size_t f32 = 4 * W + (size_t)c.action_dim * W + c.action_dim + W + 128 + (size_t)c.depth * 2 * W;
+  return act * es + f32 * 4 + 64 * 1024 * (size_t)(16 + 6 * c.depth);
+}
+
+int pick_bn(int N) { return N >= 2048 ? 256 : 128; }
+
+int build_weight_maps(pi0x_handle *h) {
+  const int L = h->cfg.depth;
+  auto mk = [&](TcGemm &g, const void *w, int N, int K) {
+    g.N = N;
+    g.K = K;
+    g.BN = pick_bn(N);
+    return make_map(&g.tmB, w, N, K, K, g.BN);
+  };
+  bool ok = mk(h->g_tin, h->tin_a, kWidth, kWidth) && mk(h->g_tout, h->tout_w, kWidth, kWidth);
+  for (int l = 0; l < L && ok; ++l) {
+    ok = mk(h->g_qkv[l], h->layer[l].qkv, kQkvDim, kWidth) && mk(h->g_o[l], h->layer[l].o, kWidth, kQDim) &&
+         mk(h->g_gu[l], h->layer[l].gu, 2 * kMlp, kWidth) && mk(h->g_down[l], h->layer[l].down, kWidth, kMlp);
+  }
+  if (!ok) {
+    g_last_error = "cuTensorMapEncodeTiled failed for a weight operand";
+    return PI0X_ECUDA;
+  }
+  return PI0X_OK;
+}
+
+void free_workspace(Workspace &ws) {
+  if (ws.arena.base) cudaFree(ws.arena.base);
+  ws.arena = Arena();
+  ws.B = ws.P = ws.N = ws.R = 0;
+}
+
+int ensure_workspace(pi0x_handle *h, int B, int P, int N) {
+  Workspace &ws = h->ws;
+  if (ws.arena.base && B <= ws.B && P <= ws.P && N <= ws.N) return PI0X_OK;
+  const int nB = B > ws.B ? B : ws.B, nP = P > ws.P ? P : ws.P, nN = N > ws.N ? N : ws.N;
+  if (h->last_stream) cudaStreamSynchronize(h->last_stream);
+  free_workspace(ws);
+  const int H = h->cfg.horizon, A = h->cfg.action_dim, L = h->cfg.depth;
+  const size_t R = (size_t)nB + (size_t)nB * H;
+  const size_t es = h->act_bytes;
+  const size_t Rp = round_up(R, 128);  // TMA boxes may cover up to 127 rows past R
+  size_t bytes = 0;
+  auto add = [&](size_t b) { bytes += round_up(b, 1024) + 1024; };
+  add(4 * nB);
+  add(4 * (size_t)nB * (nP > 0 ? nP : 1));
+  add(4 * (size_t)nN * kWidth);
+  add(4 * (size_t)nB * H * A);
+  add(4 * Rp * kWidth);
+  add(4 * Rp * 2 * kMlp);
+  add(es * Rp * kWidth);
+  add(es * Rp * kQDim);
+  add(es * (size_t)L * Rp * kHeadDim);
+  add(es * (size_t)L * Rp * kHeadDim);
+  add(es * Rp * kQDim);
+  add(es * Rp * kMlp);
+  add(es * Rp * kWidth);
+  add(es * Rp * kWidth);
+  void *base = nullptr;
+  CK(cudaMalloc(&base, bytes));
+  ws.arena.base = static_cast<uint8_t *>(base);
+  ws.arena.size = bytes;
+  ws.nvalid = (int *)ws.arena.take(4 * nB);
+  ws.vidx = (int *)ws.arena.take(4 * (size_t)nB * (nP > 0 ? nP : 1));
+  ws.tvec = (float *)ws.arena.take(4 * (size_t)nN * kWidth);
+  ws.xw = (float *)ws.arena.take(4 * (size_t)nB * H * A);
+  ws.h = (float *)ws.arena.take(4 * Rp * kWidth);
+  ws.raw = (float *)ws.arena.take(4 * Rp * 2 * kMlp);
+  ws.xn = ws.arena.take(es * Rp * kWidth);
+  ws.q = ws.arena.take(es * Rp * kQDim);
+  ws.ks = ws.arena.take(es * (size_t)L * Rp * kHeadDim);
+  ws.vs = ws.arena.take(es * (size_t)L * Rp * kHeadDim);
+  ws.att = ws.arena.take(es * Rp * kQDim);
+  ws.act = ws.arena.take(es * Rp * kMlp);
+  ws.a_emb = ws.arena.take(es * Rp * kWidth);
+  ws.u_emb = ws.arena.take(es * Rp * kWidth);
+  CK(cudaMemset(base, 0, bytes));
+  ws.B = nB;
+  ws.P = nP;
+  ws.N = nN;
+  ws.R = (int)R;
+  if (h->bf16) {
+    bool ok = make_map(&ws.m_xn, ws.xn, Rp, kWidth, kWidth, 128) &&
+              make_map(&ws.m_att, ws.att, Rp, kQDim, kQDim, 128) &&
+              make_map(&ws.m_act, ws.act, Rp, kMlp, kMlp, 128) &&
+              make_map(&ws.m_aemb, ws.a_emb, Rp, kWidth, kWidth, 128) &&
+              make_map(&ws.m_uemb, ws.u_emb, Rp, kWidth, kWidth, 128);
+    if (!ok) {
+      g_last_error = "cuTensorMapEncodeTiled failed for an activation operand";
+      return PI0X_ECUDA;
+    }
+  }
+  return PI0X_OK;
+}
+
+int ensure_stage(pi0x_handle *h, int B, int P) {
+  Workspace &ws = h->ws;
+  if (ws.stage.base && (size_t)B <= ws.stage_B && (size_t)P <= ws.stage_P) return PI0X_OK;
+  if (h->last_stream) cudaStreamSynchronize(h->last_stream);
+  if (ws.stage.base) cudaFree(ws.stage.base);
+  ws.stage = Arena();
+  const int L = h->cfg.depth, H = h->cfg.horizon, A = h->cfg.action_dim, S = h->cfg.state_dim;
+  const size_t kv = (size_t)L * B * (size_t)(P > 0 ? P : 1) * kHeadDim * 2;
+  size_t bytes = 2 * round_up(kv, 1024) + round_up((size_t)B * (P > 0 ? P : 1), 1024) +
+                 round_up(4 * (size_t)B * S, 1024) + round_up(4 * (size_t)B * H * A, 1024) + 8 * 1024;
+  void *base = nullptr;
+  CK(cudaMalloc(&base, bytes));
+  ws.stage.base = (uint8_t *)base;
+  ws.stage.size = bytes;
+  ws.st_k = (bf16 *)ws.stage.take(kv);
+  ws.st_v = (bf16 *)ws.stage.take(kv);
+  ws.st_mask = (uint8_t *)ws.stage.take((size_t)B * (P > 0 ? P : 1));
+  ws.st_state = (float *)ws.stage.take(4 * (size_t)B * S);
+  ws.st_x = (float *)ws.stage.take(4 * (size_t)B * H * A);
+  ws.stage_B = B;
+  ws.stage_P = P;
+  return PI0X_OK;
+}
+
+bool is_device_ptr(const void *p) {
+  cudaPointerAttributes a;
+  if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  return a.type == cudaMemoryTypeDevice || a.type == cudaMemoryTypeManaged;
+}
+
+// ---- the Euler loop -------------------------------------------------------------
+template <typename T>
+int enqueue_loop(pi0x_handle *h, int B, int P, int N, cudaStream_t s) {
+  Workspace &ws = h->ws;
+  const pi0x_config &c = h->cfg;
+  const int H = c.horizon, A = c.action_dim, L = c.depth;
+  Geo g{B, H, A, c.state_dim, P, B + B * H};
+  const int R = g.R, BH = B * H;
+  const float dt = (float)(-1.0 / (double)N);
+  const bool tc = h->bf16;
+  T *xn = (T *)ws.xn, *q = (T *)ws.q, *att = (T *)ws.att, *act = (T *)ws.act;
+  T *aemb = (T *)ws.a_emb, *uemb = (T *)ws.u_emb;
+  const size_t kv_stride = (size_t)R * kHeadDim;
+
+  launch_prep_mask(h->d_ptrs, B, P, ws.nvalid, ws.vidx, s);
+  launch_time_vec<T>((const T *)h->tin_t, h->tin_b, N, ws.tvec, s);
+  launch_copy_x1(h->d_ptrs, BH * A, ws.xw, s);
+
+  for (int k = 0; k < N; ++k) {
+    const int step0 = (k == 0);
+    const int row0 = step0 ? 0 : B;
+    const int M = R - row0;
+    if (step0) launch_state_embed<T>(h->d_ptrs, (const T *)h->state_w, h->state_b, B, c.state_dim, ws.h, s);
+    launch_action_in<T, T>(ws.xw, (const T *)h->ain_w, h->ain_b, BH, A, aemb, s);
+    GemmOut o_u{uemb, kWidth, 0, ws.tvec + (size_t)k * kWidth};
+    GemmOut o_h{ws.h, kWidth, B, h->tout_b};
+    if (tc) {
+      TcGemm gt = h->g_tin;
+      gt.tmA = ws.m_aemb;
+      launch_gemm_tc<bf16>(gt, 0, BH, EPI_VEC_SILU, o_u, h->d_err, s);
+      TcGemm go = h->g_tout;
+      go.tmA = ws.m_uemb;
+      launch_gemm_tc<bf16>(go, 0, BH, EPI_BIAS_F32, o_h, h->d_err, s);
+    } else {
+      launch_gemm_simt<float>((const float *)aemb, kWidth, (const float *)h->tin_a, kWidth, BH, kWidth, kWidth,
+                              EPI_VEC_SILU, o_u, s);
+      launch_gemm_simt<float>((const float *)uemb, kWidth, (const float *)h->tout_w, kWidth, BH, kWidth, kWidth,
+                              EPI_BIAS_F32, o_h, s);
+    }
+    for (int l = 0; l < L; ++l) {
+      const LayerW &lw = h->layer[l];
+      T *ks = (T *)ws.ks + (size_t)l * kv_stride, *vs = (T *)ws.vs + (size_t)l * kv_stride;
+      launch_rmsnorm<T>(ws.h, row0, M, lw.in_norm, xn, s);
+      GemmOut o_raw{ws.raw, kQkvDim, row0, nullptr};
+      if (tc) {
+        TcGemm gq = h->g_qkv[l];
+        gq.tmA = ws.m_xn;
+        launch_gemm_tc<bf16>(gq, row0, M, EPI_STORE_F32, o_raw, h->d_err, s);
+      } else {
+        launch_gemm_simt<float>((const float *)xn + (size_t)row0 * kWidth, kWidth, (const float *)lw.qkv, kWidth,
+                                M, kQkvDim, kWidth, EPI_STORE_F32, o_raw, s);
+      }
+      launch_rope_qkv<T>(ws.raw, row0, M, g, ws.nvalid, h->inv_freq, q, ks, vs, s);
+      launch_attention<T>(q, ks, vs, h->d_ptrs, l, ws.nvalid, ws.vidx, g, step0, att, s);
+      GemmOut o_res{ws.h, kWidth, row0, nullptr};
+      if (tc) {
+        TcGemm gO = h->g_o[l];
+        gO.tmA = ws.m_att;
+        launch_gemm_tc<bf16>(gO, row0, M, EPI_RESID_F32, o_res, h->d_err, s);
+      } else {
+        launch_gemm_simt<float>((const float *)att + (size_t)row0 * kQDim, kQDim, (const float *)lw.o, kQDim, M,
+                                kWidth, kQDim, EPI_RESID_F32, o_res, s);
+      }
+      launch_rmsnorm<T>(ws.h, row0, M, lw.post_norm, xn, s);
+      GemmOut o_gu{ws.raw, 2 * kMlp, row0, nullptr};
+      if (tc) {
+        TcGemm gg = h->g_gu[l];
+        gg.tmA = ws.m_xn;
+        launch_gemm_tc<bf16>(gg, row0, M, EPI_STORE_F32, o_gu, h->d_err, s);
+      } else {
+        launch_gemm_simt<float>((const float *)xn + (size_t)row0 * kWidth, kWidth, (const float *)lw.gu, kWidth, M,
+                                2 * kMlp, kWidth, EPI_STORE_F32, o_gu, s);
+      }
+      launch_geglu<T>(ws.raw, row0, M, act, s);
+      if (tc) {
+        TcGemm gd = h->g_down[l];
+        gd.tmA = ws.m_act;
+        launch_gemm_tc<bf16>(gd, row0, M, EPI_RESID_F32, o_res, h->d_err, s);
+      } else {
+        launch_gemm_simt<float>((const float *)act + (size_t)row0 * kMlp, kMlp, (const float *)lw.down, kMlp, M,
+                                kWidth, kMlp, EPI_RESID_F32, o_res, s);
+      }
+    }
+    launch_final_euler(ws.h, g, h->fnorm, h->aout_w, h->aout_b, dt, ws.xw, h->d_ptrs, k == N - 1, s);
+  }
+  CK(cudaGetLastError());
+  return PI0X_OK;
+}
+
+}  // namespace
+
+// ================================ C ABI =====================================
+extern "C" {
+
+int pi0x_version(void) { return 100; }
+
+int pi0x_debug_gemm_bf16(const void *A, const void *Bw, int M, int N, int K, float *D, int bn, void *stream) {
+  if (!A || !Bw || !D || M < 1 || N < 1 || K < 64 || K % 64 || (bn != 64 && bn != 128 && bn != 256) || N % bn)
+    return PI0X_EINVAL;
+  static unsigned *d_err = nullptr;
+  if (!d_err) {
+    CK(cudaMalloc(&d_err, sizeof(unsigned)));
+    CK(cudaMemset(d_err, 0, sizeof(unsigned)));
+  }
+  TcGemm g;
+  g.N = N;
+  g.K = K;
+  g.BN = bn;
+  if (!make_map(&g.tmA, A, M, K, K, 128) || !make_map(&g.tmB, Bw, N, K, K, bn)) {
+    g_last_error = "cuTensorMapEncodeTiled failed";
+    return PI0X_ECUDA;
+  }
+  cudaStream_t s = (cudaStream_t)stream;
+  GemmOut o{D, N, 0, nullptr};
+  launch_gemm_tc<float>(g, 0, M, EPI_STORE_F32, o, d_err, s);
+  CK(cudaGetLastError());
+  CK(cudaStreamSynchronize(s));
+  unsigned err = 0;
+  CK(cudaMemcpy(&err, d_err, sizeof(err), cudaMemcpyDeviceToHost));
+  if (err) {
+    cudaMemset(d_err, 0, sizeof(unsigned));
+    g_last_error = "device error word 0x" + std::to_string(err);
+    return PI0X_ETIMEOUT;
+  }
+  return PI0X_OK;
+}
+
+const char *pi0x_status_string(int st) {
+  switch (st) {
+    case PI0X_OK: return "ok";
+    case PI0X_EINVAL: return "invalid argument";
+    case PI0X_EUNSUPPORTED: return "unsupported configuration";
+    case PI0X_ENOMEM: return "out of memory";
+    case PI0X_ECUDA: return "CUDA error";
+    case PI0X_ETIMEOUT: return "device wait timed out";
+    case PI0X_EDEVICE: return "device reported an invalid launch";
+    default: return "unknown status";
+  }
+}
+
+const char *pi0x_last_error(void) { return g_last_error.c_str(); }
+
+int pi0x_create(const pi0x_config *cfg, const pi0x_weights *w, pi0x_handle **out) {
+  if (!out || !cfg || !w || !w->layers) return PI0X_EINVAL;
+  *out = nullptr;
+  int st = validate_config(cfg);
+  if (st) return st;
+  if (w->dtype != PI0X_DTYPE_BF16 && w->dtype != PI0X_DTYPE_F32) return PI0X_EINVAL;
+  int dev = 0;
+  CK(cudaGetDevice(&dev));
+  cudaDeviceProp prop;
+  CK(cudaGetDeviceProperties(&prop, dev));
+  if (prop.major != 10) {
+    g_last_error = "this library is built for sm_100 (B200)";
+    return PI0X_EUNSUPPORTED;
+  }
+  pi0x_handle *h = new (std::nothrow) pi0x_handle();
+  if (!h) return PI0X_ENOMEM;
+  h->cfg = *cfg;
+  h->device = dev;
+  h->bf16 = cfg->precision == PI0X_BF16;
+  h->act_bytes = h->bf16 ? 2 : 4;
+  if (h->bf16 && !get_encode()) {
+    g_last_error = "cuTensorMapEncodeTiled unavailable";
+    delete h;
+    return PI0X_ECUDA;
+  }
+  const pi0x_config &c = *cfg;
+  const size_t W = kWidth;
+  auto fail = [&](int code) {
+    pi0x_destroy(h);
+    return code;
+  };
+  void *base = nullptr;
+  size_t bytes = weight_bytes(c, h->act_bytes);
+  cudaError_t e = cudaMalloc(&base, bytes);
+  if (e != cudaSuccess) {
+    cuda_fail(e, "cudaMalloc(weights)");
+    delete h;
+    return PI0X_ENOMEM;
+  }
+  h->warena.base = (uint8_t *)base;
+  h->warena.size = bytes;
+  std::vector<float> v, v2, v3;
+  void *p = nullptr;
+#define FETCH(ptr, n, vec)                 \
+  do {                                     \
+    st = fetch((ptr), (n), w->dtype, vec); \
+    if (st) return fail(st);               \
+  } while (0)
+#define UP(vec, as_act, dst)                  \
+  do {                                        \
+    st = upload(h, vec, as_act, (void **)&(dst)); \
+    if (st) return fail(st);                  \
+  } while (0)
+  FETCH(w->state_proj_w, W * c.state_dim, v);  UP(v, true, h->state_w);
+  FETCH(w->state_proj_b, W, v);                UP(v, false, h->state_b);
+  FETCH(w->action_in_w, W * c.action_dim, v);  UP(v, true, h->ain_w);
+  FETCH(w->action_in_b, W, v);                 UP(v, false, h->ain_b);
+  FETCH(w->time_in_w, W * 2 * W, v);
+  v2.resize(W * W);
+  v3.resize(W * W);
+  for (size_t n = 0; n < W; ++n)
+    for (size_t i = 0; i < W; ++i) {
+      v2[n * W + i] = v[n * 2 * W + i];       // action half: columns 0..W-1
+      v3[n * W + i] = v[n * 2 * W + W + i];   // time half:   columns W..2W-1
+    }
+  UP(v2, true, h->tin_a);
+  UP(v3, true, h->tin_t);
+  FETCH(w->time_in_b, W, v);                   UP(v, false, h->tin_b);
+  FETCH(w->time_out_w, W * W, v);              UP(v, true, h->tout_w);
+  FETCH(w->time_out_b, W, v);                  UP(v, false, h->tout_b);
+  FETCH(w->action_out_w, W * c.action_dim, v); UP(v, false, h->aout_w);
+  FETCH(w->action_out_b, (size_t)c.action_dim, v); UP(v, false, h->aout_b);
+  FETCH(w->final_norm_w, W, v);                UP(v, false, h->fnorm);
+  for (int l = 0; l < c.depth; ++l) {
+    const pi0x_layer_weights &lw = w->layers[l];
+    LayerW &d = h->layer[l];
+    FETCH(lw.in_norm_w, W, v);   UP(v, false, d.in_norm);
+    FETCH(lw.post_norm_w, W, v); UP(v, false, d.post_norm);
+    // [q; k; v] rows -> one (2560, 1024) operand
+    std::vector<float> qkv;
+    FETCH(lw.q_w, (size_t)kQDim * W, v);
+    qkv.insert(qkv.end(), v.begin(), v.end());
+    FETCH(lw.k_w, (size_t)kHeadDim * W, v);
+    qkv.insert(qkv.end(), v.begin(), v.end());
+    FETCH(lw.v_w, (size_t)kHeadDim * W, v);
+    qkv.insert(qkv.end(), v.begin(), v.end());
+    UP(qkv, true, d.qkv);
+    FETCH(lw.o_w, W * kQDim, v); UP(v, true, d.o);
+    // [gate; up] rows -> one (8192, 1024) operand
+    std::vector<float> gu;
+    FETCH(lw.gate_w, (size_t)kMlp * W, v);
+    gu.insert(gu.end(), v.begin(), v.end());
+    FETCH(lw.up_w, (size_t)kMlp * W, v);
+    gu.insert(gu.end(), v.begin(), v.end());
+    UP(gu, true, d.gu);
+    FETCH(lw.down_w, W * kMlp, v); UP(v, true, d.down);
+  }
+  // RoPE inverse frequencies: 10000^(-2i/256), evaluated in double, rounded to fp32.
+  v.resize(kHeadDim / 2);
+  for (int i = 0; i < kHeadDim / 2; ++i) v[i] = (float)std::pow(10000.0, -2.0 * i / (double)kHeadDim);
+  UP(v, false, h->inv_freq);
+#undef FETCH
+#undef UP
+  if (h->bf16) {
+    st = build_weight_maps(h);
+    if (st) return fail(st);
+  }
+  e = cudaMalloc(&h->d_ptrs, sizeof(CallPtrs));
+  if (e == cudaSuccess) e = cudaMalloc(&h->d_err, sizeof(unsigned));
+  if (e == cudaSuccess) e = cudaMemset(h->d_err, 0, sizeof(unsigned));
+  if (e != cudaSuccess) return fail(cuda_fail(e, "cudaMalloc(handle)"));
+  *out = h;
+  return PI0X_OK;
+}
+
+int pi0x_sample(pi0x_handle *h, const void *const *prefix_k, const void *const *prefix_v,
+                const uint8_t *prefix_valid_mask, int B, int P, const float *state, const float *x1, int num_steps,
+                float *x0, void *stream) {
+  if (!h || !prefix_k || !prefix_v || !state || !x1 || !x0) return PI0X_EINVAL;
+  if (P > 0 && !prefix_valid_mask) return PI0X_EINVAL;
+  if (B < 1 || B > 4096 || P < 0 || P > 8192 || num_steps < 1 || num_steps > 1024) return PI0X_EINVAL;
+  const pi0x_config &c = h->cfg;
+  for (int l = 0; l < c.depth; ++l)
+    if (P > 0 && (!prefix_k[l] || !prefix_v[l])) return PI0X_EINVAL;
+  cudaStream_t s = (cudaStream_t)stream;
+  int st = ensure_workspace(h, B, P, num_steps);
+  if (st) return st;
+  const int H = c.horizon, A = c.action_dim, L = c.depth;
+  const size_t kv_elems = (size_t)B * P * kHeadDim;
+  CallPtrs cp;
+  memset(&cp, 0, sizeof(cp));
+  bool host_any = (P > 0 && !is_device_ptr(prefix_valid_mask)) || !is_device_ptr(state) ||
+                  !is_device_ptr(x1) || !is_device_ptr(x0);
+  for (int l = 0; l < L && !host_any && P > 0; ++l)
+    host_any = !is_device_ptr(prefix_k[l]) || !is_device_ptr(prefix_v[l]);
+  if (host_any) {
+    st = ensure_stage(h, B, P);
+    if (st) return st;
+  }
+  Workspace &ws = h->ws;
+  for (int l = 0; l < L; ++l) {
+    for (int kvi = 0; kvi < 2; ++kvi) {
+      const void *src = kvi ? prefix_v[l] : prefix_k[l];
+      const bf16 **dst = kvi ? &cp.prefix_v[l] : &cp.prefix_k[l];
+      if (P == 0) {
+        *dst = nullptr;
+      } else if (is_device_ptr(src)) {
+        *dst = (const bf16 *)src;
+      } else {
+        bf16 *stg = (kvi ? ws.st_v : ws.st_k) + (size_t)l * kv_elems;
+        CK(cudaMemcpyAsync(stg, src, kv_elems * 2, cudaMemcpyHostToDevice, s));
+        *dst = stg;
+      }
+    }
+  }
+  auto stage_in = [&](const void *src, void *stg, size_t bytes, const void **dst) -> int {
+    if (is_device_ptr(src)) {
+      *dst = src;
+    } else {
+      CK(cudaMemcpyAsync(stg, src, bytes, cudaMemcpyHostToDevice, s));
+      *dst = stg;
+    }
+    return PI0X_OK;
+  };
+  const void *tmp;
+  if (P > 0) {
+    if ((st = stage_in(prefix_valid_mask, ws.st_mask, (size_t)B * P, &tmp))) return st;
+    cp.mask = (const uint8_t *)tmp;
+  }
+  if ((st = stage_in(state, ws.st_state, 4 * (size_t)B * c.state_dim, &tmp))) return st;
+  cp.state = (const float *)tmp;
+  if ((st = stage_in(x1, ws.st_x, 4 * (size_t)B * H * A, &tmp))) return st;
+  cp.x1 = (const float *)tmp;
+  const bool x0_host = !is_device_ptr(x0);
+  cp.x0 = x0_host ? ws.st_x : x0;  // staged x1 is consumed before x0 is written
+  CK(cudaMemcpyAsync(h->d_ptrs, &cp, sizeof(cp), cudaMemcpyHostToDevice, s));
+  st = h->bf16 ? enqueue_loop<bf16>(h, B, P, num_steps, s) : enqueue_loop<float>(h, B, P, num_steps, s);
+  if (st) return st;
+  if (x0_host) CK(cudaMemcpyAsync(x0, ws.st_x, 4 * (size_t)B * H * A, cudaMemcpyDeviceToHost, s));
+  h->last_stream = s;
+  return PI0X_OK;
+}
+
+int pi0x_sync_status(pi0x_handle *h) {
+  if (!h) return PI0X_EINVAL;
+  CK(cudaStreamSynchronize(h->last_stream));
+  unsigned err = 0;
+  CK(cudaMemcpy(&err, h->d_err, sizeof(err), cudaMemcpyDeviceToHost));
+  if (err) {
+    cudaMemset(h->d_err, 0, sizeof(unsigned));
+    g_last_error = "device error word 0x" + std::to_string(err);
+    return (err & (kErrTimeoutProducer | kErrTimeoutMma | kErrTimeoutEpilogue)) ? PI0X_ETIMEOUT : PI0X_EDEVICE;
+  }
+  return PI0X_OK;
+}
+
+long pi0x_launch_count(const pi0x_handle *h, int B, int P, int num_steps) {
+  if (!h || B < 1 || P < 0 || num_steps < 1) return -1;
+  const long per_layer = 9, L = h->cfg.depth;
+  return 3 + 1 + (long)num_steps * (3 + L * per_layer + 1);
+}
+
+void pi0x_destroy(pi0x_handle *h) {
+  if (!h) return;
+  if (h->last_stream) cudaStreamSynchronize(h->last_stream);
+  cudaDeviceSynchronize();
+  free_workspace(h->ws);
+  if (h->ws.stage.base) cudaFree(h->ws.stage.base);
+  if (h->warena.base) cudaFree(h->warena.base);
+  if (h->d_ptrs) cudaFree(h->d_ptrs);
+  if (h->d_err) cudaFree(h->d_err);
+  delete h;
+}
+
+}  // extern "C"
