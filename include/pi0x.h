@@ -135,6 +135,27 @@ int pi0x_sync_status(pi0x_handle *h);
  * kernels only, not memory copies), or -1 for invalid arguments. */
 long pi0x_launch_count(const pi0x_handle *h, int B, int P, int num_steps);
 
+/* ---- per-kernel-class device timing ------------------------------------------
+ * With profiling on, the next pi0x_sample calls record a CUDA event pair around
+ * every kernel launch (inside the captured graph, so kernels still run back to
+ * back); pi0x_profile_read then reports, for the most recent such call, how many
+ * kernels of a class ran and their summed device time in milliseconds.  It
+ * synchronizes the handle's last stream.  Profiled calls use a separate graph, so
+ * turning profiling on does not change the unprofiled path. */
+enum {
+  PI0X_K_PREP = 0,   /* mask compaction, time-MLP half, x_1 copy (once per call) */
+  PI0X_K_EMBED = 1,  /* state and action input projections */
+  PI0X_K_GEMM = 2,   /* every Linear of the expert and of the action-time MLP */
+  PI0X_K_NORM = 3,   /* RMSNorm */
+  PI0X_K_ROPE = 4,   /* RoPE of q/k, v copy */
+  PI0X_K_ATTN = 5,   /* masked MQA attention */
+  PI0X_K_GEGLU = 6,  /* gated GELU(tanh) */
+  PI0X_K_FINAL = 7,  /* final norm + action out-proj + Euler update */
+  PI0X_K_COUNT = 8
+};
+int pi0x_profile_enable(pi0x_handle *h, int on);
+int pi0x_profile_read(pi0x_handle *h, int kclass, long *launches, double *total_ms);
+
 /* Human-readable name of a status code; never NULL. */
 const char *pi0x_status_string(int status);
 

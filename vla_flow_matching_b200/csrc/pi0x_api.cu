@@ -127,6 +127,17 @@ struct pi0x_handle {
   CallPtrs *d_ptrs = nullptr;
   unsigned *d_err = nullptr;
   cudaStream_t last_stream = nullptr;
+  cudaStream_t cap = nullptr;   // capture stream (graphs are launched on the caller's stream)
+  struct Graph {
+    int B, P, N, prof;
+    cudaGraphExec_t exec;
+    std::vector<std::pair<int, int>> marks;  // profiling graphs: (class, start event)
+  };
+  std::vector<Graph> graphs;
+  // per-kernel-class event timing (pi0x_profile_*)
+  bool prof_on = false;
+  std::vector<cudaEvent_t> prof_ev;
+  std::vector<std::pair<int, int>> prof_marks;  // marks of the last profiled call
 };
 
 namespace {
@@ -206,6 +217,11 @@ int build_weight_maps(pi0x_handle *h) {
   return PI0X_OK;
 }
 
+void drop_graphs(pi0x_handle *h) {
+  for (auto &g : h->graphs) cudaGraphExecDestroy(g.exec);
+  h->graphs.clear();
+}
+
 void free_workspace(Workspace &ws) {
   if (ws.arena.base) cudaFree(ws.arena.base);
   ws.arena = Arena();
@@ -217,6 +233,7 @@ int ensure_workspace(pi0x_handle *h, int B, int P, int N) {
   if (ws.arena.base && B <= ws.B && P <= ws.P && N <= ws.N) return PI0X_OK;
   const int nB = B > ws.B ? B : ws.B, nP = P > ws.P ? P : ws.P, nN = N > ws.N ? N : ws.N;
   if (h->last_stream) cudaStreamSynchronize(h->last_stream);
+  drop_graphs(h);
   free_workspace(ws);
   const int H = h->cfg.horizon, A = h->cfg.action_dim, L = h->cfg.depth;
   const size_t R = (size_t)nB + (size_t)nB * H;
@@ -308,9 +325,41 @@ bool is_device_ptr(const void *p) {
   return a.type == cudaMemoryTypeDevice || a.type == cudaMemoryTypeManaged;
 }
 
+// ---- per-kernel-class timing marks (recorded into the profiling graph) ---------
+struct Marker {
+  pi0x_handle *h;
+  cudaStream_t s;
+  int cls = 0;
+  void begin(int c) {
+    if (!h->prof_on) return;
+    cls = c;
+    const size_t i = h->prof_marks.size() * 2;
+    while (h->prof_ev.size() < i + 2) {
+      cudaEvent_t e;
+      cudaEventCreate(&e);
+      h->prof_ev.push_back(e);
+    }
+    cudaEventRecord(h->prof_ev[i], s);
+  }
+  void end() {
+    if (!h->prof_on) return;
+    const size_t i = h->prof_marks.size() * 2;
+    cudaEventRecord(h->prof_ev[i + 1], s);
+    h->prof_marks.push_back({cls, (int)i});
+  }
+};
+#define RUN(cls, ...) \
+  do {                \
+    mk.begin(cls);    \
+    __VA_ARGS__;      \
+    mk.end();         \
+  } while (0)
+
 // ---- the Euler loop -------------------------------------------------------------
 template <typename T>
 int enqueue_loop(pi0x_handle *h, int B, int P, int N, cudaStream_t s) {
+  Marker mk{h, s};
+  if (h->prof_on) h->prof_marks.clear();
   Workspace &ws = h->ws;
   const pi0x_config &c = h->cfg;
   const int H = c.horizon, A = c.action_dim, L = c.depth;
@@ -322,78 +371,109 @@ int enqueue_loop(pi0x_handle *h, int B, int P, int N, cudaStream_t s) {
   T *aemb = (T *)ws.a_emb, *uemb = (T *)ws.u_emb;
   const size_t kv_stride = (size_t)R * kHeadDim;
 
-  launch_prep_mask(h->d_ptrs, B, P, ws.nvalid, ws.vidx, s);
-  launch_time_vec<T>((const T *)h->tin_t, h->tin_b, N, ws.tvec, s);
-  launch_copy_x1(h->d_ptrs, BH * A, ws.xw, s);
+  RUN(PI0X_K_PREP, launch_prep_mask(h->d_ptrs, B, P, ws.nvalid, ws.vidx, s));
+  RUN(PI0X_K_PREP, launch_time_vec<T>((const T *)h->tin_t, h->tin_b, N, ws.tvec, s));
+  RUN(PI0X_K_PREP, launch_copy_x1(h->d_ptrs, BH * A, ws.xw, s));
 
   for (int k = 0; k < N; ++k) {
     const int step0 = (k == 0);
     const int row0 = step0 ? 0 : B;
     const int M = R - row0;
-    if (step0) launch_state_embed<T>(h->d_ptrs, (const T *)h->state_w, h->state_b, B, c.state_dim, ws.h, s);
-    launch_action_in<T, T>(ws.xw, (const T *)h->ain_w, h->ain_b, BH, A, aemb, s);
+    if (step0)
+      RUN(PI0X_K_EMBED, launch_state_embed<T>(h->d_ptrs, (const T *)h->state_w, h->state_b, B, c.state_dim, ws.h, s));
+    RUN(PI0X_K_EMBED, launch_action_in<T, T>(ws.xw, (const T *)h->ain_w, h->ain_b, BH, A, aemb, s));
     GemmOut o_u{uemb, kWidth, 0, ws.tvec + (size_t)k * kWidth};
     GemmOut o_h{ws.h, kWidth, B, h->tout_b};
     if (tc) {
       TcGemm gt = h->g_tin;
       gt.tmA = ws.m_aemb;
-      launch_gemm_tc<bf16>(gt, 0, BH, EPI_VEC_SILU, o_u, h->d_err, s);
+      RUN(PI0X_K_GEMM, launch_gemm_tc<bf16>(gt, 0, BH, EPI_VEC_SILU, o_u, h->d_err, s));
       TcGemm go = h->g_tout;
       go.tmA = ws.m_uemb;
-      launch_gemm_tc<bf16>(go, 0, BH, EPI_BIAS_F32, o_h, h->d_err, s);
+      RUN(PI0X_K_GEMM, launch_gemm_tc<bf16>(go, 0, BH, EPI_BIAS_F32, o_h, h->d_err, s));
     } else {
-      launch_gemm_simt<float>((const float *)aemb, kWidth, (const float *)h->tin_a, kWidth, BH, kWidth, kWidth,
-                              EPI_VEC_SILU, o_u, s);
-      launch_gemm_simt<float>((const float *)uemb, kWidth, (const float *)h->tout_w, kWidth, BH, kWidth, kWidth,
-                              EPI_BIAS_F32, o_h, s);
+      RUN(PI0X_K_GEMM, launch_gemm_simt<float>((const float *)aemb, kWidth, (const float *)h->tin_a, kWidth, BH, kWidth, kWidth,
+                              EPI_VEC_SILU, o_u, s));
+      RUN(PI0X_K_GEMM, launch_gemm_simt<float>((const float *)uemb, kWidth, (const float *)h->tout_w, kWidth, BH, kWidth, kWidth,
+                              EPI_BIAS_F32, o_h, s));
     }
     for (int l = 0; l < L; ++l) {
       const LayerW &lw = h->layer[l];
       T *ks = (T *)ws.ks + (size_t)l * kv_stride, *vs = (T *)ws.vs + (size_t)l * kv_stride;
-      launch_rmsnorm<T>(ws.h, row0, M, lw.in_norm, xn, s);
+      RUN(PI0X_K_NORM, launch_rmsnorm<T>(ws.h, row0, M, lw.in_norm, xn, s));
       GemmOut o_raw{ws.raw, kQkvDim, row0, nullptr};
       if (tc) {
         TcGemm gq = h->g_qkv[l];
         gq.tmA = ws.m_xn;
-        launch_gemm_tc<bf16>(gq, row0, M, EPI_STORE_F32, o_raw, h->d_err, s);
+        RUN(PI0X_K_GEMM, launch_gemm_tc<bf16>(gq, row0, M, EPI_STORE_F32, o_raw, h->d_err, s));
       } else {
-        launch_gemm_simt<float>((const float *)xn + (size_t)row0 * kWidth, kWidth, (const float *)lw.qkv, kWidth,
-                                M, kQkvDim, kWidth, EPI_STORE_F32, o_raw, s);
+        RUN(PI0X_K_GEMM, launch_gemm_simt<float>((const float *)xn + (size_t)row0 * kWidth, kWidth, (const float *)lw.qkv, kWidth,
+                                M, kQkvDim, kWidth, EPI_STORE_F32, o_raw, s));
       }
-      launch_rope_qkv<T>(ws.raw, row0, M, g, ws.nvalid, h->inv_freq, q, ks, vs, s);
-      launch_attention<T>(q, ks, vs, h->d_ptrs, l, ws.nvalid, ws.vidx, g, step0, att, s);
+      RUN(PI0X_K_ROPE, launch_rope_qkv<T>(ws.raw, row0, M, g, ws.nvalid, h->inv_freq, q, ks, vs, s));
+      RUN(PI0X_K_ATTN, launch_attention<T>(q, ks, vs, h->d_ptrs, l, ws.nvalid, ws.vidx, g, step0, att, s));
       GemmOut o_res{ws.h, kWidth, row0, nullptr};
       if (tc) {
         TcGemm gO = h->g_o[l];
         gO.tmA = ws.m_att;
-        launch_gemm_tc<bf16>(gO, row0, M, EPI_RESID_F32, o_res, h->d_err, s);
+        RUN(PI0X_K_GEMM, launch_gemm_tc<bf16>(gO, row0, M, EPI_RESID_F32, o_res, h->d_err, s));
       } else {
-        launch_gemm_simt<float>((const float *)att + (size_t)row0 * kQDim, kQDim, (const float *)lw.o, kQDim, M,
-                                kWidth, kQDim, EPI_RESID_F32, o_res, s);
+        RUN(PI0X_K_GEMM, launch_gemm_simt<float>((const float *)att + (size_t)row0 * kQDim, kQDim, (const float *)lw.o, kQDim, M,
+                                kWidth, kQDim, EPI_RESID_F32, o_res, s));
       }
-      launch_rmsnorm<T>(ws.h, row0, M, lw.post_norm, xn, s);
+      RUN(PI0X_K_NORM, launch_rmsnorm<T>(ws.h, row0, M, lw.post_norm, xn, s));
       GemmOut o_gu{ws.raw, 2 * kMlp, row0, nullptr};
       if (tc) {
         TcGemm gg = h->g_gu[l];
         gg.tmA = ws.m_xn;
-        launch_gemm_tc<bf16>(gg, row0, M, EPI_STORE_F32, o_gu, h->d_err, s);
+        RUN(PI0X_K_GEMM, launch_gemm_tc<bf16>(gg, row0, M, EPI_STORE_F32, o_gu, h->d_err, s));
       } else {
-        launch_gemm_simt<float>((const float *)xn + (size_t)row0 * kWidth, kWidth, (const float *)lw.gu, kWidth, M,
-                                2 * kMlp, kWidth, EPI_STORE_F32, o_gu, s);
+        RUN(PI0X_K_GEMM, launch_gemm_simt<float>((const float *)xn + (size_t)row0 * kWidth, kWidth, (const float *)lw.gu, kWidth, M,
+                                2 * kMlp, kWidth, EPI_STORE_F32, o_gu, s));
       }
-      launch_geglu<T>(ws.raw, row0, M, act, s);
+      RUN(PI0X_K_GEGLU, launch_geglu<T>(ws.raw, row0, M, act, s));
       if (tc) {
         TcGemm gd = h->g_down[l];
         gd.tmA = ws.m_act;
-        launch_gemm_tc<bf16>(gd, row0, M, EPI_RESID_F32, o_res, h->d_err, s);
+        RUN(PI0X_K_GEMM, launch_gemm_tc<bf16>(gd, row0, M, EPI_RESID_F32, o_res, h->d_err, s));
       } else {
-        launch_gemm_simt<float>((const float *)act + (size_t)row0 * kMlp, kMlp, (const float *)lw.down, kMlp, M,
-                                kWidth, kMlp, EPI_RESID_F32, o_res, s);
+        RUN(PI0X_K_GEMM, launch_gemm_simt<float>((const float *)act + (size_t)row0 * kMlp, kMlp, (const float *)lw.down, kMlp, M,
+                                kWidth, kMlp, EPI_RESID_F32, o_res, s));
       }
     }
-    launch_final_euler(ws.h, g, h->fnorm, h->aout_w, h->aout_b, dt, ws.xw, h->d_ptrs, k == N - 1, s);
+    RUN(PI0X_K_FINAL, launch_final_euler(ws.h, g, h->fnorm, h->aout_w, h->aout_b, dt, ws.xw, h->d_ptrs, k == N - 1, s));
   }
   CK(cudaGetLastError());
+  return PI0X_OK;
+}
+
+// The whole call (all Euler steps) as one CUDA graph per (B, P, N, profiling),
+// captured on the handle's own stream and launched on the caller's.  Every
+// caller-owned pointer reaches the kernels through the device table d_ptrs, so a
+// graph stays valid across calls; graphs are dropped when the workspace moves.
+int get_graph(pi0x_handle *h, int B, int P, int N, cudaGraphExec_t *out) {
+  const int prof = h->prof_on ? 1 : 0;
+  for (auto &g : h->graphs)
+    if (g.B == B && g.P == P && g.N == N && g.prof == prof) {
+      *out = g.exec;
+      if (prof) h->prof_marks = g.marks;
+      return PI0X_OK;
+    }
+  cudaGraph_t graph = nullptr;
+  CK(cudaStreamBeginCapture(h->cap, cudaStreamCaptureModeThreadLocal));
+  int st = h->bf16 ? enqueue_loop<bf16>(h, B, P, N, h->cap) : enqueue_loop<float>(h, B, P, N, h->cap);
+  cudaError_t e = cudaStreamEndCapture(h->cap, &graph);
+  if (st) {
+    if (graph) cudaGraphDestroy(graph);
+    return st;
+  }
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamEndCapture");
+  cudaGraphExec_t exec = nullptr;
+  e = cudaGraphInstantiate(&exec, graph, 0);
+  cudaGraphDestroy(graph);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGraphInstantiate");
+  h->graphs.push_back({B, P, N, prof, exec, prof ? h->prof_marks : std::vector<std::pair<int, int>>()});
+  *out = exec;
   return PI0X_OK;
 }
 
@@ -558,6 +638,7 @@ int pi0x_create(const pi0x_config *cfg, const pi0x_weights *w, pi0x_handle **out
     if (st) return fail(st);
   }
   e = cudaMalloc(&h->d_ptrs, sizeof(CallPtrs));
+  if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&h->cap, cudaStreamNonBlocking);
   if (e == cudaSuccess) e = cudaMalloc(&h->d_err, sizeof(unsigned));
   if (e == cudaSuccess) e = cudaMemset(h->d_err, 0, sizeof(unsigned));
   if (e != cudaSuccess) return fail(cuda_fail(e, "cudaMalloc(handle)"));
@@ -626,8 +707,10 @@ int pi0x_sample(pi0x_handle *h, const void *const *prefix_k, const void *const *
   const bool x0_host = !is_device_ptr(x0);
   cp.x0 = x0_host ? ws.st_x : x0;  // staged x1 is consumed before x0 is written
   CK(cudaMemcpyAsync(h->d_ptrs, &cp, sizeof(cp), cudaMemcpyHostToDevice, s));
-  st = h->bf16 ? enqueue_loop<bf16>(h, B, P, num_steps, s) : enqueue_loop<float>(h, B, P, num_steps, s);
+  cudaGraphExec_t exec = nullptr;
+  st = get_graph(h, B, P, num_steps, &exec);
   if (st) return st;
+  CK(cudaGraphLaunch(exec, s));
   if (x0_host) CK(cudaMemcpyAsync(x0, ws.st_x, 4 * (size_t)B * H * A, cudaMemcpyDeviceToHost, s));
   h->last_stream = s;
   return PI0X_OK;
@@ -646,6 +729,29 @@ int pi0x_sync_status(pi0x_handle *h) {
   return PI0X_OK;
 }
 
+int pi0x_profile_enable(pi0x_handle *h, int on) {
+  if (!h) return PI0X_EINVAL;
+  h->prof_on = on != 0;
+  return PI0X_OK;
+}
+
+int pi0x_profile_read(pi0x_handle *h, int kclass, long *launches, double *total_ms) {
+  if (!h || kclass < 0 || kclass >= PI0X_K_COUNT || !launches || !total_ms) return PI0X_EINVAL;
+  if (h->last_stream) CK(cudaStreamSynchronize(h->last_stream));
+  long n = 0;
+  double ms = 0.0;
+  for (auto &m : h->prof_marks) {
+    if (m.first != kclass) continue;
+    float t = 0.f;
+    CK(cudaEventElapsedTime(&t, h->prof_ev[m.second], h->prof_ev[m.second + 1]));
+    ++n;
+    ms += t;
+  }
+  *launches = n;
+  *total_ms = ms;
+  return PI0X_OK;
+}
+
 long pi0x_launch_count(const pi0x_handle *h, int B, int P, int num_steps) {
   if (!h || B < 1 || P < 0 || num_steps < 1) return -1;
   const long per_layer = 9, L = h->cfg.depth;
@@ -656,6 +762,9 @@ void pi0x_destroy(pi0x_handle *h) {
   if (!h) return;
   if (h->last_stream) cudaStreamSynchronize(h->last_stream);
   cudaDeviceSynchronize();
+  drop_graphs(h);
+  for (cudaEvent_t ev : h->prof_ev) cudaEventDestroy(ev);
+  if (h->cap) cudaStreamDestroy(h->cap);
   free_workspace(h->ws);
   if (h->ws.stage.base) cudaFree(h->ws.stage.base);
   if (h->warena.base) cudaFree(h->warena.base);

@@ -21,7 +21,10 @@ PI0X_DTYPE_BF16, PI0X_DTYPE_F32 = 0, 1
 #: Every symbol include/pi0x.h declares.
 EXPORTED = ["pi0x_create", "pi0x_sample", "pi0x_sync_status", "pi0x_launch_count",
             "pi0x_status_string", "pi0x_last_error", "pi0x_destroy", "pi0x_version",
-            "pi0x_debug_gemm_bf16"]
+            "pi0x_debug_gemm_bf16", "pi0x_profile_enable", "pi0x_profile_read"]
+
+#: kernel classes of pi0x_profile_read
+K_CLASSES = ["prep", "embed", "gemm", "norm", "rope", "attn", "geglu", "final"]
 
 
 class Pi0xError(RuntimeError):
@@ -90,6 +93,11 @@ def load() -> ctypes.CDLL:
     lib.pi0x_debug_gemm_bf16.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_int,
                                          ctypes.c_int, ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p]
     lib.pi0x_debug_gemm_bf16.restype = ctypes.c_int
+    lib.pi0x_profile_enable.argtypes = [ctypes.c_void_p, ctypes.c_int]
+    lib.pi0x_profile_enable.restype = ctypes.c_int
+    lib.pi0x_profile_read.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.POINTER(ctypes.c_long),
+                                      ctypes.POINTER(ctypes.c_double)]
+    lib.pi0x_profile_read.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -183,6 +191,19 @@ class Sampler:
                                      int(num_steps), _ptr(x0), ctypes.c_void_p(stream)),
                "pi0x_sample")
         return x0
+
+    def profile(self, on: bool = True):
+        _check(self._lib.pi0x_profile_enable(self._h, int(on)), "pi0x_profile_enable")
+
+    def profile_read(self) -> dict:
+        """{class: (launches, total_ms)} of the most recent profiled call."""
+        out = {}
+        for i, name in enumerate(K_CLASSES):
+            n, ms = ctypes.c_long(), ctypes.c_double()
+            _check(self._lib.pi0x_profile_read(self._h, i, ctypes.byref(n), ctypes.byref(ms)),
+                   "pi0x_profile_read")
+            out[name] = (int(n.value), float(ms.value))
+        return out
 
     def sync(self):
         _check(self._lib.pi0x_sync_status(self._h), "pi0x_sync_status")
