@@ -266,6 +266,9 @@ def main():
         ms = float(t.item())
     ms_per = ms / args.steps
     value = world * B * args.steps / (ms / 1000.0)
+    if rank == 0:
+        print(f"[bench] {wl.name} {args.precision}: {1000 * ms_per:.1f} us per call, "
+              f"{value:.1f} {UNIT}", file=sys.stderr, flush=True)
 
     # ---- end to end through the public call with host buffers ----
     pin = lambda a: torch.from_numpy(np.ascontiguousarray(a)).pin_memory()

@@ -339,12 +339,12 @@ struct Marker {
       cudaEventCreate(&e);
       h->prof_ev.push_back(e);
     }
-    cudaEventRecord(h->prof_ev[i], s);
+    cudaEventRecordWithFlags(h->prof_ev[i], s, cudaEventRecordExternal);
   }
   void end() {
     if (!h->prof_on) return;
     const size_t i = h->prof_marks.size() * 2;
-    cudaEventRecord(h->prof_ev[i + 1], s);
+    cudaEventRecordWithFlags(h->prof_ev[i + 1], s, cudaEventRecordExternal);
     h->prof_marks.push_back({cls, (int)i});
   }
 };
