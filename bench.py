@@ -307,6 +307,10 @@ def main():
             a[1] += t
     sampler.profile(False)
     sampler.sync()
+    if rank == 0:
+        print("[bench] per-call kernel ms (launches): " + ", ".join(
+            f"{k}={v[1] / max(1, args.profile_steps):.3f} ({v[0] // max(1, args.profile_steps)})"
+            for k, v in acc.items()), file=sys.stderr, flush=True)
 
     roofline = None
     kernel_ms = {}

@@ -271,6 +271,13 @@ void launch_copy_x1(const CallPtrs *cp, int n, float *x, cudaStream_t s) {
   k_copy_x1<<<(n + 255) / 256 < 1024 ? (n + 255) / 256 : 1024, 256, 0, s>>>(cp, n, x);
 }
 
+// Holds the stream for `ns` nanoseconds of wall time (bounded by construction).
+__global__ void k_delay(unsigned long long ns) {
+  const unsigned long long t0 = globaltimer_ns();
+  while (globaltimer_ns() - t0 < ns) __nanosleep(2000);
+}
+void launch_delay_ns(unsigned long long ns, cudaStream_t s) { k_delay<<<1, 1, 0, s>>>(ns); }
+
 // ---- explicit instantiations ----
 template void launch_time_vec<float>(const float *, const float *, int, float *, cudaStream_t);
 template void launch_time_vec<bf16>(const bf16 *, const float *, int, float *, cudaStream_t);

@@ -67,6 +67,7 @@ void launch_geglu(const float *raw, int row0, int rows, T *act, cudaStream_t s);
 void launch_final_euler(const float *h, const Geo &g, const float *gain, const float *w_out, const float *b_out,
                         float dt, float *x, const CallPtrs *cp, int last, cudaStream_t s);
 void launch_copy_x1(const CallPtrs *cp, int n, float *x, cudaStream_t s);
+void launch_delay_ns(unsigned long long ns, cudaStream_t s);
 
 // ---- attention (k_attn.cu) ----
 template <typename T>
