@@ -126,7 +126,8 @@ struct pi0x_handle {
   Workspace ws;
   CallPtrs *d_ptrs = nullptr;
   unsigned *d_err = nullptr;
-  cudaStream_t last_stream = nullptr;
+  cudaStream_t last_stream = nullptr;  // stream of the last call (NULL = legacy default)
+  bool called = false;
   cudaStream_t cap = nullptr;   // capture stream (graphs are launched on the caller's stream)
   struct Graph {
     int B, P, N, prof;
@@ -232,7 +233,7 @@ int ensure_workspace(pi0x_handle *h, int B, int P, int N) {
   Workspace &ws = h->ws;
   if (ws.arena.base && B <= ws.B && P <= ws.P && N <= ws.N) return PI0X_OK;
   const int nB = B > ws.B ? B : ws.B, nP = P > ws.P ? P : ws.P, nN = N > ws.N ? N : ws.N;
-  if (h->last_stream) cudaStreamSynchronize(h->last_stream);
+  if (h->called) cudaStreamSynchronize(h->last_stream);
   drop_graphs(h);
   free_workspace(ws);
   const int H = h->cfg.horizon, A = h->cfg.action_dim, L = h->cfg.depth;
@@ -295,7 +296,7 @@ int ensure_workspace(pi0x_handle *h, int B, int P, int N) {
 int ensure_stage(pi0x_handle *h, int B, int P) {
   Workspace &ws = h->ws;
   if (ws.stage.base && (size_t)B <= ws.stage_B && (size_t)P <= ws.stage_P) return PI0X_OK;
-  if (h->last_stream) cudaStreamSynchronize(h->last_stream);
+  if (h->called) cudaStreamSynchronize(h->last_stream);
   if (ws.stage.base) cudaFree(ws.stage.base);
   ws.stage = Arena();
   const int L = h->cfg.depth, H = h->cfg.horizon, A = h->cfg.action_dim, S = h->cfg.state_dim;
@@ -722,6 +723,7 @@ int pi0x_sample(pi0x_handle *h, const void *const *prefix_k, const void *const *
   }
   if (x0_host) CK(cudaMemcpyAsync(x0, ws.st_x, 4 * (size_t)B * H * A, cudaMemcpyDeviceToHost, s));
   h->last_stream = s;
+  h->called = true;
   return PI0X_OK;
 }
 
@@ -746,7 +748,7 @@ int pi0x_profile_enable(pi0x_handle *h, int on) {
 
 int pi0x_profile_read(pi0x_handle *h, int kclass, long *launches, double *total_ms) {
   if (!h || kclass < 0 || kclass >= PI0X_K_COUNT || !launches || !total_ms) return PI0X_EINVAL;
-  if (h->last_stream) CK(cudaStreamSynchronize(h->last_stream));
+  if (h->called) CK(cudaStreamSynchronize(h->last_stream));
   long n = 0;
   double ms = 0.0;
   for (auto &m : h->prof_marks) {
@@ -769,7 +771,7 @@ long pi0x_launch_count(const pi0x_handle *h, int B, int P, int num_steps) {
 
 void pi0x_destroy(pi0x_handle *h) {
   if (!h) return;
-  if (h->last_stream) cudaStreamSynchronize(h->last_stream);
+  if (h->called) cudaStreamSynchronize(h->last_stream);
   cudaDeviceSynchronize();
   drop_graphs(h);
   for (cudaEvent_t ev : h->prof_ev) cudaEventDestroy(ev);
