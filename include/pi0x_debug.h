@@ -19,6 +19,20 @@ extern "C" {
  * a bounded device wait gave up. */
 int pi0x_debug_gemm_bf16(const void *A, const void *Bw, int M, int N, int K, float *D, int bn, void *stream);
 
+/* One layer of the suffix attention (the `_attend` step of the pi0 page) for B
+ * samples with horizon H and prefix length P, all device pointers, bf16 unless
+ * noted, activation rows laid out as in the sampler (state rows 0..B-1, then
+ * action rows B + b*H + j-1):
+ *   q (R, 2048) with R = B + B*H (post-RoPE, 8 heads x 256), ks/vs (R, 256)
+ *   suffix keys/values, prefix_k/prefix_v (B, P, 256), mask (B, P) uint8.
+ * step0 != 0 includes the state queries (first Euler step).  impl 0 = SIMT
+ * kernel, 1 = tcgen05 kernel (split-KV as the sampler chooses), 2 = tcgen05
+ * without split-KV.  Writes out (R, 2048); rows not queried are left as they
+ * are.  Synchronous (allocates its scratch with cudaMalloc). */
+int pi0x_debug_attention(const void *q, const void *ks, const void *vs, const void *prefix_k,
+                         const void *prefix_v, const void *mask, int B, int H, int P, int step0, int impl,
+                         void *out, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

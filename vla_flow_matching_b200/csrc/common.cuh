@@ -169,6 +169,35 @@ __device__ __forceinline__ uint64_t smem_desc_k_sw128(uint32_t tile_base, uint32
          (2ull << 61) /* 128-byte swizzle */;
 }
 
+// Descriptor for an MN-major operand in 128-byte-swizzled 64-element spans: each
+// 128 B row holds 64 consecutive MN elements of one K index (rows swizzled by
+// row % 8), 8 K-rows form a 1024 B atom.  `lbo` = bytes between 64-element MN
+// spans, `sbo` = bytes between 8-row K groups.
+__device__ __forceinline__ uint64_t smem_desc_mn_sw128(uint32_t start, uint32_t lbo, uint32_t sbo) {
+  return (uint64_t)((start >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+         ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
+}
+
+// ---- cp.async (16-byte, L2-only) and proxy fences ------------------------------
+// Copies 16 bytes, or writes 16 zero bytes when `valid` is false.
+__device__ __forceinline__ void cp_async16(uint32_t smem_dst, const void *gsrc, bool valid) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_dst), "l"(gsrc),
+               "r"(valid ? 16 : 0)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+// Make this thread's generic-proxy shared-memory writes visible to the async proxy
+// (tcgen05.mma operand reads).
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+// Byte offset of 16-byte chunk `cc` (0..7) of row `r` in a 128-byte-swizzled tile.
+__device__ __forceinline__ uint32_t sw128_off(uint32_t r, uint32_t cc) { return r * 128u + ((cc ^ (r & 7u)) << 4); }
+
 // Instruction descriptor: kind::f16, A = B = bf16 (K-major), D = fp32, M x N.
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
   return (1u << 4)            // D format fp32

@@ -1,0 +1,373 @@
+// Masked MQA attention on the tcgen05 tensor cores (bf16 mode).
+//
+// Computes, per sample and per query head, softmax(q . K^T / sqrt(256) + mask) . V
+// over [valid prefix keys ; state key ; action keys] (`_attend` with the block mask
+// of `denoise_step` on the vllm-omni pi0 page).  The 8 query heads share the one
+// KV head, so a CTA takes 128 query rows (token-major: row = token*8 + head) of
+// one sample against the sample's key list, in blocks of 64 keys.
+//
+// Keys are gathered by index with cp.async (16 B per thread) into 128-byte-
+// swizzled shared memory, so masked prefix positions are never read; the page adds
+// -2.38e38 to their logits, whose exp is exactly 0 in fp32.
+//
+// Softmax in two passes over the key blocks: pass 1 forms the exact row max m and
+// sum l (S = Q K^T in TMEM, read back by the thread owning the row); pass 2
+// recomputes S and writes P = exp(s - m) / l rounded to bf16 (the page casts the
+// fp32 probabilities to the query dtype before P.V) and accumulates O += P V in
+// TMEM.  O therefore never needs rescaling.  With split-KV (small batches) every
+// split normalises by its own (m, l) and k_attn_combine merges the splits.
+#include <math.h>
+
+#include "common.cuh"
+#include "kernels.cuh"
+
+namespace pi0x {
+
+namespace {
+constexpr int kRowsPerCta = 128;
+constexpr int kKeyBlock = 64;
+constexpr uint32_t kQBytes = 128 * 512;       // 4 sub-tiles of [128 rows x 64 dims]
+constexpr uint32_t kKVBytes = 64 * 512;       // 4 sub-tiles of [64 keys x 64 dims]
+constexpr uint32_t kPBytes = 128 * 128;       // [128 rows x 64 keys]
+constexpr uint32_t kSmemQ = 0;
+constexpr uint32_t kSmemK0 = kSmemQ + kQBytes;
+constexpr uint32_t kSmemV0 = kSmemK0 + 2 * kKVBytes;
+constexpr uint32_t kSmemP = kSmemV0 + 2 * kKVBytes;
+constexpr uint32_t kSmemBar = kSmemP + kPBytes;
+constexpr uint32_t kSmemTotal = kSmemBar + 64 + 1024;  // + alignment slack
+constexpr uint32_t kTmemCols = 512;   // S at column 0 (64 cols), O at column 256 (256 cols)
+constexpr uint32_t kTmemO = 256;
+constexpr float kLog2e = 1.4426950408889634f;
+}  // namespace
+
+// Source row (256 bf16) of key `kk` of sample b: valid prefix positions first, then
+// the state key, then the action keys.
+__device__ __forceinline__ const bf16 *key_row(int kk, int nv, int b, const Geo &g, const bf16 *pref,
+                                                const int *vi, const bf16 *suf) {
+  if (kk < nv) return pref + ((size_t)b * g.P + vi[kk]) * kHeadDim;
+  const int row = (kk == nv) ? b : g.B + b * g.H + (kk - nv - 1);
+  return suf + (size_t)row * kHeadDim;
+}
+
+__global__ void __launch_bounds__(128, 1)
+    k_attn_tc(const bf16 *q, const bf16 *ks, const bf16 *vs, const CallPtrs *cp, int layer, const int *nvalid,
+              const int *vidx, Geo g, int step0, int blocks_per_split, bf16 *out, float *part_o, float *part_ml,
+              unsigned *err) {
+  if (*(volatile unsigned *)err != 0) return;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  uint64_t *bar_s = reinterpret_cast<uint64_t *>(smem + kSmemBar);
+  uint64_t *bar_o = bar_s + 1;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar_s + 2);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int b = blockIdx.z, split = blockIdx.y, nsplit = gridDim.y;
+  const int Tq = step0 ? g.H + 1 : g.H;
+  const int nrows = kHeads * Tq;
+  const int row0 = blockIdx.x * kRowsPerCta;
+  const int nv = nvalid[b];
+  const int nk = nv + 1 + g.H;
+  const int nblk_all = (nk + kKeyBlock - 1) / kKeyBlock;
+  const int blk0 = split * blocks_per_split;
+  const int blk1 = min(nblk_all, blk0 + blocks_per_split);
+  const int nb = blk1 > blk0 ? blk1 - blk0 : 0;
+
+  // this thread's query row
+  const int qi = row0 + tid;
+  const bool row_ok = qi < nrows;
+  const int jq = qi / kHeads, head = qi % kHeads;
+  int tok = 0;
+  if (row_ok) tok = step0 ? (jq == 0 ? b : g.B + b * g.H + jq - 1) : g.B + b * g.H + jq;
+  const bool state_q = step0 && jq == 0;
+  const int key_lim = state_q ? nv + 1 : nk;  // keys [0, key_lim) visible to this row
+
+  const bf16 *pref_k = cp->prefix_k[layer], *pref_v = cp->prefix_v[layer];
+  const int *vi = vidx + (size_t)b * g.P;
+
+  if (tid == 0) {
+    mbar_init(bar_s, 1);
+    mbar_init(bar_o, 1);
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+
+  // ---- Q tile: rows [row0, row0+128), 4 swizzled sub-tiles of 64 dims ----
+  {
+    // chunk c: row = c / 32, cr = c % 32 (sub-tile cr/8, chunk cr%8); a warp copies one 512 B row
+    for (int i = 0; i < 32; ++i) {
+      const int c = tid + 128 * i;
+      const int r = c >> 5, cr = c & 31;
+      const int qr = row0 + r;
+      const bool ok = qr < nrows;
+      int t = 0, hd = 0;
+      if (ok) {
+        const int j = qr / kHeads;
+        hd = qr % kHeads;
+        t = step0 ? (j == 0 ? b : g.B + b * g.H + j - 1) : g.B + b * g.H + j;
+      }
+      const bf16 *src = q + (size_t)t * kQDim + hd * kHeadDim + cr * 8;
+      cp_async16(sbase + kSmemQ + (cr >> 3) * (128 * 128) + sw128_off(r, cr & 7), src, ok);
+    }
+  }
+  auto load_block = [&](int blk, int buf, bool with_v) {
+    const uint32_t kb = sbase + kSmemK0 + buf * kKVBytes, vb = sbase + kSmemV0 + buf * kKVBytes;
+    for (int i = 0; i < 16; ++i) {
+      const int c = tid + 128 * i;
+      const int r = c >> 5, cr = c & 31;
+      const int kk = blk * kKeyBlock + r;
+      const bool ok = kk < nk;
+      const uint32_t off = (cr >> 3) * (64 * 128) + sw128_off(r, cr & 7);
+      const bf16 *ksrc = ok ? key_row(kk, nv, b, g, pref_k, vi, ks) + cr * 8 : ks;
+      cp_async16(kb + off, ksrc, ok);
+      if (with_v) {
+        const bf16 *vsrc = ok ? key_row(kk, nv, b, g, pref_v, vi, vs) + cr * 8 : vs;
+        cp_async16(vb + off, vsrc, ok);
+      }
+    }
+  };
+
+  const int nitems = 2 * nb;
+  if (nitems > 0) load_block(blk0, 0, false);
+  cp_async_commit();
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t t_lane = (uint32_t)(warp * 32) << 16;
+
+  constexpr uint32_t idesc_s = idesc_bf16_f32(128, kKeyBlock);
+  constexpr uint32_t idesc_o = idesc_bf16_f32(128, kHeadDim) | (1u << 16);  // B (V) MN-major
+  const float scale_l2 = 0.0625f * kLog2e;
+
+  float m = -INFINITY, l = 0.f, inv_l = 0.f;
+  uint32_t ph_s = 0, ph_o = 0;
+  bool ok_all = true;
+  for (int w = 0; w < nitems; ++w) {
+    const int pass = w / nb, j = w % nb, buf = w & 1;
+    const int blk = blk0 + j;
+    // The PV MMA of item w-1 reads V[buf^1] and P: wait for it before reusing them.
+    if (w >= 1 && (w - 1) / nb == 1) {
+      if (!mbar_wait(bar_o, ph_o, err, kErrTimeoutMma)) ok_all = false;
+      ph_o ^= 1u;
+    }
+    if (w + 1 < nitems) {
+      const int wn = w + 1;
+      load_block(blk0 + wn % nb, wn & 1, wn / nb == 1);
+    }
+    cp_async_commit();
+    cp_async_wait<1>();
+    fence_proxy_async_smem();
+    tc_fence_before();
+    ok_all = __syncthreads_and(ok_all);
+    tc_fence_after();
+    if (!ok_all) break;
+    if (tid == 0) {
+      const uint32_t kb = sbase + kSmemK0 + buf * kKVBytes;
+#pragma unroll
+      for (int s = 0; s < 4; ++s)
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          tc_mma_bf16(tmem, smem_desc_k_sw128(sbase + kSmemQ + s * (128 * 128), kk * 32),
+                      smem_desc_k_sw128(kb + s * (64 * 128), kk * 32), idesc_s, (s | kk) != 0);
+      tc_commit(bar_s);
+    }
+    __syncwarp();
+    if (!mbar_wait(bar_s, ph_s, err, kErrTimeoutEpilogue)) ok_all = false;
+    ph_s ^= 1u;
+    __syncwarp();
+    tc_fence_after();
+    float sv[64];
+    {
+      float t0[32], t1[32];
+      tmem_ld_32x32b_x32(tmem + t_lane + 0, t0);
+      tmem_ld_32x32b_x32(tmem + t_lane + 32, t1);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        sv[i] = t0[i];
+        sv[32 + i] = t1[i];
+      }
+    }
+    const int kbase = blk * kKeyBlock;
+    if (pass == 0) {
+      float bm = -INFINITY;
+#pragma unroll
+      for (int i = 0; i < 64; ++i) {
+        sv[i] = (kbase + i < key_lim) ? sv[i] * scale_l2 : -INFINITY;
+        bm = fmaxf(bm, sv[i]);
+      }
+      const float mn = fmaxf(m, bm);
+      if (mn != -INFINITY) {
+        float add = 0.f;
+#pragma unroll
+        for (int i = 0; i < 64; ++i) add += exp2f(sv[i] - mn);
+        l = l * exp2f(m - mn) + add;
+        m = mn;
+      }
+      if (j == nb - 1) inv_l = l > 0.f ? 1.0f / l : 0.f;
+    } else {
+      // P row -> bf16 -> swizzled [128 x 64] tile
+      uint8_t *prow = smem + kSmemP;
+#pragma unroll
+      for (int cc = 0; cc < 8; ++cc) {
+        uint32_t pk[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int i0 = cc * 8 + 2 * e;
+          const float p0 = (kbase + i0 < key_lim) ? exp2f(sv[i0] * scale_l2 - m) * inv_l : 0.f;
+          const float p1 = (kbase + i0 + 1 < key_lim) ? exp2f(sv[i0 + 1] * scale_l2 - m) * inv_l : 0.f;
+          const __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
+          pk[e] = *reinterpret_cast<const uint32_t *>(&h2);
+        }
+        *reinterpret_cast<uint4 *>(prow + sw128_off(tid, cc)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      ok_all = __syncthreads_and(ok_all);
+      tc_fence_after();
+      if (!ok_all) break;
+      if (tid == 0) {
+        const uint32_t vb = sbase + kSmemV0 + buf * kKVBytes;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          tc_mma_bf16(tmem + kTmemO, smem_desc_k_sw128(sbase + kSmemP, kk * 32),
+                      smem_desc_mn_sw128(vb + kk * 2048, 64 * 128, 1024), idesc_o, (j | kk) != 0);
+        tc_commit(bar_o);
+      }
+      __syncwarp();
+    }
+  }
+  // last PV MMA
+  if (nitems > 0 && ok_all) {
+    if (!mbar_wait(bar_o, ph_o, err, kErrTimeoutMma)) ok_all = false;
+    __syncwarp();
+  }
+  cp_async_wait<0>();
+  tc_fence_after();
+  const bool write = __syncthreads_and(ok_all);
+  if (write) {
+    if (nsplit == 1) {
+      bf16 *dst = out + (size_t)tok * kQDim + head * kHeadDim;
+      for (int c = 0; c < kHeadDim; c += 32) {
+        float v[32];
+        tmem_ld_32x32b_x32(tmem + t_lane + kTmemO + c, v);  // warp-collective: all lanes
+        if (row_ok) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const __nv_bfloat162 h2 = __floats2bfloat162_rn(v[2 * e], v[2 * e + 1]);
+            pk[e] = *reinterpret_cast<const uint32_t *>(&h2);
+          }
+          uint4 *d4 = reinterpret_cast<uint4 *>(dst + c);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) d4[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+        }
+      }
+    } else {
+      // split partials: O normalised by this split's l, plus (m, l) in log2 units
+      const size_t prow = ((size_t)b * nsplit + split) * (size_t)(gridDim.x * kRowsPerCta) + qi;
+      for (int c = 0; c < kHeadDim; c += 32) {
+        float v[32];
+        if (nb > 0) {
+          tmem_ld_32x32b_x32(tmem + t_lane + kTmemO + c, v);
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) v[e] = 0.f;
+        }
+        if (row_ok) {
+          float4 *d4 = reinterpret_cast<float4 *>(part_o + prow * kHeadDim + c);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) d4[e] = make_float4(v[4 * e], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]);
+        }
+      }
+      if (row_ok) {
+        part_ml[2 * prow] = m;
+        part_ml[2 * prow + 1] = l;
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// Merge split-KV partials: O = sum_s w_s O_s with w_s = l_s 2^(m_s - M) / sum_t l_t 2^(m_t - M).
+__global__ void __launch_bounds__(256) k_attn_combine(const float *part_o, const float *part_ml, Geo g, int step0,
+                                                       int nsplit, int rows_pad, bf16 *out) {
+  const int b = blockIdx.y;
+  const int Tq = step0 ? g.H + 1 : g.H;
+  const int qi = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (qi >= kHeads * Tq) return;
+  float M = -INFINITY;
+  for (int s = 0; s < nsplit; ++s) {
+    const size_t pr = ((size_t)b * nsplit + s) * rows_pad + qi;
+    M = fmaxf(M, part_ml[2 * pr]);
+  }
+  float den = 0.f, acc[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+  for (int s = 0; s < nsplit; ++s) {
+    const size_t pr = ((size_t)b * nsplit + s) * rows_pad + qi;
+    const float ms = part_ml[2 * pr], ls = part_ml[2 * pr + 1];
+    if (ls == 0.f) continue;
+    const float wgt = ls * exp2f(ms - M);
+    den += wgt;
+    const float *src = part_o + pr * kHeadDim;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[e] = fmaf(wgt, src[lane + 32 * e], acc[e]);
+  }
+  const int j = qi / kHeads, hd = qi % kHeads;
+  const int tok = step0 ? (j == 0 ? b : g.B + b * g.H + j - 1) : g.B + b * g.H + j;
+  bf16 *dst = out + (size_t)tok * kQDim + hd * kHeadDim;
+  const float inv = 1.0f / den;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) dst[lane + 32 * e] = __float2bfloat16_rn(acc[e] * inv);
+}
+
+int attn_tc_splits(const Geo &g, int step0, int max_keys) {
+  const int Tq = step0 ? g.H + 1 : g.H;
+  const int mtiles = (kHeads * Tq + kRowsPerCta - 1) / kRowsPerCta;
+  const int nblk = (max_keys + kKeyBlock - 1) / kKeyBlock;
+  const int ctas = mtiles * g.B;
+  if (ctas >= 96) return 1;
+  int splits = (148 + ctas - 1) / ctas;
+  const int max_split = (nblk + 1) / 2;  // at least two key blocks per split
+  if (splits > max_split) splits = max_split;
+  return splits < 1 ? 1 : splits;
+}
+
+size_t attn_tc_partial_floats(const Geo &g, int step0, int splits) {
+  if (splits <= 1) return 0;
+  const int Tq = step0 ? g.H + 1 : g.H;
+  const int mtiles = (kHeads * Tq + kRowsPerCta - 1) / kRowsPerCta;
+  return (size_t)g.B * splits * mtiles * kRowsPerCta * (kHeadDim + 2);
+}
+
+void launch_attention_tc(const bf16 *q, const bf16 *ks, const bf16 *vs, const CallPtrs *cp, int layer,
+                         const int *nvalid, const int *vidx, const Geo &g, int step0, int splits, bf16 *out,
+                         float *part, unsigned *err, cudaStream_t s) {
+  cudaFuncSetAttribute(k_attn_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemTotal);
+  const int Tq = step0 ? g.H + 1 : g.H;
+  const int mtiles = (kHeads * Tq + kRowsPerCta - 1) / kRowsPerCta;
+  const int max_keys = g.P + 1 + g.H;
+  const int nblk = (max_keys + kKeyBlock - 1) / kKeyBlock;
+  const int bps = (nblk + splits - 1) / splits;
+  float *part_o = part;
+  float *part_ml = splits > 1 ? part + (size_t)g.B * splits * mtiles * kRowsPerCta * kHeadDim : nullptr;
+  dim3 grid(mtiles, splits, g.B);
+  k_attn_tc<<<grid, 128, kSmemTotal, s>>>(q, ks, vs, cp, layer, nvalid, vidx, g, step0, bps, out, part_o,
+                                          part_ml, err);
+  if (splits > 1) {
+    dim3 cg((kHeads * Tq + 7) / 8, g.B);
+    k_attn_combine<<<cg, 256, 0, s>>>(part_o, part_ml, g, step0, splits, mtiles * kRowsPerCta, out);
+  }
+}
+
+}  // namespace pi0x

@@ -74,6 +74,14 @@ template <typename T>
 void launch_attention(const T *q, const T *ks, const T *vs, const CallPtrs *cp, int layer, const int *nvalid,
                       const int *vidx, const Geo &g, int step0, T *out, cudaStream_t s);
 
+// tcgen05 attention (k_attn_tc.cu); `part` holds attn_tc_partial_floats() floats
+// when splits > 1.
+int attn_tc_splits(const Geo &g, int step0, int max_keys);
+size_t attn_tc_partial_floats(const Geo &g, int step0, int splits);
+void launch_attention_tc(const bf16 *q, const bf16 *ks, const bf16 *vs, const CallPtrs *cp, int layer,
+                         const int *nvalid, const int *vidx, const Geo &g, int step0, int splits, bf16 *out,
+                         float *part, unsigned *err, cudaStream_t s);
+
 // ---- GEMMs ----
 template <typename OutT>
 void launch_gemm_simt(const float *A, int lda, const float *Bw, int ldb, int M, int N, int K, int epi,

@@ -98,6 +98,7 @@ struct Workspace {
   Arena arena;
   int *nvalid, *vidx;
   float *tvec, *xw, *h, *raw;
+  float *part;   // split-KV attention partials (bf16 mode)
   void *xn, *q, *ks, *vs, *att, *act, *a_emb, *u_emb;
   // host-input staging (device side), allocated lazily
   Arena stage;
@@ -256,6 +257,9 @@ int ensure_workspace(pi0x_handle *h, int B, int P, int N) {
   add(es * Rp * kMlp);
   add(es * Rp * kWidth);
   add(es * Rp * kWidth);
+  // split-KV partials: splits*mtiles*B stays below 96 + 148 CTAs (attn_tc_splits)
+  const size_t part_floats = h->bf16 ? (size_t)256 * 128 * (kHeadDim + 2) : 0;
+  add(4 * part_floats);
   void *base = nullptr;
   CK(cudaMalloc(&base, bytes));
   ws.arena.base = static_cast<uint8_t *>(base);
@@ -274,6 +278,7 @@ int ensure_workspace(pi0x_handle *h, int B, int P, int N) {
   ws.act = ws.arena.take(es * Rp * kMlp);
   ws.a_emb = ws.arena.take(es * Rp * kWidth);
   ws.u_emb = ws.arena.take(es * Rp * kWidth);
+  ws.part = (float *)ws.arena.take(4 * part_floats);
   CK(cudaMemset(base, 0, bytes));
   ws.B = nB;
   ws.P = nP;
@@ -412,7 +417,14 @@ int enqueue_loop(pi0x_handle *h, int B, int P, int N, cudaStream_t s) {
                                 M, kQkvDim, kWidth, EPI_STORE_F32, o_raw, s));
       }
       RUN(PI0X_K_ROPE, launch_rope_qkv<T>(ws.raw, row0, M, g, ws.nvalid, h->inv_freq, q, ks, vs, s));
-      RUN(PI0X_K_ATTN, launch_attention<T>(q, ks, vs, h->d_ptrs, l, ws.nvalid, ws.vidx, g, step0, att, s));
+      if (tc) {
+        const int splits = attn_tc_splits(g, step0, P + 1 + H);
+        RUN(PI0X_K_ATTN, launch_attention_tc((const bf16 *)q, (const bf16 *)ks, (const bf16 *)vs, h->d_ptrs, l,
+                                             ws.nvalid, ws.vidx, g, step0, splits, (bf16 *)att, ws.part, h->d_err,
+                                             s));
+      } else {
+        RUN(PI0X_K_ATTN, launch_attention<T>(q, ks, vs, h->d_ptrs, l, ws.nvalid, ws.vidx, g, step0, att, s));
+      }
       GemmOut o_res{ws.h, kWidth, row0, nullptr};
       if (tc) {
         TcGemm gO = h->g_o[l];
@@ -513,6 +525,63 @@ int pi0x_debug_gemm_bf16(const void *A, const void *Bw, int M, int N, int K, flo
     return PI0X_ETIMEOUT;
   }
   return PI0X_OK;
+}
+
+int pi0x_debug_attention(const void *q, const void *ks, const void *vs, const void *prefix_k,
+                         const void *prefix_v, const void *mask, int B, int H, int P, int step0, int impl,
+                         void *out, void *stream) {
+  if (!q || !ks || !vs || !out || (P > 0 && (!prefix_k || !prefix_v || !mask)) || B < 1 || H < 1 || P < 0 ||
+      impl < 0 || impl > 2)
+    return PI0X_EINVAL;
+  cudaStream_t s = (cudaStream_t)stream;
+  Geo g{B, H, 32, 32, P, B + B * H};
+  CallPtrs cp;
+  memset(&cp, 0, sizeof(cp));
+  cp.prefix_k[0] = (const bf16 *)prefix_k;
+  cp.prefix_v[0] = (const bf16 *)prefix_v;
+  cp.mask = (const uint8_t *)mask;
+  CallPtrs *d_cp = nullptr;
+  int *nvalid = nullptr, *vidx = nullptr;
+  float *part = nullptr;
+  unsigned *err = nullptr;
+  const size_t part_floats = (size_t)256 * 128 * (kHeadDim + 2);
+  int st = PI0X_OK;
+  cudaError_t e = cudaMalloc(&d_cp, sizeof(cp));
+  if (e == cudaSuccess) e = cudaMalloc(&nvalid, 4 * (size_t)B);
+  if (e == cudaSuccess) e = cudaMalloc(&vidx, 4 * (size_t)B * (P > 0 ? P : 1));
+  if (e == cudaSuccess) e = cudaMalloc(&part, 4 * part_floats);
+  if (e == cudaSuccess) e = cudaMalloc(&err, 4);
+  if (e == cudaSuccess) e = cudaMemset(err, 0, 4);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(d_cp, &cp, sizeof(cp), cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess) {
+    launch_prep_mask(d_cp, B, P, nvalid, vidx, s);
+    if (impl == 0) {
+      launch_attention<bf16>((const bf16 *)q, (const bf16 *)ks, (const bf16 *)vs, d_cp, 0, nvalid, vidx, g, step0,
+                             (bf16 *)out, s);
+    } else {
+      const int splits = impl == 2 ? 1 : attn_tc_splits(g, step0, P + 1 + H);
+      launch_attention_tc((const bf16 *)q, (const bf16 *)ks, (const bf16 *)vs, d_cp, 0, nvalid, vidx, g, step0,
+                          splits, (bf16 *)out, part, err, s);
+    }
+    e = cudaGetLastError();
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  }
+  if (e != cudaSuccess) {
+    st = cuda_fail(e, "pi0x_debug_attention");
+  } else {
+    unsigned w = 0;
+    cudaMemcpy(&w, err, 4, cudaMemcpyDeviceToHost);
+    if (w) {
+      g_last_error = "device error word 0x" + std::to_string(w);
+      st = PI0X_ETIMEOUT;
+    }
+  }
+  cudaFree(d_cp);
+  cudaFree(nvalid);
+  cudaFree(vidx);
+  cudaFree(part);
+  cudaFree(err);
+  return st;
 }
 
 const char *pi0x_status_string(int st) {
@@ -765,8 +834,16 @@ int pi0x_profile_read(pi0x_handle *h, int kclass, long *launches, double *total_
 
 long pi0x_launch_count(const pi0x_handle *h, int B, int P, int num_steps) {
   if (!h || B < 1 || P < 0 || num_steps < 1) return -1;
-  const long per_layer = 9, L = h->cfg.depth;
-  return 3 + 1 + (long)num_steps * (3 + L * per_layer + 1);
+  const long L = h->cfg.depth, H = h->cfg.horizon;
+  Geo g{B, (int)H, h->cfg.action_dim, h->cfg.state_dim, P, B + B * (int)H};
+  long n = 3 + 1;  // mask prep, time-MLP half, x_1 copy; state token embed
+  for (int k = 0; k < num_steps; ++k) {
+    // action_in, two time-MLP GEMMs, 9 kernels per layer, final norm + Euler
+    long per_layer = 9;
+    if (h->bf16 && attn_tc_splits(g, k == 0, P + 1 + (int)H) > 1) per_layer += 1;  // split-KV combine
+    n += 3 + L * per_layer + 1;
+  }
+  return n;
 }
 
 void pi0x_destroy(pi0x_handle *h) {

@@ -21,7 +21,7 @@ PI0X_DTYPE_BF16, PI0X_DTYPE_F32 = 0, 1
 #: Every symbol include/pi0x.h declares.
 EXPORTED = ["pi0x_create", "pi0x_sample", "pi0x_sync_status", "pi0x_launch_count",
             "pi0x_status_string", "pi0x_last_error", "pi0x_destroy", "pi0x_version",
-            "pi0x_debug_gemm_bf16", "pi0x_profile_enable", "pi0x_profile_read"]
+            "pi0x_debug_gemm_bf16", "pi0x_debug_attention", "pi0x_profile_enable", "pi0x_profile_read"]
 
 #: kernel classes of pi0x_profile_read
 K_CLASSES = ["prep", "embed", "gemm", "norm", "rope", "attn", "geglu", "final"]
@@ -93,6 +93,8 @@ def load() -> ctypes.CDLL:
     lib.pi0x_debug_gemm_bf16.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_int,
                                          ctypes.c_int, ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p]
     lib.pi0x_debug_gemm_bf16.restype = ctypes.c_int
+    lib.pi0x_debug_attention.argtypes = [ctypes.c_void_p] * 6 + [ctypes.c_int] * 5 + [ctypes.c_void_p] * 2
+    lib.pi0x_debug_attention.restype = ctypes.c_int
     lib.pi0x_profile_enable.argtypes = [ctypes.c_void_p, ctypes.c_int]
     lib.pi0x_profile_enable.restype = ctypes.c_int
     lib.pi0x_profile_read.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.POINTER(ctypes.c_long),
@@ -129,6 +131,14 @@ def debug_gemm_bf16(A, Bw, D, bn: int = 128, stream: int = 0):
     _check(load().pi0x_debug_gemm_bf16(_ptr(A), _ptr(Bw), M, N, K, _ptr(D), bn, ctypes.c_void_p(stream)),
            "pi0x_debug_gemm_bf16")
     return D
+
+
+def debug_attention(q, ks, vs, prefix_k, prefix_v, mask, B, H, P, step0, out, impl=1, stream: int = 0):
+    """One layer of suffix attention with the library's kernels (device torch tensors)."""
+    _check(load().pi0x_debug_attention(_ptr(q), _ptr(ks), _ptr(vs), _ptr(prefix_k), _ptr(prefix_v), _ptr(mask),
+                                       B, H, P, int(step0), int(impl), _ptr(out), ctypes.c_void_p(stream)),
+           "pi0x_debug_attention")
+    return out
 
 
 class Sampler:
