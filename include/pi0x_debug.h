@@ -33,6 +33,30 @@ int pi0x_debug_attention(const void *q, const void *ks, const void *vs, const vo
                          const void *prefix_v, const void *mask, int B, int H, int P, int step0, int impl,
                          void *out, void *stream);
 
+/* The same attention as pi0x_debug_attention with impl 1 (tcgen05, split-KV as the
+ * sampler chooses), for callers that cannot allocate device memory while they run
+ * — e.g. a robot control loop that must never stall in cudaMalloc, or an
+ * application whose device memory is owned by its own pool.  It calls no
+ * cudaMalloc/cudaFree and no allocating library routine: all its scratch (a call
+ * table, an error word, the valid-prefix index list and the split-KV partials)
+ * lives in one static device array of 16 MiB inside libpi0x, which every GPU that
+ * loads the library holds until the process exits.  The pages have no counterpart
+ * to this entry point; it is a deployment variant of the `_attend` step.
+ *
+ * Arguments as for pi0x_debug_attention.  Returns PI0X_EINVAL when the problem's
+ * scratch (about 4 B per prefix position per sample plus the split-KV partials,
+ * 4 B x 258 per query row per split) does not fit in the 16 MiB; B=1..8 with the
+ * pi0 prefix lengths fit.  The first call on each device looks up the device
+ * address of the array (cudaGetSymbolAddress, with that device current); make that
+ * first call before any stream capture.  Every call clears the error word it uses;
+ * the array keeps the contents of the last call.  All calls share the one array,
+ * so calls that overlap on the GPU (other streams, other host threads) race.
+ * Synchronous: returns after `stream` has finished the work, with PI0X_ETIMEOUT if
+ * a bounded device wait gave up. */
+int pi0x_attention_noalloc(const void *q, const void *ks, const void *vs, const void *prefix_k,
+                           const void *prefix_v, const void *mask, int B, int H, int P, int step0, void *out,
+                           void *stream);
+
 #ifdef __cplusplus
 }
 #endif

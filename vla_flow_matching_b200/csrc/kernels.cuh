@@ -82,6 +82,9 @@ void launch_attention_tc(const bf16 *q, const bf16 *ks, const bf16 *vs, const Ca
                          const int *nvalid, const int *vidx, const Geo &g, int step0, int splits, bf16 *out,
                          float *part, unsigned *err, cudaStream_t s);
 
+// Text for pi0x_last_error() (this thread).
+void set_last_error(const char *msg);
+
 // ---- GEMMs ----
 template <typename OutT>
 void launch_gemm_simt(const float *A, int lda, const float *Bw, int ldb, int M, int N, int K, int epi,

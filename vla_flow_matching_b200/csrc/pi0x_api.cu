@@ -491,6 +491,10 @@ int get_graph(pi0x_handle *h, int B, int P, int N, cudaGraphExec_t *out) {
 
 }  // namespace
 
+namespace pi0x {
+void set_last_error(const char *msg) { g_last_error = msg; }
+}  // namespace pi0x
+
 // ================================ C ABI =====================================
 extern "C" {
 
