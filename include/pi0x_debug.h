@@ -13,11 +13,13 @@ extern "C" {
 /* D = A * Bw^T on the tcgen05 tensor cores (the GEMM every expert projection
  * uses in PI0X_BF16 mode): A (M, K) bf16 row-major, Bw (N, K) bf16 row-major
  * (nn.Linear weight layout), D (M, N) fp32 row-major; all device pointers,
- * 16-byte aligned.  K % 64 == 0, N % bn == 0, bn in {64, 128, 256}, M >= 1.
- * Enqueued on `stream`; returns PI0X_EINVAL for bad sizes, PI0X_ECUDA if a
- * tensor map cannot be built, PI0X_ETIMEOUT (after synchronizing the stream) if
- * a bounded device wait gave up. */
-int pi0x_debug_gemm_bf16(const void *A, const void *Bw, int M, int N, int K, float *D, int bn, void *stream);
+ * 16-byte aligned.  K % 64 == 0, N % bn == 0, bn in {32, 64, 128, 256}, M >= 1.
+ * splits > 1 splits K over that many CTAs per tile (bn 64 only, at most 148
+ * tiles x splits), the partial tiles being summed in split order by the last
+ * CTA to finish.  Synchronous; returns PI0X_EINVAL for bad sizes, PI0X_ECUDA if
+ * a tensor map cannot be built, PI0X_ETIMEOUT if a bounded device wait gave up. */
+int pi0x_debug_gemm_bf16(const void *A, const void *Bw, int M, int N, int K, float *D, int bn, int splits,
+                         void *stream);
 
 /* One layer of the suffix attention (the `_attend` step of the pi0 page) for B
  * samples with horizon H and prefix length P, all device pointers, bf16 unless

@@ -68,14 +68,18 @@ def test_attention_kernels_match_reference(B, H, P, masked, step0, impl):
     assert (torch.linalg.norm(got - want) / torch.linalg.norm(want)).item() < 6e-3
 
 
-@pytest.mark.parametrize("M,N,K,bn", [
-    (128, 128, 64, 128),      # one tile, one K block
-    (51, 2560, 1024, 256),    # B=1 suffix rows, QKV shape
-    (300, 1024, 2048, 128),   # ragged M over three tiles, O-proj shape
-    (77, 256, 4096, 64),      # ragged tail, long K (ring wraps many times)
-    (1000, 8192, 1024, 256),  # gate/up shape
+@pytest.mark.parametrize("M,N,K,bn,splits", [
+    (128, 128, 64, 128, 1),      # one tile, one K block
+    (51, 2560, 1024, 256, 1),    # B=1 suffix rows, QKV shape
+    (300, 1024, 2048, 128, 1),   # ragged M over three tiles, O-proj shape
+    (77, 256, 4096, 64, 1),      # ragged tail, long K (ring wraps many times)
+    (1000, 8192, 1024, 256, 1),  # gate/up shape
+    (40, 256, 512, 32, 1),       # narrowest tile
+    (51, 2560, 1024, 64, 3),     # split-K as planned for B=1 QKV (uneven last split)
+    (51, 1024, 4096, 64, 8),     # split-K as planned for B=1 down-proj
+    (200, 512, 2048, 64, 9),     # two row tiles, uneven splits
 ])
-def test_tc_gemm_matches_fp32_matmul(M, N, K, bn):
+def test_tc_gemm_matches_fp32_matmul(M, N, K, bn, splits):
     torch = _torch()
     from vla_flow_matching_b200 import build, pi0x
     build.build()
@@ -83,7 +87,8 @@ def test_tc_gemm_matches_fp32_matmul(M, N, K, bn):
     A = torch.randn(M, K, device="cuda", generator=g).to(torch.bfloat16)
     W = (0.05 * torch.randn(N, K, device="cuda", generator=g)).to(torch.bfloat16)
     D = torch.full((M, N), float("nan"), device="cuda")
-    pi0x.debug_gemm_bf16(A, W, D, bn=bn, stream=torch.cuda.current_stream().cuda_stream)
+    for _ in range(2):   # twice: the split-K counters must be back at zero
+        pi0x.debug_gemm_bf16(A, W, D, bn=bn, splits=splits, stream=torch.cuda.current_stream().cuda_stream)
     torch.backends.cuda.matmul.allow_tf32 = False
     ref = A.float() @ W.float().T
     err = (D - ref).abs().max().item()

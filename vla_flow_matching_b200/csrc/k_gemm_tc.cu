@@ -7,6 +7,19 @@
 // MMAs (one elected thread, as tcgen05 wants), then all four warps read the
 // 128 x BN accumulator from TMEM (warp w owns TMEM lanes 32w..32w+31, i.e. rows)
 // and run the epilogue.  Every wait is bounded (common.cuh).
+//
+// Split-K (small row counts): blockIdx.z takes a contiguous range of K blocks and
+// stores its fp32 partial tile; the last CTA of a tile to arrive (counter in global
+// memory) sums the partials in split order — so results do not depend on timing —
+// and runs the epilogue.
+//
+// Fused epilogues (column orders are fixed by a row permutation of the weights at
+// pi0x_create, see pi0x_api.cu):
+//  * EPI_QKV_ROPE: columns come in groups of 16 = 8 rotation pairs (i, i+128) of
+//    one head; the epilogue applies rotate-half RoPE at position n_b + j and writes
+//    q (bf16, 8 heads), k and v (bf16, the layer's suffix K/V rows).
+//  * EPI_GEGLU: groups of 16 = 8 gate then the matching 8 up features; writes
+//    gelu_tanh(gate) * up in bf16.
 #include "common.cuh"
 #include "kernels.cuh"
 
@@ -21,10 +34,101 @@ struct TcCfg {
   static constexpr int kSmem = STAGES * kStage + 1024 /* alignment slack */ + 256 /* barriers */;
 };
 
-template <int BN, int STAGES, typename OutT>
+__device__ __forceinline__ void row_to_bj_tc(int r, int B, int H, int &b, int &j) {
+  if (r < B) {
+    b = r;
+    j = 0;
+  } else {
+    b = (r - B) / H;
+    j = 1 + (r - B) % H;
+  }
+}
+
+__device__ __forceinline__ uint4 pack8_bf16(const float *v) {
+  uint32_t p[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const __nv_bfloat162 h2 = __floats2bfloat162_rn(v[2 * e], v[2 * e + 1]);
+    p[e] = *reinterpret_cast<const uint32_t *>(&h2);
+  }
+  return make_uint4(p[0], p[1], p[2], p[3]);
+}
+
+// Epilogue of 32 consecutive output columns [n, n+32) of GEMM row r.
+template <int EPI>
+__device__ __forceinline__ void epilogue32(const EpiArgs &e, int r, int n, float (&v)[32]) {
+  const int orow = e.out_row0 + r;
+  if constexpr (EPI == EPI_STORE_F32 || EPI == EPI_BIAS_F32 || EPI == EPI_RESID_F32) {
+    float4 *dst = reinterpret_cast<float4 *>(e.out_f32 + (size_t)orow * e.ldo + n);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      float4 w = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+      if constexpr (EPI == EPI_BIAS_F32) {
+        const float4 bb = reinterpret_cast<const float4 *>(e.vec + n)[i];
+        w.x += bb.x; w.y += bb.y; w.z += bb.z; w.w += bb.w;
+      } else if constexpr (EPI == EPI_RESID_F32) {
+        const float4 old = dst[i];
+        w.x += old.x; w.y += old.y; w.z += old.z; w.w += old.w;
+      }
+      dst[i] = w;
+    }
+  } else if constexpr (EPI == EPI_VEC_SILU) {
+    float t[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) t[i] = silu_f(v[i] + e.vec[n + i]);
+    uint4 *dst = reinterpret_cast<uint4 *>(e.out_bf16 + (size_t)orow * e.ldo + n);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) dst[i] = pack8_bf16(t + 8 * i);
+  } else if constexpr (EPI == EPI_QKV_ROPE) {
+    int b, j;
+    row_to_bj_tc(orow, e.B, e.H, b, j);
+    const float pos = (float)(e.nvalid[b] + j);
+#pragma unroll
+    for (int gi = 0; gi < 2; ++gi) {
+      const int gc = (n >> 4) + gi;
+      const int hd = gc >> 4, ib = (gc & 15) * 8;
+      float lo[8], hi[8];
+#pragma unroll
+      for (int w = 0; w < 8; ++w) {
+        lo[w] = v[16 * gi + w];
+        hi[w] = v[16 * gi + 8 + w];
+      }
+      if (hd < kHeads + 1) {
+#pragma unroll
+        for (int w = 0; w < 8; ++w) {
+          float sn, cs;
+          sincosf(pos * e.inv_freq[ib + w], &sn, &cs);
+          const float a = lo[w], bb = hi[w];
+          lo[w] = a * cs - bb * sn;
+          hi[w] = bb * cs + a * sn;
+        }
+      }
+      bf16 *dst;
+      if (hd < kHeads)
+        dst = e.q + (size_t)orow * kQDim + hd * kHeadDim + ib;
+      else if (hd == kHeads)
+        dst = e.ks + (size_t)orow * kHeadDim + ib;
+      else
+        dst = e.vs + (size_t)orow * kHeadDim + ib;
+      *reinterpret_cast<uint4 *>(dst) = pack8_bf16(lo);
+      *reinterpret_cast<uint4 *>(dst + kHeadDim / 2) = pack8_bf16(hi);
+    }
+  } else if constexpr (EPI == EPI_GEGLU) {
+#pragma unroll
+    for (int gi = 0; gi < 2; ++gi) {
+      const int f0 = ((n >> 4) + gi) * 8;
+      float a[8];
+#pragma unroll
+      for (int w = 0; w < 8; ++w) a[w] = gelu_tanh_f(v[16 * gi + w]) * v[16 * gi + 8 + w];
+      *reinterpret_cast<uint4 *>(e.out_bf16 + (size_t)orow * kMlp + f0) = pack8_bf16(a);
+    }
+  }
+}
+
+template <int BN, int STAGES, int EPI>
 __global__ void __launch_bounds__(128, 1)
     k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, int a_row0, int M,
-              int K, int epi, GemmOut o, unsigned *err) {
+              int nk, int kb_per_split, EpiArgs e, unsigned *err) {
   using C = TcCfg<BN, STAGES>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -32,10 +136,13 @@ __global__ void __launch_bounds__(128, 1)
   uint64_t *empty = full + STAGES;
   uint64_t *done = empty + STAGES;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(done + 1);
+  int *last_flag = reinterpret_cast<int *>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int m0 = blockIdx.x * 128, n0 = blockIdx.y * BN;
-  const int nk = K / 64;
+  const int splits = gridDim.z;
+  const int kb0 = blockIdx.z * kb_per_split;
+  const int kb1 = min(nk, kb0 + kb_per_split);
   // After any earlier wait gave up, later GEMMs of the call do nothing (the call's
   // results are already invalid and the host reports PI0X_ETIMEOUT).
   if (*(volatile unsigned *)err != 0) return;
@@ -60,9 +167,9 @@ __global__ void __launch_bounds__(128, 1)
   const uint32_t tmem = *tmem_slot;
 
   if (threadIdx.x == 0) {
-    for (int kb = 0; kb < nk; ++kb) {
-      const int s = kb % STAGES;
-      const uint32_t round = kb / STAGES;
+    for (int kb = kb0; kb < kb1; ++kb) {
+      const int i = kb - kb0, s = i % STAGES;
+      const uint32_t round = i / STAGES;
       if (!mbar_wait(&empty[s], (round & 1u) ^ 1u, err, kErrTimeoutProducer)) break;
       uint8_t *a_dst = smem + s * C::kStage;
       mbar_arrive_expect_tx(&full[s], C::kStage);
@@ -71,9 +178,9 @@ __global__ void __launch_bounds__(128, 1)
     }
   } else if (threadIdx.x == 32) {
     constexpr uint32_t idesc = idesc_bf16_f32(128, BN);
-    for (int kb = 0; kb < nk; ++kb) {
-      const int s = kb % STAGES;
-      const uint32_t round = kb / STAGES;
+    for (int kb = kb0; kb < kb1; ++kb) {
+      const int i = kb - kb0, s = i % STAGES;
+      const uint32_t round = i / STAGES;
       if (!mbar_wait(&full[s], round & 1u, err, kErrTimeoutMma)) break;
       tc_fence_after();
       const uint32_t a_base = smem_u32(smem + s * C::kStage);
@@ -81,7 +188,7 @@ __global__ void __launch_bounds__(128, 1)
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk)
         tc_mma_bf16(tmem, smem_desc_k_sw128(a_base, kk * 32), smem_desc_k_sw128(b_base, kk * 32), idesc,
-                    (kb | kk) != 0);
+                    (i | kk) != 0);
       tc_commit(&empty[s]);
     }
     tc_commit(done);
@@ -90,34 +197,59 @@ __global__ void __launch_bounds__(128, 1)
   const bool ok = mbar_wait(done, 0, err, kErrTimeoutEpilogue);
   __syncwarp();
   tc_fence_after();
-  if (__all_sync(0xffffffffu, ok)) {
-    const int r = m0 + warp * 32 + lane;
-    const size_t orow = (size_t)(o.out_row0 + r) * o.ldo;
+  const bool all_ok = __syncthreads_and(ok);
+  const int rr = warp * 32 + lane;  // row within the tile
+  const int r = m0 + rr;
+  const uint32_t t_lane = (uint32_t)(warp * 32) << 16;
+  if (all_ok) {
+    if (splits == 1) {
 #pragma unroll 1
-    for (int c = 0; c < BN; c += 32) {
-      float v[32];
-      tmem_ld_32x32b_x32(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)c, v);
-      if (r < M) {
-        const int n = n0 + c;
-        if (epi == EPI_STORE_F32 || epi == EPI_BIAS_F32 || epi == EPI_RESID_F32) {
-          float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(o.out) + orow + n);
+      for (int c = 0; c < BN; c += 32) {
+        float v[32];
+        tmem_ld_32x32b_x32(tmem + t_lane + (uint32_t)c, v);
+        if (r < M) epilogue32<EPI>(e, r, n0 + c, v);
+      }
+    } else {
+      const int tile = blockIdx.x * gridDim.y + blockIdx.y;
+      float *mine = e.part + ((size_t)tile * splits + blockIdx.z) * (128 * BN) + (size_t)rr * BN;
+#pragma unroll 1
+      for (int c = 0; c < BN; c += 32) {
+        float v[32];
+        tmem_ld_32x32b_x32(tmem + t_lane + (uint32_t)c, v);
+        if (r < M) {
+          float4 *d4 = reinterpret_cast<float4 *>(mine + c);
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            float4 w = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
-            if (epi == EPI_BIAS_F32) {
-              const float4 bb = reinterpret_cast<const float4 *>(o.vec + n)[i];
-              w.x += bb.x; w.y += bb.y; w.z += bb.z; w.w += bb.w;
-            } else if (epi == EPI_RESID_F32) {
-              const float4 old = dst[i];
-              w.x += old.x; w.y += old.y; w.z += old.z; w.w += old.w;
-            }
-            dst[i] = w;
-          }
-        } else if (epi == EPI_VEC_SILU) {
-          OutT *dst = static_cast<OutT *>(o.out) + orow + n;
-#pragma unroll
-          for (int i = 0; i < 32; ++i) dst[i] = from_f32<OutT>(silu_f(v[i] + o.vec[n + i]));
+          for (int i = 0; i < 8; ++i) d4[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
         }
+      }
+      __threadfence();
+      __syncthreads();
+      if (threadIdx.x == 0) {
+        const int prev = atomicAdd(e.counters + tile, 1);
+        *last_flag = (prev == splits - 1);
+      }
+      __syncthreads();
+      if (*last_flag) {
+        __threadfence();
+        const float *base = e.part + (size_t)tile * splits * (128 * BN) + (size_t)rr * BN;
+        if (r < M) {
+#pragma unroll 1
+          for (int c = 0; c < BN; c += 32) {
+            float v[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = 0.f;
+            for (int s = 0; s < splits; ++s) {
+              const float4 *p4 = reinterpret_cast<const float4 *>(base + (size_t)s * (128 * BN) + c);
+#pragma unroll
+              for (int i = 0; i < 8; ++i) {
+                const float4 t = __ldcg(p4 + i);
+                v[4 * i] += t.x; v[4 * i + 1] += t.y; v[4 * i + 2] += t.z; v[4 * i + 3] += t.w;
+              }
+            }
+            epilogue32<EPI>(e, r, n0 + c, v);
+          }
+        }
+        if (threadIdx.x == 0) e.counters[tile] = 0;  // ready for the next GEMM that uses it
       }
     }
   }
@@ -129,29 +261,66 @@ __global__ void __launch_bounds__(128, 1)
   }
 }
 
-template <int BN, int STAGES, typename OutT>
-static void launch_bn(const TcGemm &g, int a_row0, int M, int epi, const GemmOut &o, unsigned *err,
-                      cudaStream_t s) {
+template <int BN, int STAGES, int EPI>
+static void launch_cfg(const CUtensorMap &tmA, const CUtensorMap &tmB, int a_row0, int M, int N, int K, int splits,
+                       const EpiArgs &e, unsigned *err, cudaStream_t s) {
   using C = TcCfg<BN, STAGES>;
-  auto kern = k_gemm_tc<BN, STAGES, OutT>;
+  auto kern = k_gemm_tc<BN, STAGES, EPI>;
   cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
-  dim3 grid((M + 127) / 128, g.N / BN);
-  kern<<<grid, 128, C::kSmem, s>>>(g.tmA, g.tmB, a_row0, M, g.K, epi, o, err);
+  const int nk = K / 64;
+  const int kps = (nk + splits - 1) / splits;
+  splits = (nk + kps - 1) / kps;
+  dim3 grid((M + 127) / 128, N / BN, splits);
+  kern<<<grid, 128, C::kSmem, s>>>(tmA, tmB, a_row0, M, nk, kps, e, err);
 }
 
-template <typename OutT>
-void launch_gemm_tc(const TcGemm &g, int a_row0, int M, int epi, const GemmOut &o, unsigned *err,
-                    cudaStream_t s) {
-  if (M <= 0) return;
-  switch (g.BN) {
-    case 64: launch_bn<64, 6, OutT>(g, a_row0, M, epi, o, err, s); break;
-    case 128: launch_bn<128, 5, OutT>(g, a_row0, M, epi, o, err, s); break;
-    case 256: launch_bn<256, 4, OutT>(g, a_row0, M, epi, o, err, s); break;
+template <int EPI>
+static void launch_epi(const CUtensorMap &tmA, const CUtensorMap &tmB, int bn, int a_row0, int M, int N, int K,
+                       int splits, const EpiArgs &e, unsigned *err, cudaStream_t s) {
+  switch (bn) {
+    case 32: launch_cfg<32, 8, EPI>(tmA, tmB, a_row0, M, N, K, splits, e, err, s); break;
+    case 64: launch_cfg<64, 6, EPI>(tmA, tmB, a_row0, M, N, K, splits, e, err, s); break;
+    case 128: launch_cfg<128, 5, EPI>(tmA, tmB, a_row0, M, N, K, splits, e, err, s); break;
+    case 256: launch_cfg<256, 4, EPI>(tmA, tmB, a_row0, M, N, K, splits, e, err, s); break;
     default: break;
   }
 }
 
-template void launch_gemm_tc<bf16>(const TcGemm &, int, int, int, const GemmOut &, unsigned *, cudaStream_t);
-template void launch_gemm_tc<float>(const TcGemm &, int, int, int, const GemmOut &, unsigned *, cudaStream_t);
+TcPlan plan_gemm_tc(int M, int N, int K) {
+  TcPlan p;
+  const int mt = (M + 127) / 128;
+  const int nk = K / 64;
+  if (mt >= 8) {
+    p.bn = N >= 2048 ? 256 : 128;
+    p.splits = 1;
+    return p;
+  }
+  p.bn = 64;
+  const int ctas = mt * (N / 64);
+  int sp = ctas >= 148 ? 1 : 148 / ctas;
+  if (sp > nk / 2) sp = nk / 2 > 0 ? nk / 2 : 1;
+  const int kps = (nk + sp - 1) / sp;
+  p.splits = (nk + kps - 1) / kps;
+  return p;
+}
+
+size_t gemm_tc_partial_floats(int M, int N, const TcPlan &p) {
+  if (p.splits <= 1) return 0;
+  return (size_t)((M + 127) / 128) * (N / p.bn) * p.splits * 128 * p.bn;
+}
+
+void launch_gemm_tc(int epi, const CUtensorMap &tmA, const CUtensorMap &tmB, const TcPlan &p, int a_row0, int M,
+                    int N, int K, const EpiArgs &e, unsigned *err, cudaStream_t s) {
+  if (M <= 0) return;
+  switch (epi) {
+    case EPI_STORE_F32: launch_epi<EPI_STORE_F32>(tmA, tmB, p.bn, a_row0, M, N, K, p.splits, e, err, s); break;
+    case EPI_BIAS_F32: launch_epi<EPI_BIAS_F32>(tmA, tmB, p.bn, a_row0, M, N, K, p.splits, e, err, s); break;
+    case EPI_VEC_SILU: launch_epi<EPI_VEC_SILU>(tmA, tmB, p.bn, a_row0, M, N, K, p.splits, e, err, s); break;
+    case EPI_RESID_F32: launch_epi<EPI_RESID_F32>(tmA, tmB, p.bn, a_row0, M, N, K, p.splits, e, err, s); break;
+    case EPI_QKV_ROPE: launch_epi<EPI_QKV_ROPE>(tmA, tmB, p.bn, a_row0, M, N, K, p.splits, e, err, s); break;
+    case EPI_GEGLU: launch_epi<EPI_GEGLU>(tmA, tmB, p.bn, a_row0, M, N, K, p.splits, e, err, s); break;
+    default: break;
+  }
+}
 
 }  // namespace pi0x

@@ -35,6 +35,30 @@ enum Epi : int {
   EPI_BIAS_F32 = 1,    // out_f32[m][n] = D + vec[n]
   EPI_VEC_SILU = 2,    // out_T[m][n] = silu(D + vec[n])
   EPI_RESID_F32 = 3,   // out_f32[m][n] += D
+  EPI_QKV_ROPE = 4,    // tcgen05 only: RoPE'd q, k and v from the permuted QKV columns
+  EPI_GEGLU = 5,       // tcgen05 only: gelu_tanh(gate) * up from the interleaved columns
+};
+
+// Arguments of the tcgen05 GEMM epilogues (rows of the output are out_row0 + m).
+struct EpiArgs {
+  float *out_f32 = nullptr;
+  bf16 *out_bf16 = nullptr;
+  int ldo = 0, out_row0 = 0;
+  const float *vec = nullptr;
+  // EPI_QKV_ROPE: destinations, per-sample valid-prefix counts, RoPE frequencies
+  bf16 *q = nullptr, *ks = nullptr, *vs = nullptr;
+  const int *nvalid = nullptr;
+  const float *inv_freq = nullptr;
+  int B = 0, H = 0;
+  // split-K partial tiles and per-tile arrival counters (zero between GEMMs)
+  float *part = nullptr;
+  int *counters = nullptr;
+};
+
+// Tile width and K split of one tcgen05 GEMM launch.
+struct TcPlan {
+  int bn = 128;
+  int splits = 1;
 };
 
 struct GemmOut {
@@ -90,12 +114,16 @@ template <typename OutT>
 void launch_gemm_simt(const float *A, int lda, const float *Bw, int ldb, int M, int N, int K, int epi,
                       const GemmOut &o, cudaStream_t s);
 
-struct TcGemm {           // one tcgen05 GEMM with its tensor maps (built once)
-  CUtensorMap tmA, tmB;
-  int N, K, BN;
+// Weight operand of a tcgen05 GEMM: tensor maps with 64-row and wide boxes.
+struct TcWeight {
+  CUtensorMap tm64, tm_wide;
+  int N = 0, K = 0, bn_wide = 128;
+  const CUtensorMap &map(int bn) const { return bn == 64 ? tm64 : tm_wide; }
 };
-template <typename OutT>
-void launch_gemm_tc(const TcGemm &g, int a_row0, int M, int epi, const GemmOut &o, unsigned *err,
-                    cudaStream_t s);
+// Tile plan for M rows: wide tiles for large M, 64-wide tiles with split-K below.
+TcPlan plan_gemm_tc(int M, int N, int K);
+size_t gemm_tc_partial_floats(int M, int N, const TcPlan &p);
+void launch_gemm_tc(int epi, const CUtensorMap &tmA, const CUtensorMap &tmB, const TcPlan &p, int a_row0, int M,
+                    int N, int K, const EpiArgs &e, unsigned *err, cudaStream_t s);
 
 }  // namespace pi0x

@@ -99,6 +99,8 @@ struct Workspace {
   int *nvalid, *vidx;
   float *tvec, *xw, *h, *raw;
   float *part;   // split-KV attention partials (bf16 mode)
+  float *gpart;  // split-K GEMM partial tiles (bf16 mode)
+  int *counters; // split-K per-tile arrival counters
   void *xn, *q, *ks, *vs, *att, *act, *a_emb, *u_emb;
   // host-input staging (device side), allocated lazily
   Arena stage;
@@ -123,7 +125,7 @@ struct pi0x_handle {
   float *state_b, *ain_b, *tin_b, *tout_b, *aout_w, *aout_b, *fnorm, *inv_freq;
   LayerW layer[kMaxDepth];
   // weight-side tensor maps + tile widths (bf16 mode)
-  TcGemm g_tin, g_tout, g_qkv[kMaxDepth], g_o[kMaxDepth], g_gu[kMaxDepth], g_down[kMaxDepth];
+  TcWeight g_tin, g_tout, g_qkv[kMaxDepth], g_o[kMaxDepth], g_gu[kMaxDepth], g_down[kMaxDepth];
   Workspace ws;
   CallPtrs *d_ptrs = nullptr;
   unsigned *d_err = nullptr;
@@ -189,6 +191,28 @@ int upload(pi0x_handle *h, const std::vector<float> &v, bool as_act, void **dst)
   return PI0X_OK;
 }
 
+// Row orders of the fused-epilogue GEMM operands (bf16 mode).  Output column c of
+// the GEMM lies in group c/16 of 16 columns.
+//  * [q; k; v] (2560 rows): group g holds, for head hd = g/16 (8 = k, 9 = v) and
+//    pairs i = 8*(g%16) .. +7, the 8 features i (first half of the head) followed
+//    by the 8 features i + 128 they rotate with.
+//  * [gate; up] (8192 rows): group g holds gate features 8g..8g+7 then the up
+//    features with the same indices.
+int qkv_row_source(int c) {
+  const int g = c >> 4, w = c & 15;
+  return (g >> 4) * kHeadDim + (w >> 3) * (kHeadDim / 2) + (g & 15) * 8 + (w & 7);
+}
+int gu_row_source(int c) {
+  const int g = c >> 4, w = c & 15;
+  return (w >> 3) * kMlp + g * 8 + (w & 7);
+}
+void permute_rows(std::vector<float> &m, size_t cols, int (*src)(int)) {
+  const size_t rows = m.size() / cols;
+  std::vector<float> out(m.size());
+  for (size_t r = 0; r < rows; ++r) memcpy(&out[r * cols], &m[(size_t)src((int)r) * cols], cols * 4);
+  m.swap(out);
+}
+
 size_t weight_bytes(const pi0x_config &c, size_t es) {
   const size_t W = kWidth;
   size_t act = W * c.state_dim + W * c.action_dim + 2 * W * W + W * W +
@@ -197,15 +221,13 @@ size_t weight_bytes(const pi0x_config &c, size_t es) {
   return act * es + f32 * 4 + 64 * 1024 * (size_t)(16 + 6 * c.depth);
 }
 
-int pick_bn(int N) { return N >= 2048 ? 256 : 128; }
-
 int build_weight_maps(pi0x_handle *h) {
   const int L = h->cfg.depth;
-  auto mk = [&](TcGemm &g, const void *w, int N, int K) {
+  auto mk = [&](TcWeight &g, const void *w, int N, int K) {
     g.N = N;
     g.K = K;
-    g.BN = pick_bn(N);
-    return make_map(&g.tmB, w, N, K, K, g.BN);
+    g.bn_wide = plan_gemm_tc(1 << 20, N, K).bn;
+    return make_map(&g.tm64, w, N, K, K, 64) && make_map(&g.tm_wide, w, N, K, K, g.bn_wide);
   };
   bool ok = mk(h->g_tin, h->tin_a, kWidth, kWidth) && mk(h->g_tout, h->tout_w, kWidth, kWidth);
   for (int l = 0; l < L && ok; ++l) {
@@ -248,7 +270,13 @@ int ensure_workspace(pi0x_handle *h, int B, int P, int N) {
   add(4 * (size_t)nN * kWidth);
   add(4 * (size_t)nB * H * A);
   add(4 * Rp * kWidth);
-  add(4 * Rp * 2 * kMlp);
+  // fp32 mode: raw GEMM outputs before the RoPE / GeGLU kernels; bf16 mode fuses both
+  const size_t raw_floats = h->bf16 ? 0 : Rp * 2 * kMlp;
+  add(4 * raw_floats);
+  // bf16 split-K GEMMs: split-K is used only while tiles x splits <= 148 (plan_gemm_tc)
+  const size_t gpart_floats = h->bf16 ? (size_t)148 * 128 * 64 : 0;
+  add(4 * gpart_floats);
+  add(4 * 1024);
   add(es * Rp * kWidth);
   add(es * Rp * kQDim);
   add(es * (size_t)L * Rp * kHeadDim);
@@ -269,7 +297,9 @@ int ensure_workspace(pi0x_handle *h, int B, int P, int N) {
   ws.tvec = (float *)ws.arena.take(4 * (size_t)nN * kWidth);
   ws.xw = (float *)ws.arena.take(4 * (size_t)nB * H * A);
   ws.h = (float *)ws.arena.take(4 * Rp * kWidth);
-  ws.raw = (float *)ws.arena.take(4 * Rp * 2 * kMlp);
+  ws.raw = (float *)ws.arena.take(4 * raw_floats);
+  ws.gpart = (float *)ws.arena.take(4 * gpart_floats);
+  ws.counters = (int *)ws.arena.take(4 * 1024);
   ws.xn = ws.arena.take(es * Rp * kWidth);
   ws.q = ws.arena.take(es * Rp * kQDim);
   ws.ks = ws.arena.take(es * (size_t)L * Rp * kHeadDim);
@@ -376,6 +406,19 @@ int enqueue_loop(pi0x_handle *h, int B, int P, int N, cudaStream_t s) {
   T *xn = (T *)ws.xn, *q = (T *)ws.q, *att = (T *)ws.att, *act = (T *)ws.act;
   T *aemb = (T *)ws.a_emb, *uemb = (T *)ws.u_emb;
   const size_t kv_stride = (size_t)R * kHeadDim;
+  // tcgen05 GEMM with its tile plan for M rows; weight row orders of QKV and gate/up
+  // were permuted at create time for the fused RoPE / GeGLU epilogues
+  EpiArgs ebase;
+  ebase.nvalid = ws.nvalid;
+  ebase.inv_freq = h->inv_freq;
+  ebase.B = B;
+  ebase.H = H;
+  ebase.part = ws.gpart;
+  ebase.counters = ws.counters;
+  auto gemm = [&](int epi, const CUtensorMap &tmA, const TcWeight &w, int a_row0, int M, const EpiArgs &e) {
+    const TcPlan p = plan_gemm_tc(M, w.N, w.K);
+    launch_gemm_tc(epi, tmA, w.map(p.bn), p, a_row0, M, w.N, w.K, e, h->d_err, s);
+  };
 
   RUN(PI0X_K_PREP, launch_prep_mask(h->d_ptrs, B, P, ws.nvalid, ws.vidx, s));
   RUN(PI0X_K_PREP, launch_time_vec<T>((const T *)h->tin_t, h->tin_b, N, ws.tvec, s));
@@ -391,12 +434,17 @@ int enqueue_loop(pi0x_handle *h, int B, int P, int N, cudaStream_t s) {
     GemmOut o_u{uemb, kWidth, 0, ws.tvec + (size_t)k * kWidth};
     GemmOut o_h{ws.h, kWidth, B, h->tout_b};
     if (tc) {
-      TcGemm gt = h->g_tin;
-      gt.tmA = ws.m_aemb;
-      RUN(PI0X_K_GEMM, launch_gemm_tc<bf16>(gt, 0, BH, EPI_VEC_SILU, o_u, h->d_err, s));
-      TcGemm go = h->g_tout;
-      go.tmA = ws.m_uemb;
-      RUN(PI0X_K_GEMM, launch_gemm_tc<bf16>(go, 0, BH, EPI_BIAS_F32, o_h, h->d_err, s));
+      EpiArgs eu = ebase;
+      eu.out_bf16 = (bf16 *)uemb;
+      eu.ldo = kWidth;
+      eu.vec = ws.tvec + (size_t)k * kWidth;
+      RUN(PI0X_K_GEMM, gemm(EPI_VEC_SILU, ws.m_aemb, h->g_tin, 0, BH, eu));
+      EpiArgs eh = ebase;
+      eh.out_f32 = ws.h;
+      eh.ldo = kWidth;
+      eh.out_row0 = B;
+      eh.vec = h->tout_b;
+      RUN(PI0X_K_GEMM, gemm(EPI_BIAS_F32, ws.m_uemb, h->g_tout, 0, BH, eh));
     } else {
       RUN(PI0X_K_GEMM, launch_gemm_simt<float>((const float *)aemb, kWidth, (const float *)h->tin_a, kWidth, BH, kWidth, kWidth,
                               EPI_VEC_SILU, o_u, s));
@@ -409,14 +457,17 @@ int enqueue_loop(pi0x_handle *h, int B, int P, int N, cudaStream_t s) {
       RUN(PI0X_K_NORM, launch_rmsnorm<T>(ws.h, row0, M, lw.in_norm, xn, s));
       GemmOut o_raw{ws.raw, kQkvDim, row0, nullptr};
       if (tc) {
-        TcGemm gq = h->g_qkv[l];
-        gq.tmA = ws.m_xn;
-        RUN(PI0X_K_GEMM, launch_gemm_tc<bf16>(gq, row0, M, EPI_STORE_F32, o_raw, h->d_err, s));
+        EpiArgs eq = ebase;
+        eq.out_row0 = row0;
+        eq.q = (bf16 *)q;
+        eq.ks = (bf16 *)ks;
+        eq.vs = (bf16 *)vs;
+        RUN(PI0X_K_GEMM, gemm(EPI_QKV_ROPE, ws.m_xn, h->g_qkv[l], row0, M, eq));
       } else {
         RUN(PI0X_K_GEMM, launch_gemm_simt<float>((const float *)xn + (size_t)row0 * kWidth, kWidth, (const float *)lw.qkv, kWidth,
                                 M, kQkvDim, kWidth, EPI_STORE_F32, o_raw, s));
+        RUN(PI0X_K_ROPE, launch_rope_qkv<T>(ws.raw, row0, M, g, ws.nvalid, h->inv_freq, q, ks, vs, s));
       }
-      RUN(PI0X_K_ROPE, launch_rope_qkv<T>(ws.raw, row0, M, g, ws.nvalid, h->inv_freq, q, ks, vs, s));
       if (tc) {
         const int splits = attn_tc_splits(g, step0, P + 1 + H);
         RUN(PI0X_K_ATTN, launch_attention_tc((const bf16 *)q, (const bf16 *)ks, (const bf16 *)vs, h->d_ptrs, l,
@@ -426,10 +477,12 @@ int enqueue_loop(pi0x_handle *h, int B, int P, int N, cudaStream_t s) {
         RUN(PI0X_K_ATTN, launch_attention<T>(q, ks, vs, h->d_ptrs, l, ws.nvalid, ws.vidx, g, step0, att, s));
       }
       GemmOut o_res{ws.h, kWidth, row0, nullptr};
+      EpiArgs eres = ebase;
+      eres.out_f32 = ws.h;
+      eres.ldo = kWidth;
+      eres.out_row0 = row0;
       if (tc) {
-        TcGemm gO = h->g_o[l];
-        gO.tmA = ws.m_att;
-        RUN(PI0X_K_GEMM, launch_gemm_tc<bf16>(gO, row0, M, EPI_RESID_F32, o_res, h->d_err, s));
+        RUN(PI0X_K_GEMM, gemm(EPI_RESID_F32, ws.m_att, h->g_o[l], row0, M, eres));
       } else {
         RUN(PI0X_K_GEMM, launch_gemm_simt<float>((const float *)att + (size_t)row0 * kQDim, kQDim, (const float *)lw.o, kQDim, M,
                                 kWidth, kQDim, EPI_RESID_F32, o_res, s));
@@ -437,18 +490,17 @@ int enqueue_loop(pi0x_handle *h, int B, int P, int N, cudaStream_t s) {
       RUN(PI0X_K_NORM, launch_rmsnorm<T>(ws.h, row0, M, lw.post_norm, xn, s));
       GemmOut o_gu{ws.raw, 2 * kMlp, row0, nullptr};
       if (tc) {
-        TcGemm gg = h->g_gu[l];
-        gg.tmA = ws.m_xn;
-        RUN(PI0X_K_GEMM, launch_gemm_tc<bf16>(gg, row0, M, EPI_STORE_F32, o_gu, h->d_err, s));
+        EpiArgs eg = ebase;
+        eg.out_bf16 = (bf16 *)act;
+        eg.out_row0 = row0;
+        RUN(PI0X_K_GEMM, gemm(EPI_GEGLU, ws.m_xn, h->g_gu[l], row0, M, eg));
       } else {
         RUN(PI0X_K_GEMM, launch_gemm_simt<float>((const float *)xn + (size_t)row0 * kWidth, kWidth, (const float *)lw.gu, kWidth, M,
                                 2 * kMlp, kWidth, EPI_STORE_F32, o_gu, s));
+        RUN(PI0X_K_GEGLU, launch_geglu<T>(ws.raw, row0, M, act, s));
       }
-      RUN(PI0X_K_GEGLU, launch_geglu<T>(ws.raw, row0, M, act, s));
       if (tc) {
-        TcGemm gd = h->g_down[l];
-        gd.tmA = ws.m_act;
-        RUN(PI0X_K_GEMM, launch_gemm_tc<bf16>(gd, row0, M, EPI_RESID_F32, o_res, h->d_err, s));
+        RUN(PI0X_K_GEMM, gemm(EPI_RESID_F32, ws.m_act, h->g_down[l], row0, M, eres));
       } else {
         RUN(PI0X_K_GEMM, launch_gemm_simt<float>((const float *)act + (size_t)row0 * kMlp, kMlp, (const float *)lw.down, kMlp, M,
                                 kWidth, kMlp, EPI_RESID_F32, o_res, s));
@@ -500,25 +552,37 @@ extern "C" {
 
 int pi0x_version(void) { return 100; }
 
-int pi0x_debug_gemm_bf16(const void *A, const void *Bw, int M, int N, int K, float *D, int bn, void *stream) {
-  if (!A || !Bw || !D || M < 1 || N < 1 || K < 64 || K % 64 || (bn != 64 && bn != 128 && bn != 256) || N % bn)
+int pi0x_debug_gemm_bf16(const void *A, const void *Bw, int M, int N, int K, float *D, int bn, int splits,
+                         void *stream) {
+  if (!A || !Bw || !D || M < 1 || N < 1 || K < 64 || K % 64 ||
+      (bn != 32 && bn != 64 && bn != 128 && bn != 256) || N % bn || splits < 1 || splits > K / 64 ||
+      (splits > 1 && (size_t)((M + 127) / 128) * (N / bn) * splits > 148) || (splits > 1 && bn != 64))
     return PI0X_EINVAL;
   static unsigned *d_err = nullptr;
+  static float *d_part = nullptr;
+  static int *d_cnt = nullptr;
   if (!d_err) {
     CK(cudaMalloc(&d_err, sizeof(unsigned)));
     CK(cudaMemset(d_err, 0, sizeof(unsigned)));
+    CK(cudaMalloc(&d_part, sizeof(float) * 148 * 128 * 64));
+    CK(cudaMalloc(&d_cnt, sizeof(int) * 1024));
+    CK(cudaMemset(d_cnt, 0, sizeof(int) * 1024));
   }
-  TcGemm g;
-  g.N = N;
-  g.K = K;
-  g.BN = bn;
-  if (!make_map(&g.tmA, A, M, K, K, 128) || !make_map(&g.tmB, Bw, N, K, K, bn)) {
+  CUtensorMap tmA, tmB;
+  if (!make_map(&tmA, A, M, K, K, 128) || !make_map(&tmB, Bw, N, K, K, bn)) {
     g_last_error = "cuTensorMapEncodeTiled failed";
     return PI0X_ECUDA;
   }
   cudaStream_t s = (cudaStream_t)stream;
-  GemmOut o{D, N, 0, nullptr};
-  launch_gemm_tc<float>(g, 0, M, EPI_STORE_F32, o, d_err, s);
+  EpiArgs e;
+  e.out_f32 = D;
+  e.ldo = N;
+  e.part = d_part;
+  e.counters = d_cnt;
+  TcPlan p;
+  p.bn = bn;
+  p.splits = splits;
+  launch_gemm_tc(EPI_STORE_F32, tmA, tmB, p, 0, M, N, K, e, d_err, s);
   CK(cudaGetLastError());
   CK(cudaStreamSynchronize(s));
   unsigned err = 0;
@@ -689,6 +753,7 @@ int pi0x_create(const pi0x_config *cfg, const pi0x_weights *w, pi0x_handle **out
     qkv.insert(qkv.end(), v.begin(), v.end());
     FETCH(lw.v_w, (size_t)kHeadDim * W, v);
     qkv.insert(qkv.end(), v.begin(), v.end());
+    if (h->bf16) permute_rows(qkv, W, qkv_row_source);
     UP(qkv, true, d.qkv);
     FETCH(lw.o_w, W * kQDim, v); UP(v, true, d.o);
     // [gate; up] rows -> one (8192, 1024) operand
@@ -697,6 +762,7 @@ int pi0x_create(const pi0x_config *cfg, const pi0x_weights *w, pi0x_handle **out
     gu.insert(gu.end(), v.begin(), v.end());
     FETCH(lw.up_w, (size_t)kMlp * W, v);
     gu.insert(gu.end(), v.begin(), v.end());
+    if (h->bf16) permute_rows(gu, W, gu_row_source);
     UP(gu, true, d.gu);
     FETCH(lw.down_w, W * kMlp, v); UP(v, true, d.down);
   }

@@ -91,7 +91,8 @@ def load() -> ctypes.CDLL:
     lib.pi0x_version.argtypes = []
     lib.pi0x_version.restype = ctypes.c_int
     lib.pi0x_debug_gemm_bf16.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_int,
-                                         ctypes.c_int, ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p]
+                                         ctypes.c_int, ctypes.c_void_p, ctypes.c_int, ctypes.c_int,
+                                         ctypes.c_void_p]
     lib.pi0x_debug_gemm_bf16.restype = ctypes.c_int
     lib.pi0x_debug_attention.argtypes = [ctypes.c_void_p] * 6 + [ctypes.c_int] * 5 + [ctypes.c_void_p] * 2
     lib.pi0x_debug_attention.restype = ctypes.c_int
@@ -124,12 +125,12 @@ def _check(status: int, what: str):
         raise Pi0xError(status, what)
 
 
-def debug_gemm_bf16(A, Bw, D, bn: int = 128, stream: int = 0):
+def debug_gemm_bf16(A, Bw, D, bn: int = 128, splits: int = 1, stream: int = 0):
     """D = A @ Bw.T with the library's tcgen05 GEMM (device torch tensors: bf16, bf16, fp32)."""
     M, K = A.shape
     N = Bw.shape[0]
-    _check(load().pi0x_debug_gemm_bf16(_ptr(A), _ptr(Bw), M, N, K, _ptr(D), bn, ctypes.c_void_p(stream)),
-           "pi0x_debug_gemm_bf16")
+    _check(load().pi0x_debug_gemm_bf16(_ptr(A), _ptr(Bw), M, N, K, _ptr(D), bn, splits,
+                                       ctypes.c_void_p(stream)), "pi0x_debug_gemm_bf16")
     return D
 
 
