@@ -113,19 +113,30 @@ __global__ void __launch_bounds__(128, 1)
       cp_async16(sbase + kSmemQ + (cr >> 3) * (128 * 128) + sw128_off(r, cr & 7), src, ok);
     }
   }
+  // Warp w copies keys [16w, 16w+16) of a block, lane = 16-byte chunk of the 512-byte
+  // row.  Lanes 0..15 first look up one key's source row each (independent loads),
+  // then every copy takes its row pointer from a shuffle.
   auto load_block = [&](int blk, int buf, bool with_v) {
     const uint32_t kb = sbase + kSmemK0 + buf * kKVBytes, vb = sbase + kSmemV0 + buf * kKVBytes;
+    const int kk_l = blk * kKeyBlock + warp * 16 + (lane & 15);
+    const bool ok_l = kk_l < nk;
+    const bf16 *krow = ks, *vrow = vs;
+    if (ok_l) {
+      krow = key_row(kk_l, nv, b, g, pref_k, vi, ks);
+      vrow = key_row(kk_l, nv, b, g, pref_v, vi, vs);
+    }
+#pragma unroll
     for (int i = 0; i < 16; ++i) {
-      const int c = tid + 128 * i;
-      const int r = c >> 5, cr = c & 31;
-      const int kk = blk * kKeyBlock + r;
-      const bool ok = kk < nk;
-      const uint32_t off = (cr >> 3) * (64 * 128) + sw128_off(r, cr & 7);
-      const bf16 *ksrc = ok ? key_row(kk, nv, b, g, pref_k, vi, ks) + cr * 8 : ks;
-      cp_async16(kb + off, ksrc, ok);
+      const int r = warp * 16 + i;
+      const bool ok = __shfl_sync(0xffffffffu, ok_l, i);
+      const uint32_t off = (lane >> 3) * (64 * 128) + sw128_off(r, lane & 7);
+      const bf16 *ksrc = reinterpret_cast<const bf16 *>(
+          __shfl_sync(0xffffffffu, reinterpret_cast<uintptr_t>(krow), i));
+      cp_async16(kb + off, ksrc + lane * 8, ok);
       if (with_v) {
-        const bf16 *vsrc = ok ? key_row(kk, nv, b, g, pref_v, vi, vs) + cr * 8 : vs;
-        cp_async16(vb + off, vsrc, ok);
+        const bf16 *vsrc = reinterpret_cast<const bf16 *>(
+            __shfl_sync(0xffffffffu, reinterpret_cast<uintptr_t>(vrow), i));
+        cp_async16(vb + off, vsrc + lane * 8, ok);
       }
     }
   };
@@ -204,8 +215,8 @@ __global__ void __launch_bounds__(128, 1)
       if (mn != -INFINITY) {
         float add = 0.f;
 #pragma unroll
-        for (int i = 0; i < 64; ++i) add += exp2f(sv[i] - mn);
-        l = l * exp2f(m - mn) + add;
+        for (int i = 0; i < 64; ++i) add += ex2_approx(sv[i] - mn);
+        l = l * ex2_approx(m - mn) + add;
         m = mn;
       }
       if (j == nb - 1) inv_l = l > 0.f ? 1.0f / l : 0.f;
@@ -218,8 +229,8 @@ __global__ void __launch_bounds__(128, 1)
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const int i0 = cc * 8 + 2 * e;
-          const float p0 = (kbase + i0 < key_lim) ? exp2f(sv[i0] * scale_l2 - m) * inv_l : 0.f;
-          const float p1 = (kbase + i0 + 1 < key_lim) ? exp2f(sv[i0 + 1] * scale_l2 - m) * inv_l : 0.f;
+          const float p0 = (kbase + i0 < key_lim) ? ex2_approx(sv[i0] * scale_l2 - m) * inv_l : 0.f;
+          const float p1 = (kbase + i0 + 1 < key_lim) ? ex2_approx(sv[i0 + 1] * scale_l2 - m) * inv_l : 0.f;
           const __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
           pk[e] = *reinterpret_cast<const uint32_t *>(&h2);
         }
@@ -317,7 +328,7 @@ __global__ void __launch_bounds__(256) k_attn_combine(const float *part_o, const
     const size_t pr = ((size_t)b * nsplit + s) * rows_pad + qi;
     const float ms = part_ml[2 * pr], ls = part_ml[2 * pr + 1];
     if (ls == 0.f) continue;
-    const float wgt = ls * exp2f(ms - M);
+    const float wgt = ls * ex2_approx(ms - M);
     den += wgt;
     const float *src = part_o + pr * kHeadDim;
 #pragma unroll
