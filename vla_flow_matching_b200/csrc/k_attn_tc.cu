@@ -10,12 +10,13 @@
 // swizzled shared memory, so masked prefix positions are never read; the page adds
 // -2.38e38 to their logits, whose exp is exactly 0 in fp32.
 //
-// Softmax in two passes over the key blocks: pass 1 forms the exact row max m and
-// sum l (S = Q K^T in TMEM, read back by the thread owning the row); pass 2
-// recomputes S and writes P = exp(s - m) / l rounded to bf16 (the page casts the
-// fp32 probabilities to the query dtype before P.V) and accumulates O += P V in
-// TMEM.  O therefore never needs rescaling.  With split-KV (small batches) every
-// split normalises by its own (m, l) and k_attn_combine merges the splits.
+// One pass over the key blocks with an online softmax.  S = Q K^T goes to one of
+// two TMEM buffers, so the MMA of block w+1 runs while the threads (one per query
+// row) turn block w into P = 2^(s - m) in bf16 and accumulate O += P V in TMEM.
+// The running max m used for P is raised (and O, l rescaled in place) only when a
+// block's max exceeds it by more than 2^8, so P stays <= 256 and rescaling is
+// rare; O / l at the end normalises.  With split-KV (small batches) every split
+// writes O/l and (m, l) and k_attn_combine merges the splits.
 #include <math.h>
 
 #include "common.cuh"
@@ -35,9 +36,10 @@ constexpr uint32_t kSmemV0 = kSmemK0 + 2 * kKVBytes;
 constexpr uint32_t kSmemP = kSmemV0 + 2 * kKVBytes;
 constexpr uint32_t kSmemBar = kSmemP + kPBytes;
 constexpr uint32_t kSmemTotal = kSmemBar + 64 + 1024;  // + alignment slack
-constexpr uint32_t kTmemCols = 512;   // S at column 0 (64 cols), O at column 256 (256 cols)
+constexpr uint32_t kTmemCols = 512;   // S buffers at columns 0 and 64, O at 256 (256 columns)
 constexpr uint32_t kTmemO = 256;
 constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kRescaleSlack = 8.0f;  // log2 units
 }  // namespace
 
 // Source row (256 bf16) of key `kk` of sample b: valid prefix positions first, then
@@ -57,9 +59,9 @@ __global__ void __launch_bounds__(128, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
-  uint64_t *bar_s = reinterpret_cast<uint64_t *>(smem + kSmemBar);
-  uint64_t *bar_o = bar_s + 1;
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar_s + 2);
+  uint64_t *bar_s = reinterpret_cast<uint64_t *>(smem + kSmemBar);  // [2]
+  uint64_t *bar_o = bar_s + 2;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar_s + 3);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int b = blockIdx.z, split = blockIdx.y, nsplit = gridDim.y;
@@ -86,7 +88,8 @@ __global__ void __launch_bounds__(128, 1)
   const int *vi = vidx + (size_t)b * g.P;
 
   if (tid == 0) {
-    mbar_init(bar_s, 1);
+    mbar_init(&bar_s[0], 1);
+    mbar_init(&bar_s[1], 1);
     mbar_init(bar_o, 1);
     fence_mbar_init();
   }
@@ -96,44 +99,45 @@ __global__ void __launch_bounds__(128, 1)
   }
 
   // ---- Q tile: rows [row0, row0+128), 4 swizzled sub-tiles of 64 dims ----
-  {
-    // chunk c: row = c / 32, cr = c % 32 (sub-tile cr/8, chunk cr%8); a warp copies one 512 B row
-    for (int i = 0; i < 32; ++i) {
-      const int c = tid + 128 * i;
-      const int r = c >> 5, cr = c & 31;
-      const int qr = row0 + r;
-      const bool ok = qr < nrows;
-      int t = 0, hd = 0;
-      if (ok) {
-        const int j = qr / kHeads;
-        hd = qr % kHeads;
-        t = step0 ? (j == 0 ? b : g.B + b * g.H + j - 1) : g.B + b * g.H + j;
-      }
-      const bf16 *src = q + (size_t)t * kQDim + hd * kHeadDim + cr * 8;
-      cp_async16(sbase + kSmemQ + (cr >> 3) * (128 * 128) + sw128_off(r, cr & 7), src, ok);
+  for (int i = 0; i < 32; ++i) {
+    const int c = tid + 128 * i;
+    const int r = c >> 5, cr = c & 31;
+    const int qr = row0 + r;
+    const bool ok = qr < nrows;
+    int t = 0, hd = 0;
+    if (ok) {
+      const int j = qr / kHeads;
+      hd = qr % kHeads;
+      t = step0 ? (j == 0 ? b : g.B + b * g.H + j - 1) : g.B + b * g.H + j;
     }
+    const bf16 *src = q + (size_t)t * kQDim + hd * kHeadDim + cr * 8;
+    cp_async16(sbase + kSmemQ + (cr >> 3) * (128 * 128) + sw128_off(r, cr & 7), src, ok);
   }
-  // Warp w copies keys [16w, 16w+16) of a block, lane = 16-byte chunk of the 512-byte
+  // Warp w copies keys [16w, 16w+16) of block j, lane = 16-byte chunk of the 512-byte
   // row.  Lanes 0..15 first look up one key's source row each (independent loads),
-  // then every copy takes its row pointer from a shuffle.
-  auto load_block = [&](int blk, int buf, bool with_v) {
+  // then every copy takes its row pointer from a shuffle.  `which`: 1 = K, 2 = V.
+  auto load_block = [&](int j, int which) {
+    if (j >= nb) return;
+    const int blk = blk0 + j, buf = j & 1;
     const uint32_t kb = sbase + kSmemK0 + buf * kKVBytes, vb = sbase + kSmemV0 + buf * kKVBytes;
     const int kk_l = blk * kKeyBlock + warp * 16 + (lane & 15);
     const bool ok_l = kk_l < nk;
     const bf16 *krow = ks, *vrow = vs;
     if (ok_l) {
-      krow = key_row(kk_l, nv, b, g, pref_k, vi, ks);
-      vrow = key_row(kk_l, nv, b, g, pref_v, vi, vs);
+      if (which & 1) krow = key_row(kk_l, nv, b, g, pref_k, vi, ks);
+      if (which & 2) vrow = key_row(kk_l, nv, b, g, pref_v, vi, vs);
     }
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
       const int r = warp * 16 + i;
       const bool ok = __shfl_sync(0xffffffffu, ok_l, i);
       const uint32_t off = (lane >> 3) * (64 * 128) + sw128_off(r, lane & 7);
-      const bf16 *ksrc = reinterpret_cast<const bf16 *>(
-          __shfl_sync(0xffffffffu, reinterpret_cast<uintptr_t>(krow), i));
-      cp_async16(kb + off, ksrc + lane * 8, ok);
-      if (with_v) {
+      if (which & 1) {
+        const bf16 *ksrc = reinterpret_cast<const bf16 *>(
+            __shfl_sync(0xffffffffu, reinterpret_cast<uintptr_t>(krow), i));
+        cp_async16(kb + off, ksrc + lane * 8, ok);
+      }
+      if (which & 2) {
         const bf16 *vsrc = reinterpret_cast<const bf16 *>(
             __shfl_sync(0xffffffffu, reinterpret_cast<uintptr_t>(vrow), i));
         cp_async16(vb + off, vsrc + lane * 8, ok);
@@ -141,8 +145,13 @@ __global__ void __launch_bounds__(128, 1)
     }
   };
 
-  const int nitems = 2 * nb;
-  if (nitems > 0) load_block(blk0, 0, false);
+  // cp.async groups, committed in this order (empty groups keep the pattern):
+  //   prologue: [Q, K0, V0] [K1] [V1];  iteration w: [K(w+2)] [V(w+1) after PV(w-1)]
+  load_block(0, 3);
+  cp_async_commit();
+  load_block(1, 1);
+  cp_async_commit();
+  load_block(1, 2);
   cp_async_commit();
 
   tc_fence_before();
@@ -155,73 +164,97 @@ __global__ void __launch_bounds__(128, 1)
   constexpr uint32_t idesc_o = idesc_bf16_f32(128, kHeadDim) | (1u << 16);  // B (V) MN-major
   const float scale_l2 = 0.0625f * kLog2e;
 
-  float m = -INFINITY, l = 0.f, inv_l = 0.f;
-  uint32_t ph_s = 0, ph_o = 0;
+  auto issue_s = [&](int j) {  // S[j&1] = Q K(j)^T
+    const uint32_t kb = sbase + kSmemK0 + (j & 1) * kKVBytes;
+    const uint32_t d = tmem + (uint32_t)((j & 1) * kKeyBlock);
+#pragma unroll
+    for (int s = 0; s < 4; ++s)
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk)
+        tc_mma_bf16(d, smem_desc_k_sw128(sbase + kSmemQ + s * (128 * 128), kk * 32),
+                    smem_desc_k_sw128(kb + s * (64 * 128), kk * 32), idesc_s, (s | kk) != 0);
+    tc_commit(&bar_s[j & 1]);
+  };
+
+  float m_used = -INFINITY, l = 0.f;
+  uint32_t ph_s0 = 0, ph_s1 = 0, ph_o = 0;
   bool ok_all = true;
-  for (int w = 0; w < nitems; ++w) {
-    const int pass = w / nb, j = w % nb, buf = w & 1;
-    const int blk = blk0 + j;
-    // The PV MMA of item w-1 reads V[buf^1] and P: wait for it before reusing them.
-    if (w >= 1 && (w - 1) / nb == 1) {
-      if (!mbar_wait(bar_o, ph_o, err, kErrTimeoutMma)) ok_all = false;
-      ph_o ^= 1u;
-    }
-    if (w + 1 < nitems) {
-      const int wn = w + 1;
-      load_block(blk0 + wn % nb, wn & 1, wn / nb == 1);
-    }
-    cp_async_commit();
-    cp_async_wait<1>();
+  if (nb > 0) {
+    cp_async_wait<2>();
     fence_proxy_async_smem();
     tc_fence_before();
     ok_all = __syncthreads_and(ok_all);
     tc_fence_after();
-    if (!ok_all) break;
-    if (tid == 0) {
-      const uint32_t kb = sbase + kSmemK0 + buf * kKVBytes;
-#pragma unroll
-      for (int s = 0; s < 4; ++s)
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          tc_mma_bf16(tmem, smem_desc_k_sw128(sbase + kSmemQ + s * (128 * 128), kk * 32),
-                      smem_desc_k_sw128(kb + s * (64 * 128), kk * 32), idesc_s, (s | kk) != 0);
-      tc_commit(bar_s);
+    if (tid == 0 && ok_all) issue_s(0);
+  }
+  for (int w = 0; w < nb && ok_all; ++w) {
+    const int buf = w & 1;
+    // (1) K(w+1) has landed: start S(w+1) on the tensor cores before the softmax of w
+    if (w + 1 < nb) {
+      cp_async_wait<1>();
+      fence_proxy_async_smem();
+      tc_fence_before();
+      ok_all = __syncthreads_and(ok_all);
+      tc_fence_after();
+      if (!ok_all) break;
+      if (tid == 0) issue_s(w + 1);
+    }
+    // (2) softmax of block w
+    {
+      uint32_t &ph = buf ? ph_s1 : ph_s0;
+      if (!mbar_wait(&bar_s[buf], ph, err, kErrTimeoutEpilogue)) ok_all = false;
+      ph ^= 1u;
     }
     __syncwarp();
-    if (!mbar_wait(bar_s, ph_s, err, kErrTimeoutEpilogue)) ok_all = false;
-    ph_s ^= 1u;
-    __syncwarp();
     tc_fence_after();
+    // K(buf) is free again (S(w) done): prefetch K(w+2)
+    load_block(w + 2, 1);
+    cp_async_commit();
     float sv[64];
     {
       float t0[32], t1[32];
-      tmem_ld_32x32b_x32(tmem + t_lane + 0, t0);
-      tmem_ld_32x32b_x32(tmem + t_lane + 32, t1);
+      tmem_ld_32x32b_x32(tmem + t_lane + buf * kKeyBlock, t0);
+      tmem_ld_32x32b_x32(tmem + t_lane + buf * kKeyBlock + 32, t1);
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
         sv[i] = t0[i];
         sv[32 + i] = t1[i];
       }
     }
-    const int kbase = blk * kKeyBlock;
-    if (pass == 0) {
-      float bm = -INFINITY;
+    const int kbase = (blk0 + w) * kKeyBlock;
+    float bm = -INFINITY;
 #pragma unroll
-      for (int i = 0; i < 64; ++i) {
-        sv[i] = (kbase + i < key_lim) ? sv[i] * scale_l2 : -INFINITY;
-        bm = fmaxf(bm, sv[i]);
-      }
-      const float mn = fmaxf(m, bm);
-      if (mn != -INFINITY) {
-        float add = 0.f;
+    for (int i = 0; i < 64; ++i) {
+      sv[i] = (kbase + i < key_lim) ? sv[i] * scale_l2 : -INFINITY;
+      bm = fmaxf(bm, sv[i]);
+    }
+    // P(w-1) and O are in use by PV(w-1) until it completes
+    if (w >= 1) {
+      if (!mbar_wait(bar_o, ph_o, err, kErrTimeoutMma)) ok_all = false;
+      ph_o ^= 1u;
+      __syncwarp();
+      tc_fence_after();
+    }
+    // V(w-1)'s buffer is free: prefetch V(w+1) (V(1) came with the prologue)
+    if (w >= 1) load_block(w + 1, 2);
+    cp_async_commit();
+    if (bm > m_used + kRescaleSlack) {
+      const float alpha = ex2_approx(m_used - bm);  // 0 while m_used = -inf
+      l *= alpha;
+      if (w >= 1) {
+        for (int c = 0; c < kHeadDim; c += 32) {
+          float o[32];
+          tmem_ld_32x32b_x32(tmem + t_lane + kTmemO + c, o);
 #pragma unroll
-        for (int i = 0; i < 64; ++i) add += ex2_approx(sv[i] - mn);
-        l = l * ex2_approx(m - mn) + add;
-        m = mn;
+          for (int i = 0; i < 32; ++i) o[i] *= alpha;
+          tmem_st_32x32b_x32(tmem + t_lane + kTmemO + c, o);
+        }
       }
-      if (j == nb - 1) inv_l = l > 0.f ? 1.0f / l : 0.f;
-    } else {
-      // P row -> bf16 -> swizzled [128 x 64] tile
+      m_used = bm;
+    }
+    {
+      // no visible key seen yet <=> m_used = -inf <=> every sv is -inf: use 0 so that 2^(-inf) = 0
+      const float mu = m_used == -INFINITY ? 0.f : m_used;
       uint8_t *prow = smem + kSmemP;
 #pragma unroll
       for (int cc = 0; cc < 8; ++cc) {
@@ -229,37 +262,40 @@ __global__ void __launch_bounds__(128, 1)
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const int i0 = cc * 8 + 2 * e;
-          const float p0 = (kbase + i0 < key_lim) ? ex2_approx(sv[i0] * scale_l2 - m) * inv_l : 0.f;
-          const float p1 = (kbase + i0 + 1 < key_lim) ? ex2_approx(sv[i0 + 1] * scale_l2 - m) * inv_l : 0.f;
+          const float p0 = ex2_approx(sv[i0] - mu), p1 = ex2_approx(sv[i0 + 1] - mu);
+          l += p0 + p1;
           const __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
           pk[e] = *reinterpret_cast<const uint32_t *>(&h2);
         }
         *reinterpret_cast<uint4 *>(prow + sw128_off(tid, cc)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
       }
-      fence_proxy_async_smem();
-      tc_fence_before();
-      ok_all = __syncthreads_and(ok_all);
-      tc_fence_after();
-      if (!ok_all) break;
-      if (tid == 0) {
-        const uint32_t vb = sbase + kSmemV0 + buf * kKVBytes;
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          tc_mma_bf16(tmem + kTmemO, smem_desc_k_sw128(sbase + kSmemP, kk * 32),
-                      smem_desc_mn_sw128(vb + kk * 2048, 64 * 128, 1024), idesc_o, (j | kk) != 0);
-        tc_commit(bar_o);
-      }
-      __syncwarp();
     }
+    // V(w) must have landed: all groups but the two just committed
+    cp_async_wait<2>();
+    fence_proxy_async_smem();
+    tc_fence_before();
+    ok_all = __syncthreads_and(ok_all);
+    tc_fence_after();
+    if (!ok_all) break;
+    if (tid == 0) {
+      const uint32_t vb = sbase + kSmemV0 + buf * kKVBytes;
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk)
+        tc_mma_bf16(tmem + kTmemO, smem_desc_k_sw128(sbase + kSmemP, kk * 32),
+                    smem_desc_mn_sw128(vb + kk * 2048, 64 * 128, 1024), idesc_o, (w | kk) != 0);
+      tc_commit(bar_o);
+    }
+    __syncwarp();
   }
   // last PV MMA
-  if (nitems > 0 && ok_all) {
+  if (nb > 0 && ok_all) {
     if (!mbar_wait(bar_o, ph_o, err, kErrTimeoutMma)) ok_all = false;
     __syncwarp();
   }
   cp_async_wait<0>();
   tc_fence_after();
   const bool write = __syncthreads_and(ok_all);
+  const float inv_l = l > 0.f ? 1.0f / l : 0.f;
   if (write) {
     if (nsplit == 1) {
       bf16 *dst = out + (size_t)tok * kQDim + head * kHeadDim;
@@ -270,7 +306,7 @@ __global__ void __launch_bounds__(128, 1)
           uint32_t pk[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
-            const __nv_bfloat162 h2 = __floats2bfloat162_rn(v[2 * e], v[2 * e + 1]);
+            const __nv_bfloat162 h2 = __floats2bfloat162_rn(v[2 * e] * inv_l, v[2 * e + 1] * inv_l);
             pk[e] = *reinterpret_cast<const uint32_t *>(&h2);
           }
           uint4 *d4 = reinterpret_cast<uint4 *>(dst + c);
@@ -292,11 +328,12 @@ __global__ void __launch_bounds__(128, 1)
         if (row_ok) {
           float4 *d4 = reinterpret_cast<float4 *>(part_o + prow * kHeadDim + c);
 #pragma unroll
-          for (int e = 0; e < 8; ++e) d4[e] = make_float4(v[4 * e], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]);
+          for (int e = 0; e < 8; ++e)
+            d4[e] = make_float4(v[4 * e] * inv_l, v[4 * e + 1] * inv_l, v[4 * e + 2] * inv_l, v[4 * e + 3] * inv_l);
         }
       }
       if (row_ok) {
-        part_ml[2 * prow] = m;
+        part_ml[2 * prow] = m_used;
         part_ml[2 * prow + 1] = l;
       }
     }
@@ -319,7 +356,7 @@ __global__ void __launch_bounds__(256) k_attn_combine(const float *part_o, const
   float M = -INFINITY;
   for (int s = 0; s < nsplit; ++s) {
     const size_t pr = ((size_t)b * nsplit + s) * rows_pad + qi;
-    M = fmaxf(M, part_ml[2 * pr]);
+    if (part_ml[2 * pr + 1] > 0.f) M = fmaxf(M, part_ml[2 * pr]);
   }
   float den = 0.f, acc[8];
 #pragma unroll
@@ -327,7 +364,7 @@ __global__ void __launch_bounds__(256) k_attn_combine(const float *part_o, const
   for (int s = 0; s < nsplit; ++s) {
     const size_t pr = ((size_t)b * nsplit + s) * rows_pad + qi;
     const float ms = part_ml[2 * pr], ls = part_ml[2 * pr + 1];
-    if (ls == 0.f) continue;
+    if (!(ls > 0.f)) continue;
     const float wgt = ls * ex2_approx(ms - M);
     den += wgt;
     const float *src = part_o + pr * kHeadDim;

@@ -261,13 +261,150 @@ __global__ void __launch_bounds__(128, 1)
   }
 }
 
+// Persistent variant (no split-K): one CTA per SM walks the output tiles
+// (row tile fastest, so concurrently running CTAs share weight tiles in L2).
+// Warp 0 = TMA producer, warp 1 = MMA issuer, warps 2..5 = epilogue.  Two TMEM
+// accumulators let the epilogue of one tile overlap the main loop of the next.
+template <int BN, int STAGES, int EPI>
+__global__ void __launch_bounds__(192, 1)
+    k_gemm_tc_persist(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, int a_row0,
+                      int M, int N, int nk, EpiArgs e, unsigned *err) {
+  using C = TcCfg<BN, STAGES>;
+  constexpr int kAcc = 2;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem + STAGES * C::kStage);
+  uint64_t *empty = full + STAGES;
+  uint64_t *acc_full = empty + STAGES;
+  uint64_t *acc_empty = acc_full + kAcc;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_empty + kAcc);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int mt = (M + 127) / 128, ntiles = mt * (N / BN);
+  if (*(volatile unsigned *)err != 0) return;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < kAcc; ++a) {
+      mbar_init(&acc_full[a], 1);
+      mbar_init(&acc_empty[a], 4);
+    }
+    fence_mbar_init();
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, kAcc * C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int it = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+        const int m0 = (t % mt) * 128, n0 = (t / mt) * BN;
+        for (int kb = 0; kb < nk; ++kb, ++it) {
+          const int s = it % STAGES;
+          const uint32_t round = it / STAGES;
+          if (!mbar_wait(&empty[s], (round & 1u) ^ 1u, err, kErrTimeoutProducer)) {
+            ok = false;
+            break;
+          }
+          uint8_t *a_dst = smem + s * C::kStage;
+          mbar_arrive_expect_tx(&full[s], C::kStage);
+          tma_load_2d(a_dst, &tmA, kb * 64, a_row0 + m0, &full[s]);
+          tma_load_2d(a_dst + C::kABytes, &tmB, kb * 64, n0, &full[s]);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(128, BN);
+      int it = 0, ti = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x, ++ti) {
+        const int a = ti % kAcc;
+        const uint32_t around = ti / kAcc;
+        if (!mbar_wait(&acc_empty[a], (around & 1u) ^ 1u, err, kErrTimeoutMma)) break;
+        tc_fence_after();
+        const uint32_t d = tmem + (uint32_t)(a * C::kTmemCols);
+        for (int kb = 0; kb < nk; ++kb, ++it) {
+          const int s = it % STAGES;
+          const uint32_t round = it / STAGES;
+          if (!mbar_wait(&full[s], round & 1u, err, kErrTimeoutMma)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_base = smem_u32(smem + s * C::kStage);
+          const uint32_t b_base = a_base + C::kABytes;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            tc_mma_bf16(d, smem_desc_k_sw128(a_base, kk * 32), smem_desc_k_sw128(b_base, kk * 32), idesc,
+                        (kb | kk) != 0);
+          tc_commit(&empty[s]);
+        }
+        tc_commit(&acc_full[a]);
+      }
+    }
+  } else {
+    // epilogue warps 2..5: TMEM lane quarter = warp % 4
+    const int q = warp & 3;
+    const uint32_t t_lane = (uint32_t)(q * 32) << 16;
+    int ti = 0;
+    for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++ti) {
+      const int a = ti % kAcc;
+      const uint32_t around = ti / kAcc;
+      const bool ok = mbar_wait(&acc_full[a], around & 1u, err, kErrTimeoutEpilogue);
+      __syncwarp();
+      if (!__all_sync(0xffffffffu, ok)) break;
+      tc_fence_after();
+      const int m0 = (t % mt) * 128, n0 = (t / mt) * BN;
+      const int r = m0 + q * 32 + lane;
+#pragma unroll 1
+      for (int c = 0; c < BN; c += 32) {
+        float v[32];
+        tmem_ld_32x32b_x32(tmem + (uint32_t)(a * C::kTmemCols) + t_lane + (uint32_t)c, v);
+        if (r < M) epilogue32<EPI>(e, r, n0 + c, v);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[a]);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kAcc * C::kTmemCols);
+  }
+}
+
 template <int BN, int STAGES, int EPI>
 static void launch_cfg(const CUtensorMap &tmA, const CUtensorMap &tmB, int a_row0, int M, int N, int K, int splits,
                        const EpiArgs &e, unsigned *err, cudaStream_t s) {
   using C = TcCfg<BN, STAGES>;
+  const int nk = K / 64;
+  if (splits == 1 && 2 * C::kTmemCols <= 512) {
+    auto kern = k_gemm_tc_persist<BN, STAGES, EPI>;
+    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int tiles = ((M + 127) / 128) * (N / BN);
+    kern<<<tiles < sms ? tiles : sms, 192, C::kSmem, s>>>(tmA, tmB, a_row0, M, N, nk, e, err);
+    return;
+  }
   auto kern = k_gemm_tc<BN, STAGES, EPI>;
   cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
-  const int nk = K / 64;
   const int kps = (nk + splits - 1) / splits;
   splits = (nk + kps - 1) / kps;
   dim3 grid((M + 127) / 128, N / BN, splits);
