@@ -54,10 +54,20 @@ __device__ __forceinline__ uint4 pack8_bf16(const float *v) {
   return make_uint4(p[0], p[1], p[2], p[3]);
 }
 
-// Epilogue of 32 consecutive output columns [n, n+32) of GEMM row r.
+// 1/sqrt(mean(h^2) + eps) of an output row from the producer's partial sums.
+__device__ __forceinline__ float row_rstd(const EpiArgs &e, int orow) {
+  float ss = 0.f;
+#pragma unroll
+  for (int t = 0; t < kNormSlots; ++t) ss += e.ss_in[(size_t)t * e.ss_ld + orow];
+  return 1.0f / sqrtf(ss / (float)kWidth + kRmsEps);
+}
+
+// Epilogue of 32 consecutive output columns [n, n+32) of GEMM row r.  Returns the
+// row's sum of squares over these columns for the fused-norm producers, else 0.
 template <int EPI>
-__device__ __forceinline__ void epilogue32(const EpiArgs &e, int r, int n, float (&v)[32]) {
+__device__ __forceinline__ float epilogue32(const EpiArgs &e, int r, int n, float (&v)[32]) {
   const int orow = e.out_row0 + r;
+  float ssq = 0.f;
   if constexpr (EPI == EPI_STORE_F32 || EPI == EPI_BIAS_F32 || EPI == EPI_RESID_F32) {
     float4 *dst = reinterpret_cast<float4 *>(e.out_f32 + (size_t)orow * e.ldo + n);
 #pragma unroll
@@ -71,6 +81,20 @@ __device__ __forceinline__ void epilogue32(const EpiArgs &e, int r, int n, float
         w.x += old.x; w.y += old.y; w.z += old.z; w.w += old.w;
       }
       dst[i] = w;
+      v[4 * i] = w.x; v[4 * i + 1] = w.y; v[4 * i + 2] = w.z; v[4 * i + 3] = w.w;
+    }
+    if constexpr (EPI != EPI_STORE_F32) {
+      if (e.gain) {  // fused RMSNorm producer: bf16(h * (1 + g)) and sum of h^2
+        float t[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          ssq = fmaf(v[i], v[i], ssq);
+          t[i] = v[i] * (1.0f + e.gain[n + i]);
+        }
+        uint4 *xd = reinterpret_cast<uint4 *>(e.xn_out + (size_t)orow * kWidth + n);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) xd[i] = pack8_bf16(t + 8 * i);
+      }
     }
   } else if constexpr (EPI == EPI_VEC_SILU) {
     float t[32];
@@ -83,6 +107,11 @@ __device__ __forceinline__ void epilogue32(const EpiArgs &e, int r, int n, float
     int b, j;
     row_to_bj_tc(orow, e.B, e.H, b, j);
     const float pos = (float)(e.nvalid[b] + j);
+    if (e.ss_in) {
+      const float rs = row_rstd(e, orow);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) v[i] *= rs;
+    }
 #pragma unroll
     for (int gi = 0; gi < 2; ++gi) {
       const int gc = (n >> 4) + gi;
@@ -114,6 +143,11 @@ __device__ __forceinline__ void epilogue32(const EpiArgs &e, int r, int n, float
       *reinterpret_cast<uint4 *>(dst + kHeadDim / 2) = pack8_bf16(hi);
     }
   } else if constexpr (EPI == EPI_GEGLU) {
+    if (e.ss_in) {
+      const float rs = row_rstd(e, orow);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) v[i] *= rs;
+    }
 #pragma unroll
     for (int gi = 0; gi < 2; ++gi) {
       const int f0 = ((n >> 4) + gi) * 8;
@@ -121,6 +155,21 @@ __device__ __forceinline__ void epilogue32(const EpiArgs &e, int r, int n, float
 #pragma unroll
       for (int w = 0; w < 8; ++w) a[w] = gelu_tanh_f(v[16 * gi + w]) * v[16 * gi + 8 + w];
       *reinterpret_cast<uint4 *>(e.out_bf16 + (size_t)orow * kMlp + f0) = pack8_bf16(a);
+    }
+  }
+  return ssq;
+}
+
+// After the last column chunk of a tile: store the row's partial sum of squares
+// into the tile's slot (and clear the unused slots once per row).
+template <int EPI>
+__device__ __forceinline__ void norm_partial_store(const EpiArgs &e, int r, int n0, int BN, int N, float ssq) {
+  if constexpr (EPI == EPI_BIAS_F32 || EPI == EPI_RESID_F32) {
+    if (e.gain && e.ss_out) {
+      const int orow = e.out_row0 + r;
+      e.ss_out[(size_t)(n0 / BN) * e.ss_ld + orow] = ssq;
+      if (n0 == 0)
+        for (int t = N / BN; t < kNormSlots; ++t) e.ss_out[(size_t)t * e.ss_ld + orow] = 0.f;
     }
   }
 }
@@ -203,12 +252,14 @@ __global__ void __launch_bounds__(128, 1)
   const uint32_t t_lane = (uint32_t)(warp * 32) << 16;
   if (all_ok) {
     if (splits == 1) {
+      float ssq = 0.f;
 #pragma unroll 1
       for (int c = 0; c < BN; c += 32) {
         float v[32];
         tmem_ld_32x32b_x32(tmem + t_lane + (uint32_t)c, v);
-        if (r < M) epilogue32<EPI>(e, r, n0 + c, v);
+        if (r < M) ssq += epilogue32<EPI>(e, r, n0 + c, v);
       }
+      if (r < M) norm_partial_store<EPI>(e, r, n0, BN, gridDim.y * BN, ssq);
     } else {
       const int tile = blockIdx.x * gridDim.y + blockIdx.y;
       float *mine = e.part + ((size_t)tile * splits + blockIdx.z) * (128 * BN) + (size_t)rr * BN;
@@ -233,6 +284,7 @@ __global__ void __launch_bounds__(128, 1)
         __threadfence();
         const float *base = e.part + (size_t)tile * splits * (128 * BN) + (size_t)rr * BN;
         if (r < M) {
+          float ssq = 0.f;
 #pragma unroll 1
           for (int c = 0; c < BN; c += 32) {
             float v[32];
@@ -246,8 +298,9 @@ __global__ void __launch_bounds__(128, 1)
                 v[4 * i] += t.x; v[4 * i + 1] += t.y; v[4 * i + 2] += t.z; v[4 * i + 3] += t.w;
               }
             }
-            epilogue32<EPI>(e, r, n0 + c, v);
+            ssq += epilogue32<EPI>(e, r, n0 + c, v);
           }
+          norm_partial_store<EPI>(e, r, n0, BN, gridDim.y * BN, ssq);
         }
         if (threadIdx.x == 0) e.counters[tile] = 0;  // ready for the next GEMM that uses it
       }
@@ -369,12 +422,14 @@ __global__ void __launch_bounds__(192, 1)
       tc_fence_after();
       const int m0 = (t % mt) * 128, n0 = (t / mt) * BN;
       const int r = m0 + q * 32 + lane;
+      float ssq = 0.f;
 #pragma unroll 1
       for (int c = 0; c < BN; c += 32) {
         float v[32];
         tmem_ld_32x32b_x32(tmem + (uint32_t)(a * C::kTmemCols) + t_lane + (uint32_t)c, v);
-        if (r < M) epilogue32<EPI>(e, r, n0 + c, v);
+        if (r < M) ssq += epilogue32<EPI>(e, r, n0 + c, v);
       }
+      if (r < M) norm_partial_store<EPI>(e, r, n0, BN, N, ssq);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&acc_empty[a]);

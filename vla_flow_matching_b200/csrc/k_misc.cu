@@ -80,43 +80,82 @@ void launch_time_vec(const TW *w_time, const float *bias, int num_steps, float *
   k_time_vec<TW><<<dim3(num_steps, kWidth / 32), 256, 0, s>>>(w_time, bias, num_steps, tvec);
 }
 
-// State token: h[b] = state_proj(state[b]) (`embed_suffix`).
+// State token: h[b] = state_proj(state[b]) (`embed_suffix`).  With `gain` set it
+// also produces the first layer's fused-RMSNorm inputs for the row: bf16(h*(1+g))
+// and the row's sum of h^2 in norm slot 0 (other slots zero).
 template <typename TW>
 __global__ void __launch_bounds__(256) k_state_embed(const CallPtrs *cp, const TW *w, const float *bias, int S,
-                                                      float *h) {
+                                                      float *h, const float *gain, bf16 *xn, float *ss,
+                                                      int ss_ld) {
   __shared__ float sv[64];
+  __shared__ float red[8];
   const int b = blockIdx.x;
   for (int i = threadIdx.x; i < S; i += blockDim.x) sv[i] = cp->state[(size_t)b * S + i];
   __syncthreads();
+  float ssq = 0.f;
   for (int n = threadIdx.x; n < kWidth; n += blockDim.x) {
     float acc = 0.f;
     for (int i = 0; i < S; ++i) acc = fmaf(to_f32(w[(size_t)n * S + i]), sv[i], acc);
-    h[(size_t)b * kWidth + n] = acc + bias[n];
+    const float hv = acc + bias[n];
+    h[(size_t)b * kWidth + n] = hv;
+    if (gain) {
+      ssq = fmaf(hv, hv, ssq);
+      xn[(size_t)b * kWidth + n] = __float2bfloat16_rn(hv * (1.0f + gain[n]));
+    }
+  }
+  if (gain) {
+    ssq = warp_sum(ssq);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ssq;
+    __syncthreads();
+    if (threadIdx.x < kNormSlots) {
+      float tot = 0.f;
+      if (threadIdx.x == 0)
+        for (int i = 0; i < 8; ++i) tot += red[i];
+      ss[(size_t)threadIdx.x * ss_ld + b] = tot;
+    }
   }
 }
 
 template <typename TW>
-void launch_state_embed(const CallPtrs *cp, const TW *w, const float *b, int B, int S, float *h, cudaStream_t s) {
-  k_state_embed<TW><<<B, 256, 0, s>>>(cp, w, b, S, h);
+void launch_state_embed(const CallPtrs *cp, const TW *w, const float *b, int B, int S, float *h, cudaStream_t s,
+                        const float *gain, bf16 *xn, float *ss, int ss_ld) {
+  k_state_embed<TW><<<B, 256, 0, s>>>(cp, w, b, S, h, gain, xn, ss, ss_ld);
 }
 
 // Action tokens: out[i] = action_in_proj(x[i]) for every (sample, horizon) row.
+// A block takes 16 rows; each thread keeps the weight rows of its 4 output
+// features in registers (read once) and reuses them for all 16 rows.
+constexpr int kActRows = 16;
 template <typename TW, typename T>
-__global__ void __launch_bounds__(256) k_action_in(const float *x, const TW *w, const float *bias, int A, T *out) {
-  __shared__ float xv[64];
-  const int r = blockIdx.x;
-  for (int i = threadIdx.x; i < A; i += blockDim.x) xv[i] = x[(size_t)r * A + i];
+__global__ void __launch_bounds__(256) k_action_in(const float *x, const TW *w, const float *bias, int rows, int A,
+                                                    T *out) {
+  __shared__ float xv[kActRows][64];
+  const int r0 = blockIdx.x * kActRows;
+  for (int e = threadIdx.x; e < kActRows * A; e += blockDim.x) {
+    const int r = e / A, i = e % A;
+    xv[r][i] = (r0 + r < rows) ? x[(size_t)(r0 + r) * A + i] : 0.f;
+  }
   __syncthreads();
-  for (int n = threadIdx.x; n < kWidth; n += blockDim.x) {
-    float acc = 0.f;
-    for (int i = 0; i < A; ++i) acc = fmaf(to_f32(w[(size_t)n * A + i]), xv[i], acc);
-    out[(size_t)r * kWidth + n] = from_f32<T>(acc + bias[n]);
+#pragma unroll 1
+  for (int o = 0; o < kWidth / 256; ++o) {
+    const int n = threadIdx.x + 256 * o;
+    float wr[64];
+#pragma unroll
+    for (int i = 0; i < 64; ++i) wr[i] = i < A ? to_f32(w[(size_t)n * A + i]) : 0.f;
+    const float bn = bias[n];
+    for (int r = 0; r < kActRows && r0 + r < rows; ++r) {
+      float acc = 0.f;
+#pragma unroll
+      for (int i = 0; i < 64; ++i)
+        if (i < A) acc = fmaf(wr[i], xv[r][i], acc);
+      out[(size_t)(r0 + r) * kWidth + n] = from_f32<T>(acc + bn);
+    }
   }
 }
 
 template <typename TW, typename T>
 void launch_action_in(const float *x, const TW *w, const float *b, int rows, int A, T *out, cudaStream_t s) {
-  k_action_in<TW, T><<<rows, 256, 0, s>>>(x, w, b, A, out);
+  k_action_in<TW, T><<<(rows + kActRows - 1) / kActRows, 256, 0, s>>>(x, w, b, rows, A, out);
 }
 
 // Gemma RMSNorm: out = h * (1/sqrt(mean(h^2) + 1e-6)) * (1 + gain), one warp per row.
@@ -282,9 +321,9 @@ void launch_delay_ns(unsigned long long ns, cudaStream_t s) { k_delay<<<1, 1, 0,
 template void launch_time_vec<float>(const float *, const float *, int, float *, cudaStream_t);
 template void launch_time_vec<bf16>(const bf16 *, const float *, int, float *, cudaStream_t);
 template void launch_state_embed<float>(const CallPtrs *, const float *, const float *, int, int, float *,
-                                        cudaStream_t);
+                                        cudaStream_t, const float *, bf16 *, float *, int);
 template void launch_state_embed<bf16>(const CallPtrs *, const bf16 *, const float *, int, int, float *,
-                                       cudaStream_t);
+                                       cudaStream_t, const float *, bf16 *, float *, int);
 template void launch_action_in<float, float>(const float *, const float *, const float *, int, int, float *,
                                              cudaStream_t);
 template void launch_action_in<bf16, bf16>(const float *, const bf16 *, const float *, int, int, bf16 *,

@@ -53,7 +53,18 @@ struct EpiArgs {
   // split-K partial tiles and per-tile arrival counters (zero between GEMMs)
   float *part = nullptr;
   int *counters = nullptr;
+  // Fused RMSNorm (bf16 mode).  Producers (EPI_BIAS_F32 / EPI_RESID_F32 with
+  // gain != null) also write xn_out = bf16(h * (1 + gain)) and, per output column
+  // tile t, ss_out[t * ss_ld + row] = sum of h^2 over the tile's columns (slots
+  // t >= N/BN are zeroed).  Consumers (EPI_QKV_ROPE / EPI_GEGLU with ss_in) scale
+  // the accumulator by 1/sqrt(sum_{t<kNormSlots} ss_in[t*ss_ld+row] / 1024 + eps).
+  const float *gain = nullptr;
+  bf16 *xn_out = nullptr;
+  float *ss_out = nullptr;
+  const float *ss_in = nullptr;
+  int ss_ld = 0;
 };
+constexpr int kNormSlots = 16;
 
 // Tile width and K split of one tcgen05 GEMM launch.
 struct TcPlan {
@@ -78,7 +89,8 @@ void launch_prep_mask(const CallPtrs *cp, int B, int P, int *nvalid, int *vidx, 
 template <typename TW>
 void launch_time_vec(const TW *w_time, const float *bias, int num_steps, float *tvec, cudaStream_t s);
 template <typename TW>
-void launch_state_embed(const CallPtrs *cp, const TW *w, const float *b, int B, int S, float *h, cudaStream_t s);
+void launch_state_embed(const CallPtrs *cp, const TW *w, const float *b, int B, int S, float *h, cudaStream_t s,
+                        const float *gain = nullptr, bf16 *xn = nullptr, float *ss = nullptr, int ss_ld = 0);
 template <typename TW, typename T>
 void launch_action_in(const float *x, const TW *w, const float *b, int rows, int A, T *out, cudaStream_t s);
 template <typename T>

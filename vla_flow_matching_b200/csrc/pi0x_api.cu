@@ -101,6 +101,8 @@ struct Workspace {
   float *part;   // split-KV attention partials (bf16 mode)
   float *gpart;  // split-K GEMM partial tiles (bf16 mode)
   int *counters; // split-K per-tile arrival counters
+  float *ss_a, *ss_m;  // fused RMSNorm partial sums of squares, kNormSlots x ss_ld (bf16 mode)
+  int ss_ld = 0;
   void *xn, *q, *ks, *vs, *att, *act, *a_emb, *u_emb;
   // host-input staging (device side), allocated lazily
   Arena stage;
@@ -277,6 +279,9 @@ int ensure_workspace(pi0x_handle *h, int B, int P, int N) {
   const size_t gpart_floats = h->bf16 ? (size_t)148 * 128 * 64 : 0;
   add(4 * gpart_floats);
   add(4 * 1024);
+  const size_t ss_floats = h->bf16 ? (size_t)kNormSlots * Rp : 0;
+  add(4 * ss_floats);
+  add(4 * ss_floats);
   add(es * Rp * kWidth);
   add(es * Rp * kQDim);
   add(es * (size_t)L * Rp * kHeadDim);
@@ -300,6 +305,9 @@ int ensure_workspace(pi0x_handle *h, int B, int P, int N) {
   ws.raw = (float *)ws.arena.take(4 * raw_floats);
   ws.gpart = (float *)ws.arena.take(4 * gpart_floats);
   ws.counters = (int *)ws.arena.take(4 * 1024);
+  ws.ss_a = (float *)ws.arena.take(4 * ss_floats);
+  ws.ss_m = (float *)ws.arena.take(4 * ss_floats);
+  ws.ss_ld = (int)Rp;
   ws.xn = ws.arena.take(es * Rp * kWidth);
   ws.q = ws.arena.take(es * Rp * kQDim);
   ws.ks = ws.arena.take(es * (size_t)L * Rp * kHeadDim);
@@ -428,8 +436,14 @@ int enqueue_loop(pi0x_handle *h, int B, int P, int N, cudaStream_t s) {
     const int step0 = (k == 0);
     const int row0 = step0 ? 0 : B;
     const int M = R - row0;
-    if (step0)
-      RUN(PI0X_K_EMBED, launch_state_embed<T>(h->d_ptrs, (const T *)h->state_w, h->state_b, B, c.state_dim, ws.h, s));
+    if (step0) {
+      if (tc)
+        RUN(PI0X_K_EMBED, launch_state_embed<T>(h->d_ptrs, (const T *)h->state_w, h->state_b, B, c.state_dim, ws.h,
+                                                s, h->layer[0].in_norm, (bf16 *)xn, ws.ss_a, ws.ss_ld));
+      else
+        RUN(PI0X_K_EMBED, launch_state_embed<T>(h->d_ptrs, (const T *)h->state_w, h->state_b, B, c.state_dim, ws.h,
+                                                s));
+    }
     RUN(PI0X_K_EMBED, launch_action_in<T, T>(ws.xw, (const T *)h->ain_w, h->ain_b, BH, A, aemb, s));
     GemmOut o_u{uemb, kWidth, 0, ws.tvec + (size_t)k * kWidth};
     GemmOut o_h{ws.h, kWidth, B, h->tout_b};
@@ -444,6 +458,10 @@ int enqueue_loop(pi0x_handle *h, int B, int P, int N, cudaStream_t s) {
       eh.ldo = kWidth;
       eh.out_row0 = B;
       eh.vec = h->tout_b;
+      eh.gain = h->layer[0].in_norm;   // fused input norm of layer 0
+      eh.xn_out = (bf16 *)xn;
+      eh.ss_out = ws.ss_a;
+      eh.ss_ld = ws.ss_ld;
       RUN(PI0X_K_GEMM, gemm(EPI_BIAS_F32, ws.m_uemb, h->g_tout, 0, BH, eh));
     } else {
       RUN(PI0X_K_GEMM, launch_gemm_simt<float>((const float *)aemb, kWidth, (const float *)h->tin_a, kWidth, BH, kWidth, kWidth,
@@ -454,14 +472,17 @@ int enqueue_loop(pi0x_handle *h, int B, int P, int N, cudaStream_t s) {
     for (int l = 0; l < L; ++l) {
       const LayerW &lw = h->layer[l];
       T *ks = (T *)ws.ks + (size_t)l * kv_stride, *vs = (T *)ws.vs + (size_t)l * kv_stride;
-      RUN(PI0X_K_NORM, launch_rmsnorm<T>(ws.h, row0, M, lw.in_norm, xn, s));
+      if (!tc) RUN(PI0X_K_NORM, launch_rmsnorm<T>(ws.h, row0, M, lw.in_norm, xn, s));
       GemmOut o_raw{ws.raw, kQkvDim, row0, nullptr};
       if (tc) {
+        // xn holds h*(1+g_in) from the producer; rstd is applied in this epilogue
         EpiArgs eq = ebase;
         eq.out_row0 = row0;
         eq.q = (bf16 *)q;
         eq.ks = (bf16 *)ks;
         eq.vs = (bf16 *)vs;
+        eq.ss_in = ws.ss_a;
+        eq.ss_ld = ws.ss_ld;
         RUN(PI0X_K_GEMM, gemm(EPI_QKV_ROPE, ws.m_xn, h->g_qkv[l], row0, M, eq));
       } else {
         RUN(PI0X_K_GEMM, launch_gemm_simt<float>((const float *)xn + (size_t)row0 * kWidth, kWidth, (const float *)lw.qkv, kWidth,
@@ -482,17 +503,24 @@ int enqueue_loop(pi0x_handle *h, int B, int P, int N, cudaStream_t s) {
       eres.ldo = kWidth;
       eres.out_row0 = row0;
       if (tc) {
-        RUN(PI0X_K_GEMM, gemm(EPI_RESID_F32, ws.m_att, h->g_o[l], row0, M, eres));
+        EpiArgs eo = eres;  // residual add + fused post-attention norm inputs
+        eo.gain = lw.post_norm;
+        eo.xn_out = (bf16 *)xn;
+        eo.ss_out = ws.ss_m;
+        eo.ss_ld = ws.ss_ld;
+        RUN(PI0X_K_GEMM, gemm(EPI_RESID_F32, ws.m_att, h->g_o[l], row0, M, eo));
       } else {
         RUN(PI0X_K_GEMM, launch_gemm_simt<float>((const float *)att + (size_t)row0 * kQDim, kQDim, (const float *)lw.o, kQDim, M,
                                 kWidth, kQDim, EPI_RESID_F32, o_res, s));
       }
-      RUN(PI0X_K_NORM, launch_rmsnorm<T>(ws.h, row0, M, lw.post_norm, xn, s));
+      if (!tc) RUN(PI0X_K_NORM, launch_rmsnorm<T>(ws.h, row0, M, lw.post_norm, xn, s));
       GemmOut o_gu{ws.raw, 2 * kMlp, row0, nullptr};
       if (tc) {
         EpiArgs eg = ebase;
         eg.out_bf16 = (bf16 *)act;
         eg.out_row0 = row0;
+        eg.ss_in = ws.ss_m;
+        eg.ss_ld = ws.ss_ld;
         RUN(PI0X_K_GEMM, gemm(EPI_GEGLU, ws.m_xn, h->g_gu[l], row0, M, eg));
       } else {
         RUN(PI0X_K_GEMM, launch_gemm_simt<float>((const float *)xn + (size_t)row0 * kWidth, kWidth, (const float *)lw.gu, kWidth, M,
@@ -500,7 +528,14 @@ int enqueue_loop(pi0x_handle *h, int B, int P, int N, cudaStream_t s) {
         RUN(PI0X_K_GEGLU, launch_geglu<T>(ws.raw, row0, M, act, s));
       }
       if (tc) {
-        RUN(PI0X_K_GEMM, gemm(EPI_RESID_F32, ws.m_act, h->g_down[l], row0, M, eres));
+        EpiArgs ed = eres;  // residual add + fused input norm of the next layer
+        if (l + 1 < L) {
+          ed.gain = h->layer[l + 1].in_norm;
+          ed.xn_out = (bf16 *)xn;
+          ed.ss_out = ws.ss_a;
+          ed.ss_ld = ws.ss_ld;
+        }
+        RUN(PI0X_K_GEMM, gemm(EPI_RESID_F32, ws.m_act, h->g_down[l], row0, M, ed));
       } else {
         RUN(PI0X_K_GEMM, launch_gemm_simt<float>((const float *)act + (size_t)row0 * kMlp, kMlp, (const float *)lw.down, kMlp, M,
                                 kWidth, kMlp, EPI_RESID_F32, o_res, s));
@@ -908,8 +943,10 @@ long pi0x_launch_count(const pi0x_handle *h, int B, int P, int num_steps) {
   Geo g{B, (int)H, h->cfg.action_dim, h->cfg.state_dim, P, B + B * (int)H};
   long n = 3 + 1;  // mask prep, time-MLP half, x_1 copy; state token embed
   for (int k = 0; k < num_steps; ++k) {
-    // action_in, two time-MLP GEMMs, 9 kernels per layer, final norm + Euler
-    long per_layer = 9;
+    // action_in, two time-MLP GEMMs, the layers, final norm + Euler.  fp32 mode: 2 norms,
+    // 2 GEMMs + RoPE, attention, O GEMM, GeGLU, down GEMM; bf16 mode fuses norms, RoPE
+    // and GeGLU into the GEMMs (4 GEMMs + attention [+ split-KV combine]).
+    long per_layer = h->bf16 ? 5 : 9;
     if (h->bf16 && attn_tc_splits(g, k == 0, P + 1 + (int)H) > 1) per_layer += 1;  // split-KV combine
     n += 3 + L * per_layer + 1;
   }
