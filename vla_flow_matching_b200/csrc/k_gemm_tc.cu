@@ -62,10 +62,20 @@ __device__ __forceinline__ float row_rstd(const EpiArgs &e, int orow) {
   return 1.0f / sqrtf(ss / (float)kWidth + kRmsEps);
 }
 
-// Epilogue of 32 consecutive output columns [n, n+32) of GEMM row r.  Returns the
-// row's sum of squares over these columns for the fused-norm producers, else 0.
+// Fused-norm scale of GEMM row r for the consumer epilogues (1 otherwise).
 template <int EPI>
-__device__ __forceinline__ float epilogue32(const EpiArgs &e, int r, int n, float (&v)[32]) {
+__device__ __forceinline__ float consumer_rstd(const EpiArgs &e, int r) {
+  if constexpr (EPI == EPI_QKV_ROPE || EPI == EPI_GEGLU) {
+    if (e.ss_in) return row_rstd(e, e.out_row0 + r);
+  }
+  return 1.f;
+}
+
+// Epilogue of 32 consecutive output columns [n, n+32) of GEMM row r (`rs` from
+// consumer_rstd).  Returns the row's sum of squares over these columns for the
+// fused-norm producers, else 0.
+template <int EPI>
+__device__ __forceinline__ float epilogue32(const EpiArgs &e, int r, int n, float (&v)[32], float rs) {
   const int orow = e.out_row0 + r;
   float ssq = 0.f;
   if constexpr (EPI == EPI_STORE_F32 || EPI == EPI_BIAS_F32 || EPI == EPI_RESID_F32) {
@@ -106,12 +116,9 @@ __device__ __forceinline__ float epilogue32(const EpiArgs &e, int r, int n, floa
   } else if constexpr (EPI == EPI_QKV_ROPE) {
     int b, j;
     row_to_bj_tc(orow, e.B, e.H, b, j);
-    const float pos = (float)(e.nvalid[b] + j);
-    if (e.ss_in) {
-      const float rs = row_rstd(e, orow);
+    const int pos = e.nvalid[b] + j;
 #pragma unroll
-      for (int i = 0; i < 32; ++i) v[i] *= rs;
-    }
+    for (int i = 0; i < 32; ++i) v[i] *= rs;
 #pragma unroll
     for (int gi = 0; gi < 2; ++gi) {
       const int gc = (n >> 4) + gi;
@@ -123,13 +130,20 @@ __device__ __forceinline__ float epilogue32(const EpiArgs &e, int r, int n, floa
         hi[w] = v[16 * gi + 8 + w];
       }
       if (hd < kHeads + 1) {
+        // (cos, sin) of fp32(pos) * inv_freq[i], tabulated per call (k_rope_table)
+        const float4 *tab =
+            reinterpret_cast<const float4 *>(e.rope_tab + ((size_t)pos * (kHeadDim / 2) + ib) * 2);
 #pragma unroll
-        for (int w = 0; w < 8; ++w) {
-          float sn, cs;
-          sincosf(pos * e.inv_freq[ib + w], &sn, &cs);
-          const float a = lo[w], bb = hi[w];
-          lo[w] = a * cs - bb * sn;
-          hi[w] = bb * cs + a * sn;
+        for (int w2 = 0; w2 < 4; ++w2) {
+          const float4 t = tab[w2];  // (cos, sin) of pairs ib+2*w2, ib+2*w2+1
+#pragma unroll
+          for (int h2 = 0; h2 < 2; ++h2) {
+            const int w = 2 * w2 + h2;
+            const float cs = h2 ? t.z : t.x, sn = h2 ? t.w : t.y;
+            const float a = lo[w], bb = hi[w];
+            lo[w] = a * cs - bb * sn;
+            hi[w] = bb * cs + a * sn;
+          }
         }
       }
       bf16 *dst;
@@ -143,11 +157,8 @@ __device__ __forceinline__ float epilogue32(const EpiArgs &e, int r, int n, floa
       *reinterpret_cast<uint4 *>(dst + kHeadDim / 2) = pack8_bf16(hi);
     }
   } else if constexpr (EPI == EPI_GEGLU) {
-    if (e.ss_in) {
-      const float rs = row_rstd(e, orow);
 #pragma unroll
-      for (int i = 0; i < 32; ++i) v[i] *= rs;
-    }
+    for (int i = 0; i < 32; ++i) v[i] *= rs;
 #pragma unroll
     for (int gi = 0; gi < 2; ++gi) {
       const int f0 = ((n >> 4) + gi) * 8;
@@ -253,11 +264,12 @@ __global__ void __launch_bounds__(128, 1)
   if (all_ok) {
     if (splits == 1) {
       float ssq = 0.f;
+      const float rs = r < M ? consumer_rstd<EPI>(e, r) : 1.f;
 #pragma unroll 1
       for (int c = 0; c < BN; c += 32) {
         float v[32];
         tmem_ld_32x32b_x32(tmem + t_lane + (uint32_t)c, v);
-        if (r < M) ssq += epilogue32<EPI>(e, r, n0 + c, v);
+        if (r < M) ssq += epilogue32<EPI>(e, r, n0 + c, v, rs);
       }
       if (r < M) norm_partial_store<EPI>(e, r, n0, BN, gridDim.y * BN, ssq);
     } else {
@@ -285,6 +297,7 @@ __global__ void __launch_bounds__(128, 1)
         const float *base = e.part + (size_t)tile * splits * (128 * BN) + (size_t)rr * BN;
         if (r < M) {
           float ssq = 0.f;
+          const float rs = consumer_rstd<EPI>(e, r);
 #pragma unroll 1
           for (int c = 0; c < BN; c += 32) {
             float v[32];
@@ -298,7 +311,7 @@ __global__ void __launch_bounds__(128, 1)
                 v[4 * i] += t.x; v[4 * i + 1] += t.y; v[4 * i + 2] += t.z; v[4 * i + 3] += t.w;
               }
             }
-            ssq += epilogue32<EPI>(e, r, n0 + c, v);
+            ssq += epilogue32<EPI>(e, r, n0 + c, v, rs);
           }
           norm_partial_store<EPI>(e, r, n0, BN, gridDim.y * BN, ssq);
         }
@@ -423,11 +436,12 @@ __global__ void __launch_bounds__(192, 1)
       const int m0 = (t % mt) * 128, n0 = (t / mt) * BN;
       const int r = m0 + q * 32 + lane;
       float ssq = 0.f;
+      const float rs = r < M ? consumer_rstd<EPI>(e, r) : 1.f;
 #pragma unroll 1
       for (int c = 0; c < BN; c += 32) {
         float v[32];
         tmem_ld_32x32b_x32(tmem + (uint32_t)(a * C::kTmemCols) + t_lane + (uint32_t)c, v);
-        if (r < M) ssq += epilogue32<EPI>(e, r, n0 + c, v);
+        if (r < M) ssq += epilogue32<EPI>(e, r, n0 + c, v, rs);
       }
       if (r < M) norm_partial_store<EPI>(e, r, n0, BN, N, ssq);
       tc_fence_before();

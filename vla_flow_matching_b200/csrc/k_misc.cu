@@ -123,8 +123,8 @@ void launch_state_embed(const CallPtrs *cp, const TW *w, const float *b, int B, 
 }
 
 // Action tokens: out[i] = action_in_proj(x[i]) for every (sample, horizon) row.
-// A block takes 16 rows; each thread keeps the weight rows of its 4 output
-// features in registers (read once) and reuses them for all 16 rows.
+// Block (rows r0..r0+15, features 256*blockIdx.y..+255): each thread keeps the
+// weight row of its output feature in registers and reuses it for the 16 rows.
 constexpr int kActRows = 16;
 template <typename TW, typename T>
 __global__ void __launch_bounds__(256) k_action_in(const float *x, const TW *w, const float *bias, int rows, int A,
@@ -136,26 +136,38 @@ __global__ void __launch_bounds__(256) k_action_in(const float *x, const TW *w, 
     xv[r][i] = (r0 + r < rows) ? x[(size_t)(r0 + r) * A + i] : 0.f;
   }
   __syncthreads();
-#pragma unroll 1
-  for (int o = 0; o < kWidth / 256; ++o) {
-    const int n = threadIdx.x + 256 * o;
-    float wr[64];
+  const int n = blockIdx.y * 256 + threadIdx.x;
+  float wr[64];
 #pragma unroll
-    for (int i = 0; i < 64; ++i) wr[i] = i < A ? to_f32(w[(size_t)n * A + i]) : 0.f;
-    const float bn = bias[n];
-    for (int r = 0; r < kActRows && r0 + r < rows; ++r) {
-      float acc = 0.f;
+  for (int i = 0; i < 64; ++i) wr[i] = i < A ? to_f32(w[(size_t)n * A + i]) : 0.f;
+  const float bn = bias[n];
+  for (int r = 0; r < kActRows && r0 + r < rows; ++r) {
+    float acc = 0.f;
 #pragma unroll
-      for (int i = 0; i < 64; ++i)
-        if (i < A) acc = fmaf(wr[i], xv[r][i], acc);
-      out[(size_t)(r0 + r) * kWidth + n] = from_f32<T>(acc + bn);
-    }
+    for (int i = 0; i < 64; ++i)
+      if (i < A) acc = fmaf(wr[i], xv[r][i], acc);
+    out[(size_t)(r0 + r) * kWidth + n] = from_f32<T>(acc + bn);
   }
 }
 
 template <typename TW, typename T>
 void launch_action_in(const float *x, const TW *w, const float *b, int rows, int A, T *out, cudaStream_t s) {
-  k_action_in<TW, T><<<(rows + kActRows - 1) / kActRows, 256, 0, s>>>(x, w, b, rows, A, out);
+  k_action_in<TW, T><<<dim3((rows + kActRows - 1) / kActRows, kWidth / 256), 256, 0, s>>>(x, w, b, rows, A, out);
+}
+
+// RoPE table for the fused QKV epilogue: tab[p][i] = (cos, sin)(fp32(p) * inv_freq[i])
+// for every position a call can use, with the accurate CUDA sincosf.
+__global__ void k_rope_table(const float *inv_freq, int npos, float *tab) {
+  const int i = threadIdx.x;  // 128 pairs
+  for (int p = blockIdx.x; p < npos; p += gridDim.x) {
+    float sn, cs;
+    sincosf((float)p * inv_freq[i], &sn, &cs);
+    tab[((size_t)p * (kHeadDim / 2) + i) * 2] = cs;
+    tab[((size_t)p * (kHeadDim / 2) + i) * 2 + 1] = sn;
+  }
+}
+void launch_rope_table(const float *inv_freq, int npos, float *tab, cudaStream_t s) {
+  k_rope_table<<<npos < 1024 ? npos : 1024, kHeadDim / 2, 0, s>>>(inv_freq, npos, tab);
 }
 
 // Gemma RMSNorm: out = h * (1/sqrt(mean(h^2) + 1e-6)) * (1 + gain), one warp per row.

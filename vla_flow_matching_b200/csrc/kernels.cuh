@@ -63,6 +63,8 @@ struct EpiArgs {
   float *ss_out = nullptr;
   const float *ss_in = nullptr;
   int ss_ld = 0;
+  // EPI_QKV_ROPE: (cos, sin) pairs of fp32(pos) * inv_freq[i], [pos][128] (k_rope_table)
+  const float *rope_tab = nullptr;
 };
 constexpr int kNormSlots = 16;
 
@@ -104,6 +106,7 @@ void launch_final_euler(const float *h, const Geo &g, const float *gain, const f
                         float dt, float *x, const CallPtrs *cp, int last, cudaStream_t s);
 void launch_copy_x1(const CallPtrs *cp, int n, float *x, cudaStream_t s);
 void launch_delay_ns(unsigned long long ns, cudaStream_t s);
+void launch_rope_table(const float *inv_freq, int npos, float *tab, cudaStream_t s);
 
 // ---- attention (k_attn.cu) ----
 template <typename T>

@@ -103,6 +103,7 @@ struct Workspace {
   int *counters; // split-K per-tile arrival counters
   float *ss_a, *ss_m;  // fused RMSNorm partial sums of squares, kNormSlots x ss_ld (bf16 mode)
   int ss_ld = 0;
+  float *rope_tab;     // (cos, sin) per position and pair (bf16 mode)
   void *xn, *q, *ks, *vs, *att, *act, *a_emb, *u_emb;
   // host-input staging (device side), allocated lazily
   Arena stage;
@@ -282,6 +283,9 @@ int ensure_workspace(pi0x_handle *h, int B, int P, int N) {
   const size_t ss_floats = h->bf16 ? (size_t)kNormSlots * Rp : 0;
   add(4 * ss_floats);
   add(4 * ss_floats);
+  // positions 0 .. P + H (n_b <= P), 128 (cos, sin) pairs each
+  const size_t rope_floats = h->bf16 ? (size_t)(nP + H + 1) * (kHeadDim / 2) * 2 : 0;
+  add(4 * rope_floats);
   add(es * Rp * kWidth);
   add(es * Rp * kQDim);
   add(es * (size_t)L * Rp * kHeadDim);
@@ -308,6 +312,7 @@ int ensure_workspace(pi0x_handle *h, int B, int P, int N) {
   ws.ss_a = (float *)ws.arena.take(4 * ss_floats);
   ws.ss_m = (float *)ws.arena.take(4 * ss_floats);
   ws.ss_ld = (int)Rp;
+  ws.rope_tab = (float *)ws.arena.take(4 * rope_floats);
   ws.xn = ws.arena.take(es * Rp * kWidth);
   ws.q = ws.arena.take(es * Rp * kQDim);
   ws.ks = ws.arena.take(es * (size_t)L * Rp * kHeadDim);
@@ -423,6 +428,7 @@ int enqueue_loop(pi0x_handle *h, int B, int P, int N, cudaStream_t s) {
   ebase.H = H;
   ebase.part = ws.gpart;
   ebase.counters = ws.counters;
+  ebase.rope_tab = ws.rope_tab;
   auto gemm = [&](int epi, const CUtensorMap &tmA, const TcWeight &w, int a_row0, int M, const EpiArgs &e) {
     const TcPlan p = plan_gemm_tc(M, w.N, w.K);
     launch_gemm_tc(epi, tmA, w.map(p.bn), p, a_row0, M, w.N, w.K, e, h->d_err, s);
@@ -431,6 +437,7 @@ int enqueue_loop(pi0x_handle *h, int B, int P, int N, cudaStream_t s) {
   RUN(PI0X_K_PREP, launch_prep_mask(h->d_ptrs, B, P, ws.nvalid, ws.vidx, s));
   RUN(PI0X_K_PREP, launch_time_vec<T>((const T *)h->tin_t, h->tin_b, N, ws.tvec, s));
   RUN(PI0X_K_PREP, launch_copy_x1(h->d_ptrs, BH * A, ws.xw, s));
+  if (tc) RUN(PI0X_K_PREP, launch_rope_table(h->inv_freq, P + H + 1, ws.rope_tab, s));
 
   for (int k = 0; k < N; ++k) {
     const int step0 = (k == 0);
@@ -941,7 +948,7 @@ long pi0x_launch_count(const pi0x_handle *h, int B, int P, int num_steps) {
   if (!h || B < 1 || P < 0 || num_steps < 1) return -1;
   const long L = h->cfg.depth, H = h->cfg.horizon;
   Geo g{B, (int)H, h->cfg.action_dim, h->cfg.state_dim, P, B + B * (int)H};
-  long n = 3 + 1;  // mask prep, time-MLP half, x_1 copy; state token embed
+  long n = 3 + 1 + (h->bf16 ? 1 : 0);  // mask prep, time-MLP half, x_1 copy; state embed; RoPE table
   for (int k = 0; k < num_steps; ++k) {
     // action_in, two time-MLP GEMMs, the layers, final norm + Euler.  fp32 mode: 2 norms,
     // 2 GEMMs + RoPE, attention, O GEMM, GeGLU, down GEMM; bf16 mode fuses norms, RoPE
