@@ -230,6 +230,15 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
          | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
+// ---- programmatic dependent launch -----------------------------------------------
+// Kernels are launched with programmatic stream serialization: a kernel may start
+// while the previous one still runs.  pdl_wait() blocks until the previous kernel
+// has completed and its writes are visible; every thread calls it before touching
+// data produced upstream.  pdl_trigger() lets the next kernel start launching.
+// Both are no-ops for a normal launch.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ---- math ----------------------------------------------------------------------
 __device__ __forceinline__ float gelu_tanh_f(float x) {
   const float k = 0.7978845608028654f;  // sqrt(2/pi)

@@ -22,6 +22,8 @@ template <typename T>
 __global__ void __launch_bounds__(128) k_attn_simt(const T *q, const T *ks, const T *vs, const CallPtrs *cp,
                                                     int layer, const int *nvalid, const int *vidx, Geo g,
                                                     int step0, T *out) {
+  pdl_wait();
+  pdl_trigger();
   extern __shared__ float sm[];
   float *Ks = sm;                                  // [32][257]
   float *Vs = Ks + kAttnKeys * (kHeadDim + 1);     // [32][256]
@@ -126,7 +128,7 @@ void launch_attention(const T *q, const T *ks, const T *vs, const CallPtrs *cp, 
   }
   const int Tq = step0 ? g.H + 1 : g.H;
   dim3 grid(g.B, kHeads, (Tq + kAttnQ - 1) / kAttnQ);
-  k_attn_simt<T><<<grid, 128, kAttnSmem, s>>>(q, ks, vs, cp, layer, nvalid, vidx, g, step0, out);
+  launch_pdl(k_attn_simt<T>, grid, 128, kAttnSmem, s, q, ks, vs, cp, layer, nvalid, vidx, g, step0, out);
 }
 
 template void launch_attention<float>(const float *, const float *, const float *, const CallPtrs *, int,

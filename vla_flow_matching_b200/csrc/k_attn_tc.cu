@@ -55,6 +55,8 @@ __global__ void __launch_bounds__(128, 1)
     k_attn_tc(const bf16 *q, const bf16 *ks, const bf16 *vs, const CallPtrs *cp, int layer, const int *nvalid,
               const int *vidx, Geo g, int step0, int blocks_per_split, bf16 *out, float *part_o, float *part_ml,
               unsigned *err) {
+  pdl_wait();
+  pdl_trigger();
   if (*(volatile unsigned *)err != 0) return;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -349,6 +351,8 @@ __global__ void __launch_bounds__(128, 1)
 // Merge split-KV partials: O = sum_s w_s O_s with w_s = l_s 2^(m_s - M) / sum_t l_t 2^(m_t - M).
 __global__ void __launch_bounds__(256) k_attn_combine(const float *part_o, const float *part_ml, Geo g, int step0,
                                                        int nsplit, int rows_pad, bf16 *out) {
+  pdl_wait();
+  pdl_trigger();
   const int b = blockIdx.y;
   const int Tq = step0 ? g.H + 1 : g.H;
   const int qi = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
@@ -410,11 +414,11 @@ void launch_attention_tc(const bf16 *q, const bf16 *ks, const bf16 *vs, const Ca
   float *part_o = part;
   float *part_ml = splits > 1 ? part + (size_t)g.B * splits * mtiles * kRowsPerCta * kHeadDim : nullptr;
   dim3 grid(mtiles, splits, g.B);
-  k_attn_tc<<<grid, 128, kSmemTotal, s>>>(q, ks, vs, cp, layer, nvalid, vidx, g, step0, bps, out, part_o,
-                                          part_ml, err);
+  launch_pdl(k_attn_tc, grid, 128, kSmemTotal, s, q, ks, vs, cp, layer, nvalid, vidx, g, step0, bps, out, part_o,
+             part_ml, err);
   if (splits > 1) {
     dim3 cg((kHeads * Tq + 7) / 8, g.B);
-    k_attn_combine<<<cg, 256, 0, s>>>(part_o, part_ml, g, step0, splits, mtiles * kRowsPerCta, out);
+    launch_pdl(k_attn_combine, cg, 256, 0, s, part_o, part_ml, g, step0, splits, mtiles * kRowsPerCta, out);
   }
 }
 

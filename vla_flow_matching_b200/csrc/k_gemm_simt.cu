@@ -9,6 +9,8 @@ namespace pi0x {
 template <typename OutT>
 __global__ void __launch_bounds__(256) k_gemm_simt(const float *A, int lda, const float *Bw, int ldb, int M, int N,
                                                     int K, int epi, GemmOut o) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ float As[16][64 + 4];
   __shared__ float Bs[16][64 + 4];
   const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
@@ -66,7 +68,7 @@ void launch_gemm_simt(const float *A, int lda, const float *Bw, int ldb, int M, 
                       const GemmOut &o, cudaStream_t s) {
   if (M <= 0) return;
   dim3 grid((M + 63) / 64, (N + 63) / 64);
-  k_gemm_simt<OutT><<<grid, 256, 0, s>>>(A, lda, Bw, ldb, M, N, K, epi, o);
+  launch_pdl(k_gemm_simt<OutT>, grid, 256, 0, s, A, lda, Bw, ldb, M, N, K, epi, o);
 }
 
 template void launch_gemm_simt<float>(const float *, int, const float *, int, int, int, int, int, const GemmOut &,

@@ -225,9 +225,19 @@ __global__ void __launch_bounds__(128, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  pdl_trigger();
 
   if (threadIdx.x == 0) {
-    for (int kb = kb0; kb < kb1; ++kb) {
+    // Weight tiles do not depend on the previous kernel: start streaming the first
+    // ring's worth before waiting for it, then add the activation tiles.
+    const int pre = min(STAGES, kb1 - kb0);
+    for (int i = 0; i < pre; ++i) {
+      mbar_arrive_expect_tx(&full[i], C::kStage);
+      tma_load_2d(smem + i * C::kStage + C::kABytes, &tmB, (kb0 + i) * 64, n0, &full[i]);
+    }
+    pdl_wait();
+    for (int i = 0; i < pre; ++i) tma_load_2d(smem + i * C::kStage, &tmA, (kb0 + i) * 64, a_row0 + m0, &full[i]);
+    for (int kb = kb0 + pre; kb < kb1; ++kb) {
       const int i = kb - kb0, s = i % STAGES;
       const uint32_t round = i / STAGES;
       if (!mbar_wait(&empty[s], (round & 1u) ^ 1u, err, kErrTimeoutProducer)) break;
@@ -236,7 +246,10 @@ __global__ void __launch_bounds__(128, 1)
       tma_load_2d(a_dst, &tmA, kb * 64, a_row0 + m0, &full[s]);
       tma_load_2d(a_dst + C::kABytes, &tmB, kb * 64, n0, &full[s]);
     }
-  } else if (threadIdx.x == 32) {
+  } else {
+    pdl_wait();
+  }
+  if (threadIdx.x == 32) {
     constexpr uint32_t idesc = idesc_bf16_f32(128, BN);
     for (int kb = kb0; kb < kb1; ++kb) {
       const int i = kb - kb0, s = i % STAGES;
@@ -370,14 +383,30 @@ __global__ void __launch_bounds__(192, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  pdl_trigger();
 
   if (warp == 0) {
     if (lane == 0) {
+      // weight tiles of this CTA's first tile before the previous kernel finishes
+      const int pre = blockIdx.x < ntiles ? min(STAGES, nk) : 0;
+      {
+        const int n0 = (blockIdx.x / mt) * BN;
+        for (int i = 0; i < pre; ++i) {
+          mbar_arrive_expect_tx(&full[i], C::kStage);
+          tma_load_2d(smem + i * C::kStage + C::kABytes, &tmB, i * 64, n0, &full[i]);
+        }
+      }
+      pdl_wait();
+      {
+        const int m0 = (blockIdx.x % mt) * 128;
+        for (int i = 0; i < pre; ++i) tma_load_2d(smem + i * C::kStage, &tmA, i * 64, a_row0 + m0, &full[i]);
+      }
       int it = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
         const int m0 = (t % mt) * 128, n0 = (t / mt) * BN;
         for (int kb = 0; kb < nk; ++kb, ++it) {
+          if (it < pre) continue;  // issued above
           const int s = it % STAGES;
           const uint32_t round = it / STAGES;
           if (!mbar_wait(&empty[s], (round & 1u) ^ 1u, err, kErrTimeoutProducer)) {
@@ -423,6 +452,7 @@ __global__ void __launch_bounds__(192, 1)
     }
   } else {
     // epilogue warps 2..5: TMEM lane quarter = warp % 4
+    pdl_wait();
     const int q = warp & 3;
     const uint32_t t_lane = (uint32_t)(q * 32) << 16;
     int ti = 0;
@@ -469,7 +499,7 @@ static void launch_cfg(const CUtensorMap &tmA, const CUtensorMap &tmB, int a_row
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int tiles = ((M + 127) / 128) * (N / BN);
-    kern<<<tiles < sms ? tiles : sms, 192, C::kSmem, s>>>(tmA, tmB, a_row0, M, N, nk, e, err);
+    launch_pdl(kern, tiles < sms ? tiles : sms, 192, C::kSmem, s, tmA, tmB, a_row0, M, N, nk, e, err);
     return;
   }
   auto kern = k_gemm_tc<BN, STAGES, EPI>;
@@ -477,7 +507,7 @@ static void launch_cfg(const CUtensorMap &tmA, const CUtensorMap &tmB, int a_row
   const int kps = (nk + splits - 1) / splits;
   splits = (nk + kps - 1) / kps;
   dim3 grid((M + 127) / 128, N / BN, splits);
-  kern<<<grid, 128, C::kSmem, s>>>(tmA, tmB, a_row0, M, nk, kps, e, err);
+  launch_pdl(kern, grid, 128, C::kSmem, s, tmA, tmB, a_row0, M, nk, kps, e, err);
 }
 
 template <int EPI>
@@ -485,7 +515,9 @@ static void launch_epi(const CUtensorMap &tmA, const CUtensorMap &tmB, int bn, i
                        int splits, const EpiArgs &e, unsigned *err, cudaStream_t s) {
   switch (bn) {
     case 32: launch_cfg<32, 8, EPI>(tmA, tmB, a_row0, M, N, K, splits, e, err, s); break;
-    case 64: launch_cfg<64, 6, EPI>(tmA, tmB, a_row0, M, N, K, splits, e, err, s); break;
+    // 4 stages (96 KB): two CTAs fit on an SM, so the next small-batch GEMM can be
+    // resident and stream its weights while the current one finishes
+    case 64: launch_cfg<64, 4, EPI>(tmA, tmB, a_row0, M, N, K, splits, e, err, s); break;
     case 128: launch_cfg<128, 5, EPI>(tmA, tmB, a_row0, M, N, K, splits, e, err, s); break;
     case 256: launch_cfg<256, 4, EPI>(tmA, tmB, a_row0, M, N, K, splits, e, err, s); break;
     default: break;

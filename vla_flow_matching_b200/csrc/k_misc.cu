@@ -13,6 +13,8 @@ namespace pi0x {
 // Count of valid prefix tokens n_b and their positions, in order
 // (`denoise_step`: position ids continue at sum(prefix_pad_masks)).
 __global__ void __launch_bounds__(256) k_prep_mask(const CallPtrs *cp, int P, int *nvalid, int *vidx) {
+  pdl_wait();
+  pdl_trigger();
   const int b = blockIdx.x;
   const uint8_t *m = cp->mask + (size_t)b * P;
   __shared__ int warp_tot[8];
@@ -41,7 +43,7 @@ __global__ void __launch_bounds__(256) k_prep_mask(const CallPtrs *cp, int P, in
 }
 
 void launch_prep_mask(const CallPtrs *cp, int B, int P, int *nvalid, int *vidx, cudaStream_t s) {
-  k_prep_mask<<<B, 256, 0, s>>>(cp, P, nvalid, vidx);
+  launch_pdl(k_prep_mask, B, 256, 0, s, cp, P, nvalid, vidx);
 }
 
 // tvec[k][n] = sum_i Wt[n][i] * temb_k[i] + b[n] for every Euler step k.
@@ -51,6 +53,8 @@ void launch_prep_mask(const CallPtrs *cp, int B, int P, int *nvalid, int *vidx, 
 // is the same for every sample and action token, so it is formed once per call.
 template <typename TW>
 __global__ void __launch_bounds__(256) k_time_vec(const TW *wt, const float *bias, int num_steps, float *tvec) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ float temb[kWidth];
   const int k = blockIdx.x;
   const double dt = -1.0 / (double)num_steps;
@@ -77,7 +81,7 @@ __global__ void __launch_bounds__(256) k_time_vec(const TW *wt, const float *bia
 
 template <typename TW>
 void launch_time_vec(const TW *w_time, const float *bias, int num_steps, float *tvec, cudaStream_t s) {
-  k_time_vec<TW><<<dim3(num_steps, kWidth / 32), 256, 0, s>>>(w_time, bias, num_steps, tvec);
+  launch_pdl(k_time_vec<TW>, dim3(num_steps, kWidth / 32), 256, 0, s, w_time, bias, num_steps, tvec);
 }
 
 // State token: h[b] = state_proj(state[b]) (`embed_suffix`).  With `gain` set it
@@ -87,6 +91,8 @@ template <typename TW>
 __global__ void __launch_bounds__(256) k_state_embed(const CallPtrs *cp, const TW *w, const float *bias, int S,
                                                       float *h, const float *gain, bf16 *xn, float *ss,
                                                       int ss_ld) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ float sv[64];
   __shared__ float red[8];
   const int b = blockIdx.x;
@@ -119,7 +125,7 @@ __global__ void __launch_bounds__(256) k_state_embed(const CallPtrs *cp, const T
 template <typename TW>
 void launch_state_embed(const CallPtrs *cp, const TW *w, const float *b, int B, int S, float *h, cudaStream_t s,
                         const float *gain, bf16 *xn, float *ss, int ss_ld) {
-  k_state_embed<TW><<<B, 256, 0, s>>>(cp, w, b, S, h, gain, xn, ss, ss_ld);
+  launch_pdl(k_state_embed<TW>, B, 256, 0, s, cp, w, b, S, h, gain, xn, ss, ss_ld);
 }
 
 // Action tokens: out[i] = action_in_proj(x[i]) for every (sample, horizon) row.
@@ -129,6 +135,8 @@ constexpr int kActRows = 16;
 template <typename TW, typename T>
 __global__ void __launch_bounds__(256) k_action_in(const float *x, const TW *w, const float *bias, int rows, int A,
                                                     T *out) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ float xv[kActRows][64];
   const int r0 = blockIdx.x * kActRows;
   for (int e = threadIdx.x; e < kActRows * A; e += blockDim.x) {
@@ -152,12 +160,15 @@ __global__ void __launch_bounds__(256) k_action_in(const float *x, const TW *w, 
 
 template <typename TW, typename T>
 void launch_action_in(const float *x, const TW *w, const float *b, int rows, int A, T *out, cudaStream_t s) {
-  k_action_in<TW, T><<<dim3((rows + kActRows - 1) / kActRows, kWidth / 256), 256, 0, s>>>(x, w, b, rows, A, out);
+  launch_pdl(k_action_in<TW, T>, dim3((rows + kActRows - 1) / kActRows, kWidth / 256), 256, 0, s, x, w, b, rows,
+             A, out);
 }
 
 // RoPE table for the fused QKV epilogue: tab[p][i] = (cos, sin)(fp32(p) * inv_freq[i])
 // for every position a call can use, with the accurate CUDA sincosf.
 __global__ void k_rope_table(const float *inv_freq, int npos, float *tab) {
+  pdl_wait();
+  pdl_trigger();
   const int i = threadIdx.x;  // 128 pairs
   for (int p = blockIdx.x; p < npos; p += gridDim.x) {
     float sn, cs;
@@ -167,12 +178,14 @@ __global__ void k_rope_table(const float *inv_freq, int npos, float *tab) {
   }
 }
 void launch_rope_table(const float *inv_freq, int npos, float *tab, cudaStream_t s) {
-  k_rope_table<<<npos < 1024 ? npos : 1024, kHeadDim / 2, 0, s>>>(inv_freq, npos, tab);
+  launch_pdl(k_rope_table, npos < 1024 ? npos : 1024, kHeadDim / 2, 0, s, inv_freq, npos, tab);
 }
 
 // Gemma RMSNorm: out = h * (1/sqrt(mean(h^2) + 1e-6)) * (1 + gain), one warp per row.
 template <typename T>
 __global__ void __launch_bounds__(256) k_rmsnorm(const float *h, int row0, int rows, const float *gain, T *out) {
+  pdl_wait();
+  pdl_trigger();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int r = blockIdx.x * 8 + warp;
   if (r >= rows) return;
@@ -203,7 +216,7 @@ __global__ void __launch_bounds__(256) k_rmsnorm(const float *h, int row0, int r
 template <typename T>
 void launch_rmsnorm(const float *h, int row0, int rows, const float *gain, T *out, cudaStream_t s) {
   if (rows <= 0) return;
-  k_rmsnorm<T><<<(rows + 7) / 8, 256, 0, s>>>(h, row0, rows, gain, out);
+  launch_pdl(k_rmsnorm<T>, (rows + 7) / 8, 256, 0, s, h, row0, rows, gain, out);
 }
 
 // (b, j) of an activation row: state rows first, then b*H + (j-1).
@@ -223,6 +236,8 @@ __device__ __forceinline__ void row_to_bj(int r, int B, int H, int &b, int &j) {
 template <typename T>
 __global__ void __launch_bounds__(256) k_rope_qkv(const float *raw, int row0, Geo g, const int *nvalid,
                                                    const float *inv_freq, T *q, T *ks, T *vs) {
+  pdl_wait();
+  pdl_trigger();
   const int r = row0 + blockIdx.x;
   int b, j;
   row_to_bj(r, g.B, g.H, b, j);
@@ -251,12 +266,14 @@ template <typename T>
 void launch_rope_qkv(const float *raw, int row0, int rows, const Geo &g, const int *nvalid, const float *inv_freq,
                      T *q, T *ks, T *vs, cudaStream_t s) {
   if (rows <= 0) return;
-  k_rope_qkv<T><<<rows, 256, 0, s>>>(raw, row0, g, nvalid, inv_freq, q, ks, vs);
+  launch_pdl(k_rope_qkv<T>, rows, 256, 0, s, raw, row0, g, nvalid, inv_freq, q, ks, vs);
 }
 
 // Gemma MLP activation: act = gelu_tanh(gate) * up, raw row = [gate(4096) | up(4096)].
 template <typename T>
 __global__ void __launch_bounds__(256) k_geglu(const float *raw, int row0, T *act) {
+  pdl_wait();
+  pdl_trigger();
   const size_t r = (size_t)(row0 + blockIdx.x);
   for (int f = threadIdx.x; f < kMlp; f += blockDim.x) {
     const float gt = raw[r * 2 * kMlp + f], up = raw[r * 2 * kMlp + kMlp + f];
@@ -267,7 +284,7 @@ __global__ void __launch_bounds__(256) k_geglu(const float *raw, int row0, T *ac
 template <typename T>
 void launch_geglu(const float *raw, int row0, int rows, T *act, cudaStream_t s) {
   if (rows <= 0) return;
-  k_geglu<T><<<rows, 256, 0, s>>>(raw, row0, act);
+  launch_pdl(k_geglu<T>, rows, 256, 0, s, raw, row0, act);
 }
 
 // Final RMSNorm of an action token, v = action_out_proj(.) in fp32, then the
@@ -276,6 +293,8 @@ void launch_geglu(const float *raw, int row0, int rows, T *act, cudaStream_t s) 
 __global__ void __launch_bounds__(256) k_final_euler(const float *h, Geo g, const float *gain, const float *w_out,
                                                       const float *b_out, float dt, float *x, const CallPtrs *cp,
                                                       int last) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ float y[kWidth];
   __shared__ float red[8];
   const int i = blockIdx.x;  // action row index b*H + (j-1)
@@ -312,14 +331,16 @@ __global__ void __launch_bounds__(256) k_final_euler(const float *h, Geo g, cons
 
 void launch_final_euler(const float *h, const Geo &g, const float *gain, const float *w_out, const float *b_out,
                         float dt, float *x, const CallPtrs *cp, int last, cudaStream_t s) {
-  k_final_euler<<<g.B * g.H, 256, 0, s>>>(h, g, gain, w_out, b_out, dt, x, cp, last);
+  launch_pdl(k_final_euler, g.B * g.H, 256, 0, s, h, g, gain, w_out, b_out, dt, x, cp, last);
 }
 
 __global__ void k_copy_x1(const CallPtrs *cp, int n, float *x) {
+  pdl_wait();
+  pdl_trigger();
   for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) x[i] = cp->x1[i];
 }
 void launch_copy_x1(const CallPtrs *cp, int n, float *x, cudaStream_t s) {
-  k_copy_x1<<<(n + 255) / 256 < 1024 ? (n + 255) / 256 : 1024, 256, 0, s>>>(cp, n, x);
+  launch_pdl(k_copy_x1, (n + 255) / 256 < 1024 ? (n + 255) / 256 : 1024, 256, 0, s, cp, n, x);
 }
 
 // Holds the stream for `ns` nanoseconds of wall time (bounded by construction).

@@ -86,6 +86,24 @@ struct Geo {
   int B, H, A, S, P, R;   // R = B + B*H
 };
 
+// Launch `kern` with programmatic stream serialization (it may overlap the previous
+// kernel on the stream until it calls pdl_wait()).
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                              Args &&...args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
 // ---- misc kernels (k_misc.cu) ----
 void launch_prep_mask(const CallPtrs *cp, int B, int P, int *nvalid, int *vidx, cudaStream_t s);
 template <typename TW>
