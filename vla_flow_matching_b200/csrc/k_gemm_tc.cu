@@ -25,9 +25,17 @@
 
 namespace pi0x {
 
-template <int BN, int STAGES>
+#ifndef PI0X_BN64_STAGES
+#define PI0X_BN64_STAGES 6
+#endif
+constexpr int kBn64Stages = PI0X_BN64_STAGES;
+
+// AR = rows of the activation tile loaded per stage: 128, or 64 when the GEMM has
+// at most 64 rows.  The MMA is always M = 128; with AR = 64 the accumulator rows
+// 64..127 see whatever follows the A tile in shared memory and are never stored.
+template <int BN, int STAGES, int AR = 128>
 struct TcCfg {
-  static constexpr int kABytes = 128 * 128;   // 128 rows x 64 bf16
+  static constexpr int kABytes = AR * 128;    // AR rows x 64 bf16
   static constexpr int kBBytes = BN * 128;    // BN rows x 64 bf16
   static constexpr int kStage = kABytes + kBBytes;
   static constexpr int kTmemCols = BN < 32 ? 32 : BN;
@@ -185,11 +193,11 @@ __device__ __forceinline__ void norm_partial_store(const EpiArgs &e, int r, int 
   }
 }
 
-template <int BN, int STAGES, int EPI>
+template <int BN, int STAGES, int EPI, int AR>
 __global__ void __launch_bounds__(128, 1)
     k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, int a_row0, int M,
               int nk, int kb_per_split, EpiArgs e, unsigned *err) {
-  using C = TcCfg<BN, STAGES>;
+  using C = TcCfg<BN, STAGES, AR>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t *full = reinterpret_cast<uint64_t *>(smem + STAGES * C::kStage);
@@ -344,11 +352,11 @@ __global__ void __launch_bounds__(128, 1)
 // (row tile fastest, so concurrently running CTAs share weight tiles in L2).
 // Warp 0 = TMA producer, warp 1 = MMA issuer, warps 2..5 = epilogue.  Two TMEM
 // accumulators let the epilogue of one tile overlap the main loop of the next.
-template <int BN, int STAGES, int EPI>
+template <int BN, int STAGES, int EPI, int AR>
 __global__ void __launch_bounds__(192, 1)
     k_gemm_tc_persist(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, int a_row0,
                       int M, int N, int nk, EpiArgs e, unsigned *err) {
-  using C = TcCfg<BN, STAGES>;
+  using C = TcCfg<BN, STAGES, AR>;
   constexpr int kAcc = 2;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -487,13 +495,13 @@ __global__ void __launch_bounds__(192, 1)
   }
 }
 
-template <int BN, int STAGES, int EPI>
+template <int BN, int STAGES, int EPI, int AR>
 static void launch_cfg(const CUtensorMap &tmA, const CUtensorMap &tmB, int a_row0, int M, int N, int K, int splits,
                        const EpiArgs &e, unsigned *err, cudaStream_t s) {
-  using C = TcCfg<BN, STAGES>;
+  using C = TcCfg<BN, STAGES, AR>;
   const int nk = K / 64;
   if (splits == 1 && 2 * C::kTmemCols <= 512) {
-    auto kern = k_gemm_tc_persist<BN, STAGES, EPI>;
+    auto kern = k_gemm_tc_persist<BN, STAGES, EPI, AR>;
     cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
@@ -502,7 +510,7 @@ static void launch_cfg(const CUtensorMap &tmA, const CUtensorMap &tmB, int a_row
     launch_pdl(kern, tiles < sms ? tiles : sms, 192, C::kSmem, s, tmA, tmB, a_row0, M, N, nk, e, err);
     return;
   }
-  auto kern = k_gemm_tc<BN, STAGES, EPI>;
+  auto kern = k_gemm_tc<BN, STAGES, EPI, AR>;
   cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
   const int kps = (nk + splits - 1) / splits;
   splits = (nk + kps - 1) / kps;
@@ -511,15 +519,21 @@ static void launch_cfg(const CUtensorMap &tmA, const CUtensorMap &tmB, int a_row
 }
 
 template <int EPI>
-static void launch_epi(const CUtensorMap &tmA, const CUtensorMap &tmB, int bn, int a_row0, int M, int N, int K,
-                       int splits, const EpiArgs &e, unsigned *err, cudaStream_t s) {
-  switch (bn) {
-    case 32: launch_cfg<32, 8, EPI>(tmA, tmB, a_row0, M, N, K, splits, e, err, s); break;
-    // 4 stages (96 KB): two CTAs fit on an SM, so the next small-batch GEMM can be
-    // resident and stream its weights while the current one finishes
-    case 64: launch_cfg<64, 4, EPI>(tmA, tmB, a_row0, M, N, K, splits, e, err, s); break;
-    case 128: launch_cfg<128, 5, EPI>(tmA, tmB, a_row0, M, N, K, splits, e, err, s); break;
-    case 256: launch_cfg<256, 4, EPI>(tmA, tmB, a_row0, M, N, K, splits, e, err, s); break;
+static void launch_epi(const CUtensorMap &tmA, const CUtensorMap &tmB, const TcPlan &p, int a_row0, int M, int N,
+                       int K, const EpiArgs &e, unsigned *err, cudaStream_t s) {
+  const int splits = p.splits;
+  switch (p.bn) {
+    case 32: launch_cfg<32, 8, EPI, 128>(tmA, tmB, a_row0, M, N, K, splits, e, err, s); break;
+    case 64:
+      // 64-wide tiles (small batches): 12 stages of 16 KB with 64-row activation
+      // tiles, else kBn64Stages of 24 KB
+      if (p.a_rows == 64)
+        launch_cfg<64, 12, EPI, 64>(tmA, tmB, a_row0, M, N, K, splits, e, err, s);
+      else
+        launch_cfg<64, kBn64Stages, EPI, 128>(tmA, tmB, a_row0, M, N, K, splits, e, err, s);
+      break;
+    case 128: launch_cfg<128, 5, EPI, 128>(tmA, tmB, a_row0, M, N, K, splits, e, err, s); break;
+    case 256: launch_cfg<256, 4, EPI, 128>(tmA, tmB, a_row0, M, N, K, splits, e, err, s); break;
     default: break;
   }
 }
@@ -534,6 +548,7 @@ TcPlan plan_gemm_tc(int M, int N, int K) {
     return p;
   }
   p.bn = 64;
+  p.a_rows = M <= 64 ? 64 : 128;
   const int ctas = mt * (N / 64);
   int sp = ctas >= 148 ? 1 : 148 / ctas;
   if (sp > nk / 2) sp = nk / 2 > 0 ? nk / 2 : 1;
@@ -551,12 +566,12 @@ void launch_gemm_tc(int epi, const CUtensorMap &tmA, const CUtensorMap &tmB, con
                     int N, int K, const EpiArgs &e, unsigned *err, cudaStream_t s) {
   if (M <= 0) return;
   switch (epi) {
-    case EPI_STORE_F32: launch_epi<EPI_STORE_F32>(tmA, tmB, p.bn, a_row0, M, N, K, p.splits, e, err, s); break;
-    case EPI_BIAS_F32: launch_epi<EPI_BIAS_F32>(tmA, tmB, p.bn, a_row0, M, N, K, p.splits, e, err, s); break;
-    case EPI_VEC_SILU: launch_epi<EPI_VEC_SILU>(tmA, tmB, p.bn, a_row0, M, N, K, p.splits, e, err, s); break;
-    case EPI_RESID_F32: launch_epi<EPI_RESID_F32>(tmA, tmB, p.bn, a_row0, M, N, K, p.splits, e, err, s); break;
-    case EPI_QKV_ROPE: launch_epi<EPI_QKV_ROPE>(tmA, tmB, p.bn, a_row0, M, N, K, p.splits, e, err, s); break;
-    case EPI_GEGLU: launch_epi<EPI_GEGLU>(tmA, tmB, p.bn, a_row0, M, N, K, p.splits, e, err, s); break;
+    case EPI_STORE_F32: launch_epi<EPI_STORE_F32>(tmA, tmB, p, a_row0, M, N, K, e, err, s); break;
+    case EPI_BIAS_F32: launch_epi<EPI_BIAS_F32>(tmA, tmB, p, a_row0, M, N, K, e, err, s); break;
+    case EPI_VEC_SILU: launch_epi<EPI_VEC_SILU>(tmA, tmB, p, a_row0, M, N, K, e, err, s); break;
+    case EPI_RESID_F32: launch_epi<EPI_RESID_F32>(tmA, tmB, p, a_row0, M, N, K, e, err, s); break;
+    case EPI_QKV_ROPE: launch_epi<EPI_QKV_ROPE>(tmA, tmB, p, a_row0, M, N, K, e, err, s); break;
+    case EPI_GEGLU: launch_epi<EPI_GEGLU>(tmA, tmB, p, a_row0, M, N, K, e, err, s); break;
     default: break;
   }
 }

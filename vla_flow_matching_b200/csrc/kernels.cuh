@@ -72,6 +72,13 @@ constexpr int kNormSlots = 16;
 struct TcPlan {
   int bn = 128;
   int splits = 1;
+  int a_rows = 128;  // rows of the activation TMA box (64 when the GEMM has <= 64 rows)
+};
+
+// Activation operand: tensor maps with 128-row and 64-row boxes.
+struct ActMap {
+  CUtensorMap m128, m64;
+  const CUtensorMap &get(int rows) const { return rows == 64 ? m64 : m128; }
 };
 
 struct GemmOut {
@@ -100,7 +107,11 @@ inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, siz
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
+#ifdef PI0X_NO_PDL
+  cfg.numAttrs = 0;  // build option: plain stream-ordered launches
+#else
   cfg.numAttrs = 1;
+#endif
   return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
 }
 

@@ -112,7 +112,7 @@ struct Workspace {
   uint8_t *st_mask = nullptr;
   float *st_state = nullptr, *st_x = nullptr;
   // tensor maps of the activation operands (bf16 mode)
-  CUtensorMap m_xn, m_att, m_act, m_aemb, m_uemb;
+  ActMap m_xn, m_att, m_act, m_aemb, m_uemb;
 };
 
 }  // namespace
@@ -328,11 +328,11 @@ int ensure_workspace(pi0x_handle *h, int B, int P, int N) {
   ws.N = nN;
   ws.R = (int)R;
   if (h->bf16) {
-    bool ok = make_map(&ws.m_xn, ws.xn, Rp, kWidth, kWidth, 128) &&
-              make_map(&ws.m_att, ws.att, Rp, kQDim, kQDim, 128) &&
-              make_map(&ws.m_act, ws.act, Rp, kMlp, kMlp, 128) &&
-              make_map(&ws.m_aemb, ws.a_emb, Rp, kWidth, kWidth, 128) &&
-              make_map(&ws.m_uemb, ws.u_emb, Rp, kWidth, kWidth, 128);
+    auto mk = [&](ActMap &m, void *p, int cols) {
+      return make_map(&m.m128, p, Rp, cols, cols, 128) && make_map(&m.m64, p, Rp, cols, cols, 64);
+    };
+    bool ok = mk(ws.m_xn, ws.xn, kWidth) && mk(ws.m_att, ws.att, kQDim) && mk(ws.m_act, ws.act, kMlp) &&
+              mk(ws.m_aemb, ws.a_emb, kWidth) && mk(ws.m_uemb, ws.u_emb, kWidth);
     if (!ok) {
       g_last_error = "cuTensorMapEncodeTiled failed for an activation operand";
       return PI0X_ECUDA;
@@ -429,9 +429,9 @@ int enqueue_loop(pi0x_handle *h, int B, int P, int N, cudaStream_t s) {
   ebase.part = ws.gpart;
   ebase.counters = ws.counters;
   ebase.rope_tab = ws.rope_tab;
-  auto gemm = [&](int epi, const CUtensorMap &tmA, const TcWeight &w, int a_row0, int M, const EpiArgs &e) {
+  auto gemm = [&](int epi, const ActMap &am, const TcWeight &w, int a_row0, int M, const EpiArgs &e) {
     const TcPlan p = plan_gemm_tc(M, w.N, w.K);
-    launch_gemm_tc(epi, tmA, w.map(p.bn), p, a_row0, M, w.N, w.K, e, h->d_err, s);
+    launch_gemm_tc(epi, am.get(p.a_rows), w.map(p.bn), p, a_row0, M, w.N, w.K, e, h->d_err, s);
   };
 
   RUN(PI0X_K_PREP, launch_prep_mask(h->d_ptrs, B, P, ws.nvalid, ws.vidx, s));
@@ -610,8 +610,12 @@ int pi0x_debug_gemm_bf16(const void *A, const void *Bw, int M, int N, int K, flo
     CK(cudaMalloc(&d_cnt, sizeof(int) * 1024));
     CK(cudaMemset(d_cnt, 0, sizeof(int) * 1024));
   }
+  TcPlan p;
+  p.bn = bn;
+  p.splits = splits;
+  p.a_rows = (bn == 64 && M <= 64) ? 64 : 128;  // as the sampler plans small GEMMs
   CUtensorMap tmA, tmB;
-  if (!make_map(&tmA, A, M, K, K, 128) || !make_map(&tmB, Bw, N, K, K, bn)) {
+  if (!make_map(&tmA, A, M, K, K, p.a_rows) || !make_map(&tmB, Bw, N, K, K, bn)) {
     g_last_error = "cuTensorMapEncodeTiled failed";
     return PI0X_ECUDA;
   }
@@ -621,9 +625,6 @@ int pi0x_debug_gemm_bf16(const void *A, const void *Bw, int M, int N, int K, flo
   e.ldo = N;
   e.part = d_part;
   e.counters = d_cnt;
-  TcPlan p;
-  p.bn = bn;
-  p.splits = splits;
   launch_gemm_tc(EPI_STORE_F32, tmA, tmB, p, 0, M, N, K, e, d_err, s);
   CK(cudaGetLastError());
   CK(cudaStreamSynchronize(s));
