@@ -41,14 +41,14 @@ int pi0x_debug_attention(const void *q, const void *ks, const void *vs, const vo
  * application whose device memory is owned by its own pool.  It calls no
  * cudaMalloc/cudaFree and no allocating library routine: all its scratch (a call
  * table, an error word, the valid-prefix index list and the split-KV partials)
- * lives in one static device array of 16 MiB inside libpi0x, which every GPU that
+ * lives in one static device array of 32 MiB inside libpi0x, which every GPU that
  * loads the library holds until the process exits.  The pages have no counterpart
  * to this entry point; it is a deployment variant of the `_attend` step.
  *
  * Arguments as for pi0x_debug_attention.  Returns PI0X_EINVAL when the problem's
- * scratch (about 4 B per prefix position per sample plus the split-KV partials,
- * 4 B x 258 per query row per split) does not fit in the 16 MiB; B=1..8 with the
- * pi0 prefix lengths fit.  The first call on each device looks up the device
+ * scratch (4 B per prefix position per sample plus the split-KV partials,
+ * 4 B x 258 per query row per split, at most 32.1 MB) does not fit in the 32 MiB;
+ * the pi0 workloads up to B = 8 fit.  The first call on each device looks up the device
  * address of the array (cudaGetSymbolAddress, with that device current); make that
  * first call before any stream capture.  Every call clears the error word it uses;
  * the array keeps the contents of the last call.  All calls share the one array,

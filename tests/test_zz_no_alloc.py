@@ -36,7 +36,7 @@ def _inputs(torch, B, H, P, seed):
     return q, ks, vs, pk, pv, mask
 
 
-@pytest.mark.parametrize("B,H,P,step0", [(1, 50, 816, 1), (1, 50, 816, 0), (4, 10, 560, 1)])
+@pytest.mark.parametrize("B,H,P,step0", [(1, 50, 816, 1), (1, 50, 816, 0), (4, 10, 560, 1), (8, 50, 816, 1)])
 def test_noalloc_attention_matches_allocating_entry_point(B, H, P, step0):
     torch = _torch()
     from vla_flow_matching_b200 import build, pi0x
@@ -69,7 +69,7 @@ def test_noalloc_rejects_problems_larger_than_its_scratch():
     f = pi0x.load().pi0x_attention_noalloc
     f.argtypes = [ctypes.c_void_p] * 6 + [ctypes.c_int] * 4 + [ctypes.c_void_p] * 2
     f.restype = ctypes.c_int
-    B, H, P = 1024, 50, 8192   # the valid-index list alone needs 32 MiB; rejected before any launch
+    B, H, P = 2048, 50, 8192   # the valid-index list alone needs 64 MiB; rejected before any launch
     dummy = torch.zeros(16, dtype=torch.bfloat16, device="cuda")
     st = f(dummy.data_ptr(), dummy.data_ptr(), dummy.data_ptr(), dummy.data_ptr(), dummy.data_ptr(),
            dummy.data_ptr(), B, H, P, 1, dummy.data_ptr(), None)

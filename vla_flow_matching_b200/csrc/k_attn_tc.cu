@@ -390,8 +390,7 @@ int attn_tc_splits(const Geo &g, int step0, int max_keys) {
   const int ctas = mtiles * g.B;
   if (ctas >= 96) return 1;
   int splits = (148 + ctas - 1) / ctas;
-  const int max_split = (nblk + 1) / 2;  // at least two key blocks per split
-  if (splits > max_split) splits = max_split;
+  if (splits > nblk) splits = nblk;  // down to one key block per split
   return splits < 1 ? 1 : splits;
 }
 

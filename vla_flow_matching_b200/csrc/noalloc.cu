@@ -26,7 +26,9 @@
 namespace pi0x {
 namespace {
 
-constexpr size_t kScratchBytes = size_t(16) << 20;  // 16 MiB
+// 32 MiB: split-KV uses at most 243 row tiles x splits (attn_tc_splits), i.e. at most
+// 243 x 128 rows x 258 floats = 32.1 MB of partials, plus the valid-index list.
+constexpr size_t kScratchBytes = size_t(32) << 20;
 __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
 
 constexpr int kMaxDevices = 64;
@@ -85,7 +87,7 @@ extern "C" int pi0x_attention_noalloc(const void *q, const void *ks, const void 
   const size_t off_part = align256(off_vidx + sizeof(int) * (size_t)B * (P > 0 ? P : 1));
   const size_t need = off_part + sizeof(float) * attn_tc_partial_floats(g, step0, splits);
   if (need > kScratchBytes) {
-    set_last_error("pi0x_attention_noalloc: the problem needs more scratch than the 16 MiB static array");
+    set_last_error("pi0x_attention_noalloc: the problem needs more scratch than the 32 MiB static array");
     return PI0X_EINVAL;
   }
 
