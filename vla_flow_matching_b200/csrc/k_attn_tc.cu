@@ -27,16 +27,18 @@ namespace pi0x {
 namespace {
 constexpr int kRowsPerCta = 128;
 constexpr int kKeyBlock = 64;
-constexpr uint32_t kQBytes = 128 * 512;       // 4 sub-tiles of [128 rows x 64 dims]
+constexpr int kKBufs = 4;                     // K ring depth (K tiles prefetched 3 blocks ahead)
 constexpr uint32_t kKVBytes = 64 * 512;       // 4 sub-tiles of [64 keys x 64 dims]
 constexpr uint32_t kPBytes = 128 * 128;       // [128 rows x 64 keys]
-constexpr uint32_t kSmemQ = 0;
-constexpr uint32_t kSmemK0 = kSmemQ + kQBytes;
-constexpr uint32_t kSmemV0 = kSmemK0 + 2 * kKVBytes;
+constexpr uint32_t kSmemK0 = 0;
+constexpr uint32_t kSmemV0 = kSmemK0 + kKBufs * kKVBytes;
 constexpr uint32_t kSmemP = kSmemV0 + 2 * kKVBytes;
 constexpr uint32_t kSmemBar = kSmemP + kPBytes;
 constexpr uint32_t kSmemTotal = kSmemBar + 64 + 1024;  // + alignment slack
-constexpr uint32_t kTmemCols = 512;   // S buffers at columns 0 and 64, O at 256 (256 columns)
+// TMEM: S buffers at columns 0 and 64, Q (the A operand of S = Q K^T: bf16 pairs,
+// K-major, row = lane) at 128..255, O at 256..511
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kTmemQ = 128;
 constexpr uint32_t kTmemO = 256;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleSlack = 8.0f;  // log2 units
@@ -100,28 +102,13 @@ __global__ void __launch_bounds__(128, 1)
     tmem_relinquish();
   }
 
-  // ---- Q tile: rows [row0, row0+128), 4 swizzled sub-tiles of 64 dims ----
-  for (int i = 0; i < 32; ++i) {
-    const int c = tid + 128 * i;
-    const int r = c >> 5, cr = c & 31;
-    const int qr = row0 + r;
-    const bool ok = qr < nrows;
-    int t = 0, hd = 0;
-    if (ok) {
-      const int j = qr / kHeads;
-      hd = qr % kHeads;
-      t = step0 ? (j == 0 ? b : g.B + b * g.H + j - 1) : g.B + b * g.H + j;
-    }
-    const bf16 *src = q + (size_t)t * kQDim + hd * kHeadDim + cr * 8;
-    cp_async16(sbase + kSmemQ + (cr >> 3) * (128 * 128) + sw128_off(r, cr & 7), src, ok);
-  }
   // Warp w copies keys [16w, 16w+16) of block j, lane = 16-byte chunk of the 512-byte
   // row.  Lanes 0..15 first look up one key's source row each (independent loads),
   // then every copy takes its row pointer from a shuffle.  `which`: 1 = K, 2 = V.
   auto load_block = [&](int j, int which) {
     if (j >= nb) return;
-    const int blk = blk0 + j, buf = j & 1;
-    const uint32_t kb = sbase + kSmemK0 + buf * kKVBytes, vb = sbase + kSmemV0 + buf * kKVBytes;
+    const int blk = blk0 + j;
+    const uint32_t kb = sbase + kSmemK0 + (j % kKBufs) * kKVBytes, vb = sbase + kSmemV0 + (j & 1) * kKVBytes;
     const int kk_l = blk * kKeyBlock + warp * 16 + (lane & 15);
     const bool ok_l = kk_l < nk;
     const bf16 *krow = ks, *vrow = vs;
@@ -148,10 +135,15 @@ __global__ void __launch_bounds__(128, 1)
   };
 
   // cp.async groups, committed in this order (empty groups keep the pattern):
-  //   prologue: [Q, K0, V0] [K1] [V1];  iteration w: [K(w+2)] [V(w+1) after PV(w-1)]
+  //   prologue: [K0, V0] [K1] [K2] [K3] [V1];
+  //   iteration w: [K(w+4)] after S(w), [V(w+1)] after PV(w-1) (empty at w = 0)
   load_block(0, 3);
   cp_async_commit();
   load_block(1, 1);
+  cp_async_commit();
+  load_block(2, 1);
+  cp_async_commit();
+  load_block(3, 1);
   cp_async_commit();
   load_block(1, 2);
   cp_async_commit();
@@ -162,19 +154,38 @@ __global__ void __launch_bounds__(128, 1)
   const uint32_t tmem = *tmem_slot;
   const uint32_t t_lane = (uint32_t)(warp * 32) << 16;
 
+  // ---- Q: this thread's query row (256 bf16) into TMEM lane `tid`, columns 128..255,
+  // two bf16 per 32-bit column (the K-major A-operand layout of tcgen05.mma) ----
+  {
+    const uint4 *src = reinterpret_cast<const uint4 *>(q + (size_t)tok * kQDim + head * kHeadDim);
+#pragma unroll 1
+    for (int c = 0; c < 4; ++c) {
+      float v[32];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const uint4 u = row_ok ? src[c * 8 + e] : make_uint4(0, 0, 0, 0);
+        v[4 * e] = __uint_as_float(u.x);
+        v[4 * e + 1] = __uint_as_float(u.y);
+        v[4 * e + 2] = __uint_as_float(u.z);
+        v[4 * e + 3] = __uint_as_float(u.w);
+      }
+      tmem_st_32x32b_x32(tmem + t_lane + kTmemQ + 32 * c, v);
+    }
+  }
+
   constexpr uint32_t idesc_s = idesc_bf16_f32(128, kKeyBlock);
   constexpr uint32_t idesc_o = idesc_bf16_f32(128, kHeadDim) | (1u << 16);  // B (V) MN-major
   const float scale_l2 = 0.0625f * kLog2e;
 
-  auto issue_s = [&](int j) {  // S[j&1] = Q K(j)^T
-    const uint32_t kb = sbase + kSmemK0 + (j & 1) * kKVBytes;
+  auto issue_s = [&](int j) {  // S[j&1] = Q K(j)^T, A (Q) from TMEM, 16 head dims per MMA
+    const uint32_t kb = sbase + kSmemK0 + (j % kKBufs) * kKVBytes;
     const uint32_t d = tmem + (uint32_t)((j & 1) * kKeyBlock);
 #pragma unroll
     for (int s = 0; s < 4; ++s)
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk)
-        tc_mma_bf16(d, smem_desc_k_sw128(sbase + kSmemQ + s * (128 * 128), kk * 32),
-                    smem_desc_k_sw128(kb + s * (64 * 128), kk * 32), idesc_s, (s | kk) != 0);
+        tc_mma_bf16_ts(d, tmem + kTmemQ + (uint32_t)(32 * s + 8 * kk), smem_desc_k_sw128(kb + s * (64 * 128), kk * 32),
+                       idesc_s, (s | kk) != 0);
     tc_commit(&bar_s[j & 1]);
   };
 
@@ -182,7 +193,7 @@ __global__ void __launch_bounds__(128, 1)
   uint32_t ph_s0 = 0, ph_s1 = 0, ph_o = 0;
   bool ok_all = true;
   if (nb > 0) {
-    cp_async_wait<2>();
+    cp_async_wait<4>();
     fence_proxy_async_smem();
     tc_fence_before();
     ok_all = __syncthreads_and(ok_all);
@@ -191,9 +202,15 @@ __global__ void __launch_bounds__(128, 1)
   }
   for (int w = 0; w < nb && ok_all; ++w) {
     const int buf = w & 1;
-    // (1) K(w+1) has landed: start S(w+1) on the tensor cores before the softmax of w
+    // (1) K(w+1) has landed: start S(w+1) on the tensor cores before the softmax of w.
+    // Groups committed after K(w+1): 3 at w = 0, 4 at w = 1, then 5.
     if (w + 1 < nb) {
-      cp_async_wait<1>();
+      if (w == 0)
+        cp_async_wait<3>();
+      else if (w == 1)
+        cp_async_wait<4>();
+      else
+        cp_async_wait<5>();
       fence_proxy_async_smem();
       tc_fence_before();
       ok_all = __syncthreads_and(ok_all);
@@ -209,8 +226,8 @@ __global__ void __launch_bounds__(128, 1)
     }
     __syncwarp();
     tc_fence_after();
-    // K(buf) is free again (S(w) done): prefetch K(w+2)
-    load_block(w + 2, 1);
+    // K(w)'s buffer is free again (S(w) done): prefetch K(w+4)
+    load_block(w + kKBufs, 1);
     cp_async_commit();
     float sv[64];
     {
@@ -272,8 +289,14 @@ __global__ void __launch_bounds__(128, 1)
         *reinterpret_cast<uint4 *>(prow + sw128_off(tid, cc)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
       }
     }
-    // V(w) must have landed: all groups but the two just committed
-    cp_async_wait<2>();
+    // V(w) must have landed: groups committed after it are 6 at w = 0 (it came with
+    // K0), 4 at w = 1 (it came last in the prologue), then the 2 of this iteration
+    if (w == 0)
+      cp_async_wait<6>();
+    else if (w == 1)
+      cp_async_wait<4>();
+    else
+      cp_async_wait<2>();
     fence_proxy_async_smem();
     tc_fence_before();
     ok_all = __syncthreads_and(ok_all);
@@ -390,7 +413,8 @@ int attn_tc_splits(const Geo &g, int step0, int max_keys) {
   const int ctas = mtiles * g.B;
   if (ctas >= 96) return 1;
   int splits = (148 + ctas - 1) / ctas;
-  if (splits > nblk) splits = nblk;  // down to one key block per split
+  const int max_split = (nblk + 1) / 2;  // at least two key blocks per split
+  if (splits > max_split) splits = max_split;
   return splits < 1 ? 1 : splits;
 }
 
