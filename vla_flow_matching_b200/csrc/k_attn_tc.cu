@@ -1,22 +1,31 @@
 // Masked MQA attention on the tcgen05 tensor cores (bf16 mode).
 //
 // Computes, per sample and per query head, softmax(q . K^T / sqrt(256) + mask) . V
-// over [valid prefix keys ; state key ; action keys] (`_attend` with the block mask
-// of `denoise_step` on the vllm-omni pi0 page).  The 8 query heads share the one
-// KV head, so a CTA takes 128 query rows (token-major: row = token*8 + head) of
-// one sample against the sample's key list, in blocks of 64 keys.
+// over the valid prefix keys, the state key and the action keys (`_attend` with the
+// block mask of `denoise_step` on the vllm-omni pi0 page).  The 8 query heads share
+// the one KV head, so a CTA takes 128 query rows (token-major: row = token*8 + head)
+// of one sample against the sample's keys, in blocks of 64 key slots.
 //
-// Keys are gathered by index with cp.async (16 B per thread) into 128-byte-
-// swizzled shared memory, so masked prefix positions are never read; the page adds
-// -2.38e38 to their logits, whose exp is exactly 0 in fp32.
+// Key slots of sample b: ceil(nv/64) blocks holding the nv valid prefix positions in
+// order (the compacted list of the mask), then ceil((H+1)/64) blocks holding the H
+// action keys and then the state key; the remaining slots are empty.  Softmax is
+// invariant to the order of the keys.  Masked prefix positions are never read (the
+// page adds -2.38e38 to their logits, whose exp is exactly 0 in fp32).
 //
-// One pass over the key blocks with an online softmax.  S = Q K^T goes to one of
-// two TMEM buffers, so the MMA of block w+1 runs while the threads (one per query
-// row) turn block w into P = 2^(s - m) in bf16 and accumulate O += P V in TMEM.
-// The running max m used for P is raised (and O, l rescaled in place) only when a
-// block's max exceeds it by more than 2^8, so P stays <= 256 and rescaling is
-// rare; O / l at the end normalises.  With split-KV (small batches) every split
-// writes O/l and (m, l) and k_attn_combine merges the splits.
+// Warp roles (224 threads):
+//  * warps 0-3: one query row per thread.  Q goes to TMEM (the A operand of
+//    S = Q K^T); per key block the thread reads its S row from TMEM, forms
+//    P = 2^(s - m) with an online softmax, writes P (bf16) to shared memory, and
+//    rescales O in TMEM when the running max grows by more than 2^8 (rare).
+//  * warp 4 / warp 5: K / V loader into 3-deep rings of 128-byte-swizzled tiles.  A
+//    run of 8 slots whose keys are consecutive rows of one tensor is one TMA box per
+//    64 dims; other runs are copied row by row with cp.async.
+//  * warp 6 lane 0: tcgen05.mma issuer: S(j+1) before PV(j), so the softmax of block
+//    j+1 overlaps the P.V of block j.
+// All hand-offs are mbarriers (TMA transaction bytes, cp.async completion, tcgen05
+// commits, thread arrivals) and every wait is bounded.  O / l at the end
+// normalises.  With split-KV (small batches) every split writes O/l and (m, l) and
+// k_attn_combine merges the splits.
 #include <math.h>
 
 #include "common.cuh"
@@ -27,45 +36,114 @@ namespace pi0x {
 namespace {
 constexpr int kRowsPerCta = 128;
 constexpr int kKeyBlock = 64;
-constexpr int kKBufs = 4;                     // K ring depth (K tiles prefetched 3 blocks ahead)
+constexpr int kKBufs = 3;
+constexpr int kVBufs = 3;
+constexpr int kPBufs = 2;
+static_assert(kVBufs >= kPBufs, "P.V completions are tracked per V buffer");
 constexpr uint32_t kKVBytes = 64 * 512;       // 4 sub-tiles of [64 keys x 64 dims]
+constexpr uint32_t kSubTile = 64 * 128;       // one sub-tile
+constexpr uint32_t kAtomBytes = 8 * 128;      // 8 keys x 64 dims: one TMA box
 constexpr uint32_t kPBytes = 128 * 128;       // [128 rows x 64 keys]
 constexpr uint32_t kSmemK0 = 0;
 constexpr uint32_t kSmemV0 = kSmemK0 + kKBufs * kKVBytes;
-constexpr uint32_t kSmemP = kSmemV0 + 2 * kKVBytes;
-constexpr uint32_t kSmemBar = kSmemP + kPBytes;
-constexpr uint32_t kSmemTotal = kSmemBar + 64 + 1024;  // + alignment slack
-// TMEM: S buffers at columns 0 and 64, Q (the A operand of S = Q K^T: bf16 pairs,
+constexpr uint32_t kSmemP0 = kSmemV0 + kVBufs * kKVBytes;
+constexpr uint32_t kSmemBar = kSmemP0 + kPBufs * kPBytes;
+constexpr int kNumBars = 2 * kKBufs /* k_full, k_empty */ + 2 * kVBufs /* v_full, pv_done */ +
+                         2 * 2 /* s_full, s_empty */ + kPBufs /* p_full */ + 2 /* q_full, mma_done */;
+constexpr uint32_t kSmemTotal = kSmemBar + kNumBars * 8 + 16 + 1024;  // + TMEM slot + alignment slack
+static_assert(kSmemTotal <= 232448, "shared memory per CTA");
+// TMEM: S buffers at columns 0 and 64, Q (A operand of S = Q K^T: bf16 pairs,
 // K-major, row = lane) at 128..255, O at 256..511
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTmemQ = 128;
 constexpr uint32_t kTmemO = 256;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleSlack = 8.0f;  // log2 units
+constexpr int kThreads = 224;
+constexpr unsigned kFull = 0xffffffffu;
 }  // namespace
 
-// Source row (256 bf16) of key `kk` of sample b: valid prefix positions first, then
-// the state key, then the action keys.
-__device__ __forceinline__ const bf16 *key_row(int kk, int nv, int b, const Geo &g, const bf16 *pref,
-                                                const int *vi, const bf16 *suf) {
-  if (kk < nv) return pref + ((size_t)b * g.P + vi[kk]) * kHeadDim;
-  const int row = (kk == nv) ? b : g.B + b * g.H + (kk - nv - 1);
-  return suf + (size_t)row * kHeadDim;
+// Source of key slot kk of sample b: 2*row for row `row` of the prefix tensor (B*P
+// rows), 2*row+1 for row `row` of this layer's suffix K/V, -1 for an empty slot.
+__device__ __forceinline__ int slot_code(int kk, int nbp, int nv, int b, const Geo &g, const int *vi) {
+  const int pre = nbp * kKeyBlock;
+  if (kk < pre) return kk < nv ? 2 * (b * g.P + vi[kk]) : -1;
+  const int s = kk - pre;
+  if (s < g.H) return 2 * (g.B + b * g.H + s) + 1;  // action key s
+  if (s == g.H) return 2 * b + 1;                     // state key
+  return -1;
 }
 
-__global__ void __launch_bounds__(128, 1)
-    k_attn_tc(const bf16 *q, const bf16 *ks, const bf16 *vs, const CallPtrs *cp, int layer, const int *nvalid,
-              const int *vidx, Geo g, int step0, int blocks_per_split, bf16 *out, float *part_o, float *part_ml,
-              unsigned *err) {
+// One warp fills the [64 keys x 256] tile at `tile` (4 sub-tiles of 64 dims) with the
+// K or V rows of key block `blk`.  Each 8-slot atom whose slots are consecutive rows of
+// one tensor, or are all empty, is one 8-row TMA box per sub-tile (an empty atom is
+// read at row -8, entirely out of bounds, which fills zeros and reads nothing); every
+// other atom is copied row by row with cp.async (16 B per lane, zeros for empty
+// slots).  `full` completes on the TMA bytes plus one cp.async arrival per lane.
+__device__ __forceinline__ void load_kv_tile(int blk, uint32_t tile, uint64_t *full, const CUtensorMap *pmap,
+                                             const CUtensorMap *smap, int sfx_row0, const bf16 *pref,
+                                             const bf16 *suf, int nbp, int nv, int b, const Geo &g, const int *vi,
+                                             int lane) {
+  const int kb = blk * kKeyBlock;
+  int code[2];
+  code[0] = slot_code(kb + lane, nbp, nv, b, g, vi);
+  code[1] = slot_code(kb + 32 + lane, nbp, nv, b, g, vi);
+  unsigned tma_atoms = 0, copy_atoms = 0;  // bit a: slots [8a, 8a + 8)
+#pragma unroll
+  for (int hh = 0; hh < 2; ++hh) {
+    const int lead = __shfl_sync(kFull, code[hh], lane & ~7);
+    const bool run = lead >= 0 && code[hh] == lead + 2 * (lane & 7);
+    const unsigned br = __ballot_sync(kFull, run), be = __ballot_sync(kFull, code[hh] < 0);
+#pragma unroll
+    for (int a = 0; a < 4; ++a) {
+      const bool whole = ((br >> (8 * a)) & 0xffu) == 0xffu || ((be >> (8 * a)) & 0xffu) == 0xffu;
+      (whole ? tma_atoms : copy_atoms) |= 1u << (4 * hh + a);
+    }
+  }
+  if (lane == 0 && tma_atoms) mbar_expect_tx(full, (uint32_t)__popc(tma_atoms) * 4u * kAtomBytes);
+  __syncwarp();
+  if ((lane & 7) == 0) {  // lane 8i issues atoms i and 4 + i
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+      const int a = 4 * hh + (lane >> 3);
+      if (!((tma_atoms >> a) & 1u)) continue;
+      const int c = code[hh];
+      const CUtensorMap *m = (c >= 0 && !(c & 1)) ? pmap : smap;
+      const int y = c < 0 ? -8 : (c & 1) ? sfx_row0 + (c >> 1) : (c >> 1);
+#pragma unroll
+      for (int sub = 0; sub < 4; ++sub) tma_load_2d(tile + sub * kSubTile + a * kAtomBytes, m, sub * 64, y, full);
+    }
+  }
+  while (copy_atoms) {  // warp-uniform
+    const int a = __ffs(copy_atoms) - 1;
+    copy_atoms &= copy_atoms - 1;
+    const int hh = a >> 2, l0 = (a & 3) * 8;
+#pragma unroll 4
+    for (int r = 0; r < 8; ++r) {
+      const int c = __shfl_sync(kFull, hh ? code[1] : code[0], l0 + r);
+      const bf16 *row = c < 0 ? suf : ((c & 1) ? suf : pref) + (size_t)(c >> 1) * kHeadDim;
+      cp_async16(tile + (lane >> 3) * kSubTile + sw128_off(8 * a + r, lane & 7), row + lane * 8, c >= 0);
+    }
+  }
+  cp_async_mbar_arrive(full);
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    k_attn_tc(const bf16 *q, const bf16 *ks, const bf16 *vs, const CallPtrs *cp, int layer, int sfx_row0,
+              const int *nvalid, const int *vidx, Geo g, int step0, int blocks_per_split, bf16 *out, float *part_o,
+              float *part_ml, unsigned *err) {
   pdl_wait();
   pdl_trigger();
   if (*(volatile unsigned *)err != 0) return;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
-  uint64_t *bar_s = reinterpret_cast<uint64_t *>(smem + kSmemBar);  // [2]
-  uint64_t *bar_o = bar_s + 2;
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar_s + 3);
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kSmemBar);
+  uint64_t *k_full = bars, *k_empty = bars + kKBufs;
+  uint64_t *v_full = bars + 2 * kKBufs, *pv_done = v_full + kVBufs;
+  uint64_t *s_full = pv_done + kVBufs, *s_empty = s_full + 2;
+  uint64_t *p_full = s_empty + 2, *q_full = p_full + kPBufs, *mma_done = q_full + 1;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mma_done + 1);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int b = blockIdx.z, split = blockIdx.y, nsplit = gridDim.y;
@@ -73,293 +151,278 @@ __global__ void __launch_bounds__(128, 1)
   const int nrows = kHeads * Tq;
   const int row0 = blockIdx.x * kRowsPerCta;
   const int nv = nvalid[b];
-  const int nk = nv + 1 + g.H;
-  const int nblk_all = (nk + kKeyBlock - 1) / kKeyBlock;
+  const int nbp = (nv + kKeyBlock - 1) / kKeyBlock;  // prefix blocks, then the suffix blocks
+  const int nblk_all = nbp + (g.H + kKeyBlock) / kKeyBlock;
   const int blk0 = split * blocks_per_split;
   const int blk1 = min(nblk_all, blk0 + blocks_per_split);
   const int nb = blk1 > blk0 ? blk1 - blk0 : 0;
 
-  // this thread's query row
-  const int qi = row0 + tid;
-  const bool row_ok = qi < nrows;
-  const int jq = qi / kHeads, head = qi % kHeads;
-  int tok = 0;
-  if (row_ok) tok = step0 ? (jq == 0 ? b : g.B + b * g.H + jq - 1) : g.B + b * g.H + jq;
-  const bool state_q = step0 && jq == 0;
-  const int key_lim = state_q ? nv + 1 : nk;  // keys [0, key_lim) visible to this row
-
-  const bf16 *pref_k = cp->prefix_k[layer], *pref_v = cp->prefix_v[layer];
-  const int *vi = vidx + (size_t)b * g.P;
-
   if (tid == 0) {
-    mbar_init(&bar_s[0], 1);
-    mbar_init(&bar_s[1], 1);
-    mbar_init(bar_o, 1);
+    for (int i = 0; i < kKBufs; ++i) {
+      mbar_init(&k_full[i], 32);  // one cp.async-completion arrival per loader lane (+ TMA bytes)
+      mbar_init(&k_empty[i], 1);  // tcgen05.commit after S
+    }
+    for (int i = 0; i < kVBufs; ++i) {
+      mbar_init(&v_full[i], 32);
+      mbar_init(&pv_done[i], 1);  // tcgen05.commit after P.V
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s_full[i], 1);     // tcgen05.commit after S
+      mbar_init(&s_empty[i], 128);  // every softmax thread has read its S row
+    }
+    for (int i = 0; i < kPBufs; ++i) mbar_init(&p_full[i], 128);
+    mbar_init(q_full, 128);
+    mbar_init(mma_done, 1);
     fence_mbar_init();
   }
   if (warp == 0) {
     tmem_alloc(tmem_slot, kTmemCols);
     tmem_relinquish();
   }
-
-  // Warp w copies keys [16w, 16w+16) of block j, lane = 16-byte chunk of the 512-byte
-  // row.  Lanes 0..15 first look up one key's source row each (independent loads),
-  // then every copy takes its row pointer from a shuffle.  `which`: 1 = K, 2 = V.
-  auto load_block = [&](int j, int which) {
-    if (j >= nb) return;
-    const int blk = blk0 + j;
-    const uint32_t kb = sbase + kSmemK0 + (j % kKBufs) * kKVBytes, vb = sbase + kSmemV0 + (j & 1) * kKVBytes;
-    const int kk_l = blk * kKeyBlock + warp * 16 + (lane & 15);
-    const bool ok_l = kk_l < nk;
-    const bf16 *krow = ks, *vrow = vs;
-    if (ok_l) {
-      if (which & 1) krow = key_row(kk_l, nv, b, g, pref_k, vi, ks);
-      if (which & 2) vrow = key_row(kk_l, nv, b, g, pref_v, vi, vs);
-    }
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const int r = warp * 16 + i;
-      const bool ok = __shfl_sync(0xffffffffu, ok_l, i);
-      const uint32_t off = (lane >> 3) * (64 * 128) + sw128_off(r, lane & 7);
-      if (which & 1) {
-        const bf16 *ksrc = reinterpret_cast<const bf16 *>(
-            __shfl_sync(0xffffffffu, reinterpret_cast<uintptr_t>(krow), i));
-        cp_async16(kb + off, ksrc + lane * 8, ok);
-      }
-      if (which & 2) {
-        const bf16 *vsrc = reinterpret_cast<const bf16 *>(
-            __shfl_sync(0xffffffffu, reinterpret_cast<uintptr_t>(vrow), i));
-        cp_async16(vb + off, vsrc + lane * 8, ok);
-      }
-    }
-  };
-
-  // cp.async groups, committed in this order (empty groups keep the pattern):
-  //   prologue: [K0, V0] [K1] [K2] [K3] [V1];
-  //   iteration w: [K(w+4)] after S(w), [V(w+1)] after PV(w-1) (empty at w = 0)
-  load_block(0, 3);
-  cp_async_commit();
-  load_block(1, 1);
-  cp_async_commit();
-  load_block(2, 1);
-  cp_async_commit();
-  load_block(3, 1);
-  cp_async_commit();
-  load_block(1, 2);
-  cp_async_commit();
-
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t t_lane = (uint32_t)(warp * 32) << 16;
+  bool ok = true;
 
-  // ---- Q: this thread's query row (256 bf16) into TMEM lane `tid`, columns 128..255,
-  // two bf16 per 32-bit column (the K-major A-operand layout of tcgen05.mma) ----
-  {
-    const uint4 *src = reinterpret_cast<const uint4 *>(q + (size_t)tok * kQDim + head * kHeadDim);
+  if (warp == 4 || warp == 5) {
+    // ------------------------------------------------------------ K / V loaders
+    const bool is_v = warp == 5;
+    const CUtensorMap *pmap = &cp->kv_map[is_v][layer], *smap = &cp->sfx_map[is_v];
+    const bf16 *pref = is_v ? cp->prefix_v[layer] : cp->prefix_k[layer];
+    const bf16 *suf = is_v ? vs : ks;
+    const int *vi = vidx + (size_t)b * g.P;
+    const int nbuf = is_v ? kVBufs : kKBufs;
+    uint64_t *full = is_v ? v_full : k_full;
+    // a buffer is free again once S (K) or P.V (V) of the block it held has completed
+    uint64_t *empty = is_v ? pv_done : k_empty;
+    const uint32_t ring = sbase + (is_v ? kSmemV0 : kSmemK0);
+    if (lane == 0) {  // (the prefix map is unused, and zero, when there is no prefix key)
+      if (nv > 0) {
+        tma_map_acquire(pmap);
+        tma_prefetch_desc(pmap);
+      }
+      tma_map_acquire(smap);
+      tma_prefetch_desc(smap);
+    }
+    __syncwarp();
+    for (int j = 0; j < nb; ++j) {
+      const int buf = j % nbuf;
+      if (j >= nbuf) ok = __all_sync(kFull, mbar_wait(&empty[buf], ((j / nbuf) - 1) & 1, err, kErrTimeoutProducer));
+      if (!ok) break;
+      load_kv_tile(blk0 + j, ring + buf * kKVBytes, &full[buf], pmap, smap, sfx_row0, pref, suf, nbp, nv, b, g, vi,
+                   lane);
+    }
+    cp_async_commit();  // nothing may still land in shared memory once the CTA exits
+    cp_async_wait<0>();
+  } else if (warp == 6) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0 && nb > 0) {
+      constexpr uint32_t idesc_s = idesc_bf16_f32(128, kKeyBlock);
+      constexpr uint32_t idesc_o = idesc_bf16_f32(128, kHeadDim) | (1u << 16);  // B (V) MN-major
+      auto issue_s = [&](int j) -> bool {  // S[j&1] = Q K(j)^T, Q from TMEM
+        const int kbuf = j % kKBufs, sb = j & 1;
+        if (!mbar_wait(&k_full[kbuf], (j / kKBufs) & 1, err, kErrTimeoutMma)) return false;
+        if (j >= 2 && !mbar_wait(&s_empty[sb], ((j >> 1) - 1) & 1, err, kErrTimeoutMma)) return false;
+        fence_proxy_async_smem();
+        tc_fence_after();
+        const uint32_t kb = sbase + kSmemK0 + kbuf * kKVBytes;
+        const uint32_t d = tmem + (uint32_t)(sb * kKeyBlock);
+#pragma unroll
+        for (int s = 0; s < 4; ++s)
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            tc_mma_bf16_ts(d, tmem + kTmemQ + (uint32_t)(32 * s + 8 * kk),
+                           smem_desc_k_sw128(kb + s * (64 * 128), kk * 32), idesc_s, (s | kk) != 0);
+        tc_commit(&s_full[sb]);
+        tc_commit(&k_empty[kbuf]);
+        return true;
+      };
+      auto issue_pv = [&](int j) -> bool {  // O += P(j) V(j)
+        const int vbuf = j % kVBufs, pb = j % kPBufs;
+        if (!mbar_wait(&p_full[pb], (j / kPBufs) & 1, err, kErrTimeoutMma)) return false;
+        if (!mbar_wait(&v_full[vbuf], (j / kVBufs) & 1, err, kErrTimeoutMma)) return false;
+        fence_proxy_async_smem();
+        tc_fence_after();
+        const uint32_t vb = sbase + kSmemV0 + vbuf * kKVBytes, pbase = sbase + kSmemP0 + pb * kPBytes;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          tc_mma_bf16(tmem + kTmemO, smem_desc_k_sw128(pbase, kk * 32),
+                      smem_desc_mn_sw128(vb + kk * 2048, 64 * 128, 1024), idesc_o, (j | kk) != 0);
+        tc_commit(&pv_done[vbuf]);  // V buffer and P buffer free, O updated
+        return true;
+      };
+      ok = mbar_wait(q_full, 0, err, kErrTimeoutMma);
+      tc_fence_after();
+      if (ok) ok = issue_s(0);
+      for (int j = 0; j < nb && ok; ++j) {
+        if (j + 1 < nb) ok = issue_s(j + 1);
+        if (ok) ok = issue_pv(j);
+      }
+      // every MMA issued (also after a failed wait) has finished before TMEM is freed
+      tc_commit(mma_done);
+      mbar_wait(mma_done, 0, err, kErrTimeoutMma);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ softmax warps 0..3
+    const int qi = row0 + tid;
+    const bool row_ok = qi < nrows;
+    const int jq = qi / kHeads, head = qi % kHeads;
+    int tok = 0;
+    if (row_ok) tok = step0 ? (jq == 0 ? b : g.B + b * g.H + jq - 1) : g.B + b * g.H + jq;
+    const bool state_q = step0 && jq == 0;
+    // visible suffix slots: the action keys (not for the state query) and the state key
+    const int sfx_lo = nbp * kKeyBlock + (state_q ? g.H : 0), sfx_hi = nbp * kKeyBlock + g.H + 1;
+    const uint32_t t_lane = (uint32_t)(warp * 32) << 16;
+    const float scale_l2 = 0.0625f * kLog2e;
+
+    // Q row -> TMEM lane tid, columns 128..255 (two bf16 per 32-bit column)
+    {
+      const uint4 *src = reinterpret_cast<const uint4 *>(q + (size_t)tok * kQDim + head * kHeadDim);
 #pragma unroll 1
-    for (int c = 0; c < 4; ++c) {
-      float v[32];
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const uint4 u = row_ok ? src[c * 8 + e] : make_uint4(0, 0, 0, 0);
-        v[4 * e] = __uint_as_float(u.x);
-        v[4 * e + 1] = __uint_as_float(u.y);
-        v[4 * e + 2] = __uint_as_float(u.z);
-        v[4 * e + 3] = __uint_as_float(u.w);
-      }
-      tmem_st_32x32b_x32(tmem + t_lane + kTmemQ + 32 * c, v);
-    }
-  }
-
-  constexpr uint32_t idesc_s = idesc_bf16_f32(128, kKeyBlock);
-  constexpr uint32_t idesc_o = idesc_bf16_f32(128, kHeadDim) | (1u << 16);  // B (V) MN-major
-  const float scale_l2 = 0.0625f * kLog2e;
-
-  auto issue_s = [&](int j) {  // S[j&1] = Q K(j)^T, A (Q) from TMEM, 16 head dims per MMA
-    const uint32_t kb = sbase + kSmemK0 + (j % kKBufs) * kKVBytes;
-    const uint32_t d = tmem + (uint32_t)((j & 1) * kKeyBlock);
-#pragma unroll
-    for (int s = 0; s < 4; ++s)
-#pragma unroll
-      for (int kk = 0; kk < 4; ++kk)
-        tc_mma_bf16_ts(d, tmem + kTmemQ + (uint32_t)(32 * s + 8 * kk), smem_desc_k_sw128(kb + s * (64 * 128), kk * 32),
-                       idesc_s, (s | kk) != 0);
-    tc_commit(&bar_s[j & 1]);
-  };
-
-  float m_used = -INFINITY, l = 0.f;
-  uint32_t ph_s0 = 0, ph_s1 = 0, ph_o = 0;
-  bool ok_all = true;
-  if (nb > 0) {
-    cp_async_wait<4>();
-    fence_proxy_async_smem();
-    tc_fence_before();
-    ok_all = __syncthreads_and(ok_all);
-    tc_fence_after();
-    if (tid == 0 && ok_all) issue_s(0);
-  }
-  for (int w = 0; w < nb && ok_all; ++w) {
-    const int buf = w & 1;
-    // (1) K(w+1) has landed: start S(w+1) on the tensor cores before the softmax of w.
-    // Groups committed after K(w+1): 3 at w = 0, 4 at w = 1, then 5.
-    if (w + 1 < nb) {
-      if (w == 0)
-        cp_async_wait<3>();
-      else if (w == 1)
-        cp_async_wait<4>();
-      else
-        cp_async_wait<5>();
-      fence_proxy_async_smem();
-      tc_fence_before();
-      ok_all = __syncthreads_and(ok_all);
-      tc_fence_after();
-      if (!ok_all) break;
-      if (tid == 0) issue_s(w + 1);
-    }
-    // (2) softmax of block w
-    {
-      uint32_t &ph = buf ? ph_s1 : ph_s0;
-      if (!mbar_wait(&bar_s[buf], ph, err, kErrTimeoutEpilogue)) ok_all = false;
-      ph ^= 1u;
-    }
-    __syncwarp();
-    tc_fence_after();
-    // K(w)'s buffer is free again (S(w) done): prefetch K(w+4)
-    load_block(w + kKBufs, 1);
-    cp_async_commit();
-    float sv[64];
-    {
-      float t0[32], t1[32];
-      tmem_ld_32x32b_x32(tmem + t_lane + buf * kKeyBlock, t0);
-      tmem_ld_32x32b_x32(tmem + t_lane + buf * kKeyBlock + 32, t1);
-#pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        sv[i] = t0[i];
-        sv[32 + i] = t1[i];
-      }
-    }
-    const int kbase = (blk0 + w) * kKeyBlock;
-    float bm = -INFINITY;
-#pragma unroll
-    for (int i = 0; i < 64; ++i) {
-      sv[i] = (kbase + i < key_lim) ? sv[i] * scale_l2 : -INFINITY;
-      bm = fmaxf(bm, sv[i]);
-    }
-    // P(w-1) and O are in use by PV(w-1) until it completes
-    if (w >= 1) {
-      if (!mbar_wait(bar_o, ph_o, err, kErrTimeoutMma)) ok_all = false;
-      ph_o ^= 1u;
-      __syncwarp();
-      tc_fence_after();
-    }
-    // V(w-1)'s buffer is free: prefetch V(w+1) (V(1) came with the prologue)
-    if (w >= 1) load_block(w + 1, 2);
-    cp_async_commit();
-    if (bm > m_used + kRescaleSlack) {
-      const float alpha = ex2_approx(m_used - bm);  // 0 while m_used = -inf
-      l *= alpha;
-      if (w >= 1) {
-        for (int c = 0; c < kHeadDim; c += 32) {
-          float o[32];
-          tmem_ld_32x32b_x32(tmem + t_lane + kTmemO + c, o);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] *= alpha;
-          tmem_st_32x32b_x32(tmem + t_lane + kTmemO + c, o);
-        }
-      }
-      m_used = bm;
-    }
-    {
-      // no visible key seen yet <=> m_used = -inf <=> every sv is -inf: use 0 so that 2^(-inf) = 0
-      const float mu = m_used == -INFINITY ? 0.f : m_used;
-      uint8_t *prow = smem + kSmemP;
-#pragma unroll
-      for (int cc = 0; cc < 8; ++cc) {
-        uint32_t pk[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int i0 = cc * 8 + 2 * e;
-          const float p0 = ex2_approx(sv[i0] - mu), p1 = ex2_approx(sv[i0 + 1] - mu);
-          l += p0 + p1;
-          const __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
-          pk[e] = *reinterpret_cast<const uint32_t *>(&h2);
-        }
-        *reinterpret_cast<uint4 *>(prow + sw128_off(tid, cc)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-      }
-    }
-    // V(w) must have landed: groups committed after it are 6 at w = 0 (it came with
-    // K0), 4 at w = 1 (it came last in the prologue), then the 2 of this iteration
-    if (w == 0)
-      cp_async_wait<6>();
-    else if (w == 1)
-      cp_async_wait<4>();
-    else
-      cp_async_wait<2>();
-    fence_proxy_async_smem();
-    tc_fence_before();
-    ok_all = __syncthreads_and(ok_all);
-    tc_fence_after();
-    if (!ok_all) break;
-    if (tid == 0) {
-      const uint32_t vb = sbase + kSmemV0 + buf * kKVBytes;
-#pragma unroll
-      for (int kk = 0; kk < 4; ++kk)
-        tc_mma_bf16(tmem + kTmemO, smem_desc_k_sw128(sbase + kSmemP, kk * 32),
-                    smem_desc_mn_sw128(vb + kk * 2048, 64 * 128, 1024), idesc_o, (w | kk) != 0);
-      tc_commit(bar_o);
-    }
-    __syncwarp();
-  }
-  // last PV MMA
-  if (nb > 0 && ok_all) {
-    if (!mbar_wait(bar_o, ph_o, err, kErrTimeoutMma)) ok_all = false;
-    __syncwarp();
-  }
-  cp_async_wait<0>();
-  tc_fence_after();
-  const bool write = __syncthreads_and(ok_all);
-  const float inv_l = l > 0.f ? 1.0f / l : 0.f;
-  if (write) {
-    if (nsplit == 1) {
-      bf16 *dst = out + (size_t)tok * kQDim + head * kHeadDim;
-      for (int c = 0; c < kHeadDim; c += 32) {
+      for (int c = 0; c < 4; ++c) {
         float v[32];
-        tmem_ld_32x32b_x32(tmem + t_lane + kTmemO + c, v);  // warp-collective: all lanes
-        if (row_ok) {
-          uint32_t pk[16];
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const __nv_bfloat162 h2 = __floats2bfloat162_rn(v[2 * e] * inv_l, v[2 * e + 1] * inv_l);
+        for (int e = 0; e < 8; ++e) {
+          const uint4 u = row_ok ? src[c * 8 + e] : make_uint4(0, 0, 0, 0);
+          v[4 * e] = __uint_as_float(u.x);
+          v[4 * e + 1] = __uint_as_float(u.y);
+          v[4 * e + 2] = __uint_as_float(u.z);
+          v[4 * e + 3] = __uint_as_float(u.w);
+        }
+        tmem_st_32x32b_x32(tmem + t_lane + kTmemQ + 32 * c, v);
+      }
+      tc_fence_before();
+      mbar_arrive(q_full);
+    }
+
+    float m_used = -INFINITY, l = 0.f;
+    for (int j = 0; j < nb && ok; ++j) {
+      const int sb = j & 1, pb = j % kPBufs;
+      ok = __all_sync(0xffffffffu, mbar_wait(&s_full[sb], (j >> 1) & 1, err, kErrTimeoutEpilogue));
+      if (!ok) break;
+      tc_fence_after();
+      float sv[64];
+      {
+        float t0[32], t1[32];
+        tmem_ld_32x32b_x32(tmem + t_lane + sb * kKeyBlock, t0);
+        tmem_ld_32x32b_x32(tmem + t_lane + sb * kKeyBlock + 32, t1);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          sv[i] = t0[i];
+          sv[32 + i] = t1[i];
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&s_empty[sb]);
+      const int kbase = (blk0 + j) * kKeyBlock;
+      const int vis_lo = blk0 + j < nbp ? 0 : sfx_lo, vis_hi = blk0 + j < nbp ? nv : sfx_hi;
+      float bm = -INFINITY;
+#pragma unroll
+      for (int i = 0; i < 64; ++i) {
+        sv[i] = (unsigned)(kbase + i - vis_lo) < (unsigned)(vis_hi - vis_lo) ? sv[i] * scale_l2 : -INFINITY;
+        bm = fmaxf(bm, sv[i]);
+      }
+      // Raise m_used (and rescale l, O) when this block's max exceeds it by more than
+      // 2^8.  O lives in TMEM and tcgen05.ld/st are warp-collective, so the whole warp
+      // takes the branch when any lane needs it; the other lanes scale by 1 (exact).
+      const bool mine = bm > m_used + kRescaleSlack;
+      if (__any_sync(0xffffffffu, mine)) {
+        const float alpha = mine ? ex2_approx(m_used - bm) : 1.0f;  // 0 while m_used = -inf
+        l *= alpha;
+        if (j >= 1) {  // O holds P.V of blocks < j: wait for the last of them
+          const int pj = j - 1;
+          ok = __all_sync(0xffffffffu, mbar_wait(&pv_done[pj % kVBufs], (pj / kVBufs) & 1, err, kErrTimeoutEpilogue));
+          if (!ok) break;
+          tc_fence_after();
+          for (int c = 0; c < kHeadDim; c += 32) {
+            float o[32];
+            tmem_ld_32x32b_x32(tmem + t_lane + kTmemO + c, o);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] *= alpha;
+            tmem_st_32x32b_x32(tmem + t_lane + kTmemO + c, o);
+          }
+          tc_fence_before();
+        }
+        if (mine) m_used = bm;
+      }
+      // P buffer pb was last read by P.V(j - 2)
+      if (j >= kPBufs) {
+        const int pj = j - kPBufs;
+        ok = __all_sync(0xffffffffu, mbar_wait(&pv_done[pj % kVBufs], (pj / kVBufs) & 1, err, kErrTimeoutEpilogue));
+        if (!ok) break;
+      }
+      {
+        // no visible key seen yet <=> m_used = -inf <=> every sv is -inf: use 0 so that 2^(-inf) = 0
+        const float mu = m_used == -INFINITY ? 0.f : m_used;
+        uint8_t *prow = smem + kSmemP0 + pb * kPBytes;
+#pragma unroll
+        for (int cc = 0; cc < 8; ++cc) {
+          uint32_t pk[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int i0 = cc * 8 + 2 * e;
+            const float p0 = ex2_approx(sv[i0] - mu), p1 = ex2_approx(sv[i0 + 1] - mu);
+            l += p0 + p1;
+            const __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
             pk[e] = *reinterpret_cast<const uint32_t *>(&h2);
           }
-          uint4 *d4 = reinterpret_cast<uint4 *>(dst + c);
-#pragma unroll
-          for (int e = 0; e < 4; ++e) d4[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+          *reinterpret_cast<uint4 *>(prow + sw128_off(tid, cc)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
         }
       }
-    } else {
-      // split partials: O normalised by this split's l, plus (m, l) in log2 units
-      const size_t prow = ((size_t)b * nsplit + split) * (size_t)(gridDim.x * kRowsPerCta) + qi;
-      for (int c = 0; c < kHeadDim; c += 32) {
-        float v[32];
-        if (nb > 0) {
-          tmem_ld_32x32b_x32(tmem + t_lane + kTmemO + c, v);
-        } else {
+      fence_proxy_async_smem();
+      mbar_arrive(&p_full[pb]);
+    }
+    // final P.V
+    if (nb > 0 && ok) {
+      const int pj = nb - 1;
+      ok = __all_sync(0xffffffffu, mbar_wait(&pv_done[pj % kVBufs], (pj / kVBufs) & 1, err, kErrTimeoutEpilogue));
+    }
+    tc_fence_after();
+    const bool write = __all_sync(0xffffffffu, ok);
+    const float inv_l = l > 0.f ? 1.0f / l : 0.f;
+    if (write) {
+      if (nsplit == 1) {
+        bf16 *dst = out + (size_t)tok * kQDim + head * kHeadDim;
+        for (int c = 0; c < kHeadDim; c += 32) {
+          float v[32];
+          tmem_ld_32x32b_x32(tmem + t_lane + kTmemO + c, v);  // warp-collective: all lanes
+          if (row_ok) {
+            uint32_t pk[16];
 #pragma unroll
-          for (int e = 0; e < 32; ++e) v[e] = 0.f;
+            for (int e = 0; e < 16; ++e) {
+              const __nv_bfloat162 h2 = __floats2bfloat162_rn(v[2 * e] * inv_l, v[2 * e + 1] * inv_l);
+              pk[e] = *reinterpret_cast<const uint32_t *>(&h2);
+            }
+            uint4 *d4 = reinterpret_cast<uint4 *>(dst + c);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) d4[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+          }
+        }
+      } else {
+        // split partials: O normalised by this split's l, plus (m, l) in log2 units
+        const size_t prow = ((size_t)b * nsplit + split) * (size_t)(gridDim.x * kRowsPerCta) + qi;
+        for (int c = 0; c < kHeadDim; c += 32) {
+          float v[32];
+          if (nb > 0) {
+            tmem_ld_32x32b_x32(tmem + t_lane + kTmemO + c, v);
+          } else {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) v[e] = 0.f;
+          }
+          if (row_ok) {
+            float4 *d4 = reinterpret_cast<float4 *>(part_o + prow * kHeadDim + c);
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              d4[e] = make_float4(v[4 * e] * inv_l, v[4 * e + 1] * inv_l, v[4 * e + 2] * inv_l,
+                                  v[4 * e + 3] * inv_l);
+          }
         }
         if (row_ok) {
-          float4 *d4 = reinterpret_cast<float4 *>(part_o + prow * kHeadDim + c);
-#pragma unroll
-          for (int e = 0; e < 8; ++e)
-            d4[e] = make_float4(v[4 * e] * inv_l, v[4 * e + 1] * inv_l, v[4 * e + 2] * inv_l, v[4 * e + 3] * inv_l);
+          part_ml[2 * prow] = m_used;
+          part_ml[2 * prow + 1] = l;
         }
-      }
-      if (row_ok) {
-        part_ml[2 * prow] = m_used;
-        part_ml[2 * prow + 1] = l;
       }
     }
   }
@@ -406,10 +469,12 @@ __global__ void __launch_bounds__(256) k_attn_combine(const float *part_o, const
   for (int e = 0; e < 8; ++e) dst[lane + 32 * e] = __float2bfloat16_rn(acc[e] * inv);
 }
 
-int attn_tc_splits(const Geo &g, int step0, int max_keys) {
+int attn_tc_blocks(int P, int H) { return (P + kKeyBlock - 1) / kKeyBlock + (H + kKeyBlock) / kKeyBlock; }
+
+int attn_tc_splits(const Geo &g, int step0) {
   const int Tq = step0 ? g.H + 1 : g.H;
   const int mtiles = (kHeads * Tq + kRowsPerCta - 1) / kRowsPerCta;
-  const int nblk = (max_keys + kKeyBlock - 1) / kKeyBlock;
+  const int nblk = attn_tc_blocks(g.P, g.H);
   const int ctas = mtiles * g.B;
   if (ctas >= 96) return 1;
   int splits = (148 + ctas - 1) / ctas;
@@ -425,20 +490,28 @@ size_t attn_tc_partial_floats(const Geo &g, int step0, int splits) {
   return (size_t)g.B * splits * mtiles * kRowsPerCta * (kHeadDim + 2);
 }
 
+bool attn_tc_maps(CallPtrs &cp, int layers, int B, int P, const void *ks, const void *vs, uint64_t sfx_rows) {
+  for (int l = 0; l < layers && P > 0; ++l)
+    if (!make_map(&cp.kv_map[0][l], cp.prefix_k[l], (uint64_t)B * P, kHeadDim, kHeadDim, 8) ||
+        !make_map(&cp.kv_map[1][l], cp.prefix_v[l], (uint64_t)B * P, kHeadDim, kHeadDim, 8))
+      return false;
+  return make_map(&cp.sfx_map[0], ks, sfx_rows, kHeadDim, kHeadDim, 8) &&
+         make_map(&cp.sfx_map[1], vs, sfx_rows, kHeadDim, kHeadDim, 8);
+}
+
 void launch_attention_tc(const bf16 *q, const bf16 *ks, const bf16 *vs, const CallPtrs *cp, int layer,
-                         const int *nvalid, const int *vidx, const Geo &g, int step0, int splits, bf16 *out,
-                         float *part, unsigned *err, cudaStream_t s) {
+                         int sfx_row0, const int *nvalid, const int *vidx, const Geo &g, int step0, int splits,
+                         bf16 *out, float *part, unsigned *err, cudaStream_t s) {
   cudaFuncSetAttribute(k_attn_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemTotal);
   const int Tq = step0 ? g.H + 1 : g.H;
   const int mtiles = (kHeads * Tq + kRowsPerCta - 1) / kRowsPerCta;
-  const int max_keys = g.P + 1 + g.H;
-  const int nblk = (max_keys + kKeyBlock - 1) / kKeyBlock;
+  const int nblk = attn_tc_blocks(g.P, g.H);
   const int bps = (nblk + splits - 1) / splits;
   float *part_o = part;
   float *part_ml = splits > 1 ? part + (size_t)g.B * splits * mtiles * kRowsPerCta * kHeadDim : nullptr;
   dim3 grid(mtiles, splits, g.B);
-  launch_pdl(k_attn_tc, grid, 128, kSmemTotal, s, q, ks, vs, cp, layer, nvalid, vidx, g, step0, bps, out, part_o,
-             part_ml, err);
+  launch_pdl(k_attn_tc, grid, kThreads, kSmemTotal, s, q, ks, vs, cp, layer, sfx_row0, nvalid, vidx, g, step0, bps,
+             out, part_o, part_ml, err);
   if (splits > 1) {
     dim3 cg((kHeads * Tq + 7) / 8, g.B);
     launch_pdl(k_attn_combine, cg, 256, 0, s, part_o, part_ml, g, step0, splits, mtiles * kRowsPerCta, out);

@@ -21,6 +21,12 @@ typedef __nv_bfloat16 bf16;
 // stays valid when the caller's buffers change between calls.
 constexpr int kMaxDepth = 32;
 struct CallPtrs {
+  // bf16 mode: TMA maps of the attention keys and values, [0] = K, [1] = V.
+  // kv_map[.][l]: layer l's prefix tensor as B*P rows of 256 (encoded per call);
+  // sfx_map[.]: the suffix K/V of all layers as one tensor of rows x 256.
+  // Boxes are 64 columns x 8 rows with the 128-byte swizzle.
+  CUtensorMap kv_map[2][kMaxDepth];
+  CUtensorMap sfx_map[2];
   const bf16 *prefix_k[kMaxDepth];
   const bf16 *prefix_v[kMaxDepth];
   const uint8_t *mask;
@@ -144,11 +150,20 @@ void launch_attention(const T *q, const T *ks, const T *vs, const CallPtrs *cp, 
 
 // tcgen05 attention (k_attn_tc.cu); `part` holds attn_tc_partial_floats() floats
 // when splits > 1.
-int attn_tc_splits(const Geo &g, int step0, int max_keys);
+// Key slots per sample: ceil(P/64) blocks of valid prefix keys, then ceil((H+1)/64)
+// blocks holding the H action keys and the state key.
+int attn_tc_blocks(int P, int H);
+int attn_tc_splits(const Geo &g, int step0);
 size_t attn_tc_partial_floats(const Geo &g, int step0, int splits);
+// Encodes cp.kv_map for layers [0, layers) (prefix tensors cp.prefix_k/v[l], B*P rows)
+// and cp.sfx_map over `sfx_rows` rows at ks / vs.  False if an encode fails (e.g. a
+// pointer that is not 16-byte aligned).
+bool attn_tc_maps(CallPtrs &cp, int layers, int B, int P, const void *ks, const void *vs, uint64_t sfx_rows);
+// ks / vs: this layer's suffix rows, which start at row `sfx_row0` of cp->sfx_map.
 void launch_attention_tc(const bf16 *q, const bf16 *ks, const bf16 *vs, const CallPtrs *cp, int layer,
-                         const int *nvalid, const int *vidx, const Geo &g, int step0, int splits, bf16 *out,
-                         float *part, unsigned *err, cudaStream_t s);
+                         int sfx_row0, const int *nvalid, const int *vidx, const Geo &g, int step0, int splits,
+                         bf16 *out, float *part, unsigned *err, cudaStream_t s);
+bool make_map(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols, uint64_t pitch, uint32_t box_rows);
 
 // Text for pi0x_last_error() (this thread).
 void set_last_error(const char *msg);

@@ -78,7 +78,7 @@ extern "C" int pi0x_attention_noalloc(const void *q, const void *ks, const void 
       P < 0)
     return PI0X_EINVAL;
   Geo g{B, H, 32, 32, P, B + B * H};
-  const int splits = attn_tc_splits(g, step0, P + 1 + H);
+  const int splits = attn_tc_splits(g, step0);
   // scratch layout: [call table][error word][n_valid][valid-index list][split partials]
   const size_t off_cp = 0;
   const size_t off_err = align256(off_cp + sizeof(CallPtrs));
@@ -110,12 +110,16 @@ extern "C" int pi0x_attention_noalloc(const void *q, const void *ks, const void 
   cp.prefix_k[0] = (const bf16 *)prefix_k;
   cp.prefix_v[0] = (const bf16 *)prefix_v;
   cp.mask = (const uint8_t *)mask;
+  if (!attn_tc_maps(cp, 1, B, P, ks, vs, (uint64_t)g.R)) {
+    set_last_error("pi0x_attention_noalloc: cuTensorMapEncodeTiled failed (pointers must be 16-byte aligned)");
+    return PI0X_EINVAL;
+  }
   cudaStream_t s = (cudaStream_t)stream;
   cudaError_t e = cudaMemcpyAsync(d_cp, &cp, sizeof(cp), cudaMemcpyHostToDevice, s);
   if (e == cudaSuccess) e = cudaMemsetAsync(d_err, 0, sizeof(unsigned), s);
   if (e == cudaSuccess) {
     launch_prep_mask(d_cp, B, P, nvalid, vidx, s);
-    launch_attention_tc((const bf16 *)q, (const bf16 *)ks, (const bf16 *)vs, d_cp, 0, nvalid, vidx, g, step0, splits,
+    launch_attention_tc((const bf16 *)q, (const bf16 *)ks, (const bf16 *)vs, d_cp, 0, 0, nvalid, vidx, g, step0, splits,
                         (bf16 *)out, part, d_err, s);
     e = cudaGetLastError();
   }

@@ -45,6 +45,10 @@ struct Arena {
 };
 size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
+}  // namespace
+
+namespace pi0x {
+
 // ---- cuTensorMapEncodeTiled through the runtime's driver entry point ---------
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
@@ -73,6 +77,10 @@ bool make_map(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols, ui
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
+
+}  // namespace pi0x
+
+namespace {
 
 uint16_t f32_to_bf16_bits(float f) {
   uint32_t u;
@@ -497,10 +505,10 @@ int enqueue_loop(pi0x_handle *h, int B, int P, int N, cudaStream_t s) {
         RUN(PI0X_K_ROPE, launch_rope_qkv<T>(ws.raw, row0, M, g, ws.nvalid, h->inv_freq, q, ks, vs, s));
       }
       if (tc) {
-        const int splits = attn_tc_splits(g, step0, P + 1 + H);
+        const int splits = attn_tc_splits(g, step0);
         RUN(PI0X_K_ATTN, launch_attention_tc((const bf16 *)q, (const bf16 *)ks, (const bf16 *)vs, h->d_ptrs, l,
-                                             ws.nvalid, ws.vidx, g, step0, splits, (bf16 *)att, ws.part, h->d_err,
-                                             s));
+                                             l * R, ws.nvalid, ws.vidx, g, step0, splits, (bf16 *)att, ws.part,
+                                             h->d_err, s));
       } else {
         RUN(PI0X_K_ATTN, launch_attention<T>(q, ks, vs, h->d_ptrs, l, ws.nvalid, ws.vidx, g, step0, att, s));
       }
@@ -651,6 +659,10 @@ int pi0x_debug_attention(const void *q, const void *ks, const void *vs, const vo
   cp.prefix_k[0] = (const bf16 *)prefix_k;
   cp.prefix_v[0] = (const bf16 *)prefix_v;
   cp.mask = (const uint8_t *)mask;
+  if (impl != 0 && !attn_tc_maps(cp, 1, B, P, ks, vs, (uint64_t)g.R)) {
+    g_last_error = "pi0x_debug_attention: cuTensorMapEncodeTiled failed (pointers must be 16-byte aligned)";
+    return PI0X_EINVAL;
+  }
   CallPtrs *d_cp = nullptr;
   int *nvalid = nullptr, *vidx = nullptr;
   float *part = nullptr;
@@ -670,8 +682,8 @@ int pi0x_debug_attention(const void *q, const void *ks, const void *vs, const vo
       launch_attention<bf16>((const bf16 *)q, (const bf16 *)ks, (const bf16 *)vs, d_cp, 0, nvalid, vidx, g, step0,
                              (bf16 *)out, s);
     } else {
-      const int splits = impl == 2 ? 1 : attn_tc_splits(g, step0, P + 1 + H);
-      launch_attention_tc((const bf16 *)q, (const bf16 *)ks, (const bf16 *)vs, d_cp, 0, nvalid, vidx, g, step0,
+      const int splits = impl == 2 ? 1 : attn_tc_splits(g, step0);
+      launch_attention_tc((const bf16 *)q, (const bf16 *)ks, (const bf16 *)vs, d_cp, 0, 0, nvalid, vidx, g, step0,
                           splits, (bf16 *)out, part, err, s);
     }
     e = cudaGetLastError();
@@ -888,6 +900,10 @@ int pi0x_sample(pi0x_handle *h, const void *const *prefix_k, const void *const *
   cp.x1 = (const float *)tmp;
   const bool x0_host = !is_device_ptr(x0);
   cp.x0 = x0_host ? ws.st_x : x0;  // staged x1 is consumed before x0 is written
+  if (h->bf16 && !attn_tc_maps(cp, L, B, P, ws.ks, ws.vs, (uint64_t)L * (B + (size_t)B * H))) {
+    g_last_error = "pi0x_sample: cuTensorMapEncodeTiled failed for the prefix K/V (pointers must be 16-byte aligned)";
+    return PI0X_EINVAL;
+  }
   CK(cudaMemcpyAsync(h->d_ptrs, &cp, sizeof(cp), cudaMemcpyHostToDevice, s));
   if (h->prof_on) {
     // Profiled call: direct launches with an event pair around each kernel.  A
@@ -955,7 +971,7 @@ long pi0x_launch_count(const pi0x_handle *h, int B, int P, int num_steps) {
     // 2 GEMMs + RoPE, attention, O GEMM, GeGLU, down GEMM; bf16 mode fuses norms, RoPE
     // and GeGLU into the GEMMs (4 GEMMs + attention [+ split-KV combine]).
     long per_layer = h->bf16 ? 5 : 9;
-    if (h->bf16 && attn_tc_splits(g, k == 0, P + 1 + (int)H) > 1) per_layer += 1;  // split-KV combine
+    if (h->bf16 && attn_tc_splits(g, k == 0) > 1) per_layer += 1;  // split-KV combine
     n += 3 + L * per_layer + 1;
   }
   return n;
