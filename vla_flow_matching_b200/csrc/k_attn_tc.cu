@@ -65,9 +65,11 @@ constexpr unsigned kFull = 0xffffffffu;
 
 // Source of key slot kk of sample b: 2*row for row `row` of the prefix tensor (B*P
 // rows), 2*row+1 for row `row` of this layer's suffix K/V, -1 for an empty slot.
-__device__ __forceinline__ int slot_code(int kk, int nbp, int nv, int b, const Geo &g, const int *vi) {
+// `contig`: the valid prefix positions are exactly [0, nv), so slot kk is position kk
+// and the valid-index list need not be read.
+__device__ __forceinline__ int slot_code(int kk, int nbp, int nv, bool contig, int b, const Geo &g, const int *vi) {
   const int pre = nbp * kKeyBlock;
-  if (kk < pre) return kk < nv ? 2 * (b * g.P + vi[kk]) : -1;
+  if (kk < pre) return kk < nv ? 2 * (b * g.P + (contig ? kk : vi[kk])) : -1;
   const int s = kk - pre;
   if (s < g.H) return 2 * (g.B + b * g.H + s) + 1;  // action key s
   if (s == g.H) return 2 * b + 1;                     // state key
@@ -75,19 +77,35 @@ __device__ __forceinline__ int slot_code(int kk, int nbp, int nv, int b, const G
 }
 
 // One warp fills the [64 keys x 256] tile at `tile` (4 sub-tiles of 64 dims) with the
-// K or V rows of key block `blk`.  Each 8-slot atom whose slots are consecutive rows of
-// one tensor, or are all empty, is one 8-row TMA box per sub-tile (an empty atom is
-// read at row -8, entirely out of bounds, which fills zeros and reads nothing); every
-// other atom is copied row by row with cp.async (16 B per lane, zeros for empty
-// slots).  `full` completes on the TMA bytes plus one cp.async arrival per lane.
+// K or V rows of key block `blk`.  A block whose 64 slots are consecutive rows of one
+// tensor is one 64-row TMA box per sub-tile.  Otherwise each 8-slot atom whose slots
+// are consecutive rows of one tensor, or are all empty, is one 8-row box per sub-tile
+// (an empty atom is read at row -8, entirely out of bounds, which fills zeros and
+// reads nothing), and every other atom is copied row by row with cp.async (16 B per
+// lane, zeros for empty slots).  `full` completes on the TMA bytes plus one cp.async
+// arrival per lane.  Maps: p* = prefix, s* = suffix; *64 = 64-row boxes.
 __device__ __forceinline__ void load_kv_tile(int blk, uint32_t tile, uint64_t *full, const CUtensorMap *pmap,
-                                             const CUtensorMap *smap, int sfx_row0, const bf16 *pref,
-                                             const bf16 *suf, int nbp, int nv, int b, const Geo &g, const int *vi,
-                                             int lane) {
+                                             const CUtensorMap *smap, const CUtensorMap *pmap64,
+                                             const CUtensorMap *smap64, int sfx_row0, const bf16 *pref,
+                                             const bf16 *suf, int nbp, int nv, bool contig, int b, const Geo &g,
+                                             const int *vi, int lane) {
   const int kb = blk * kKeyBlock;
   int code[2];
-  code[0] = slot_code(kb + lane, nbp, nv, b, g, vi);
-  code[1] = slot_code(kb + 32 + lane, nbp, nv, b, g, vi);
+  code[0] = slot_code(kb + lane, nbp, nv, contig, b, g, vi);
+  code[1] = slot_code(kb + 32 + lane, nbp, nv, contig, b, g, vi);
+  const int c0 = __shfl_sync(kFull, code[0], 0);
+  if (__all_sync(kFull, c0 >= 0 && code[0] == c0 + 2 * lane && code[1] == c0 + 2 * (32 + lane))) {
+    if (lane == 0) {
+      mbar_expect_tx(full, kKVBytes);
+      const CUtensorMap *m = (c0 & 1) ? smap64 : pmap64;
+      const int y = (c0 & 1) ? sfx_row0 + (c0 >> 1) : (c0 >> 1);
+#pragma unroll
+      for (int sub = 0; sub < 4; ++sub) tma_load_2d(tile + sub * kSubTile, m, sub * 64, y, full);
+    }
+    __syncwarp();
+    cp_async_mbar_arrive(full);
+    return;
+  }
   unsigned tma_atoms = 0, copy_atoms = 0;  // bit a: slots [8a, 8a + 8)
 #pragma unroll
   for (int hh = 0; hh < 2; ++hh) {
@@ -189,9 +207,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ K / V loaders
     const bool is_v = warp == 5;
     const CUtensorMap *pmap = &cp->kv_map[is_v][layer], *smap = &cp->sfx_map[is_v];
+    const CUtensorMap *pmap64 = &cp->kv_map64[is_v][layer], *smap64 = &cp->sfx_map64[is_v];
     const bf16 *pref = is_v ? cp->prefix_v[layer] : cp->prefix_k[layer];
     const bf16 *suf = is_v ? vs : ks;
     const int *vi = vidx + (size_t)b * g.P;
+    // the list is strictly increasing, so its last entry is nv - 1 iff it is 0 .. nv-1
+    const bool contig = nv == 0 || vi[nv - 1] == nv - 1;
     const int nbuf = is_v ? kVBufs : kKBufs;
     uint64_t *full = is_v ? v_full : k_full;
     // a buffer is free again once S (K) or P.V (V) of the block it held has completed
@@ -200,59 +221,72 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {  // (the prefix map is unused, and zero, when there is no prefix key)
       if (nv > 0) {
         tma_map_acquire(pmap);
+        tma_map_acquire(pmap64);
         tma_prefetch_desc(pmap);
+        tma_prefetch_desc(pmap64);
       }
       tma_map_acquire(smap);
+      tma_map_acquire(smap64);
       tma_prefetch_desc(smap);
+      tma_prefetch_desc(smap64);
     }
     __syncwarp();
     for (int j = 0; j < nb; ++j) {
       const int buf = j % nbuf;
       if (j >= nbuf) ok = __all_sync(kFull, mbar_wait(&empty[buf], ((j / nbuf) - 1) & 1, err, kErrTimeoutProducer));
       if (!ok) break;
-      load_kv_tile(blk0 + j, ring + buf * kKVBytes, &full[buf], pmap, smap, sfx_row0, pref, suf, nbp, nv, b, g, vi,
-                   lane);
+      load_kv_tile(blk0 + j, ring + buf * kKVBytes, &full[buf], pmap, smap, pmap64, smap64, sfx_row0, pref, suf, nbp,
+                   nv, contig, b, g, vi, lane);
     }
     cp_async_commit();  // nothing may still land in shared memory once the CTA exits
     cp_async_wait<0>();
   } else if (warp == 6) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0 && nb > 0) {
+    // The whole warp runs the loop (waits and descriptors stay warp-uniform); one
+    // elected lane issues each MMA and commit.
+    if (nb > 0) {
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, kKeyBlock);
       constexpr uint32_t idesc_o = idesc_bf16_f32(128, kHeadDim) | (1u << 16);  // B (V) MN-major
+      // descriptor bases; the start-address field (bits 0..13, address >> 4) takes byte
+      // offsets >> 4 directly: every operand lies below 256 KB
+      const uint64_t kdesc0 = smem_desc_k_sw128(sbase + kSmemK0, 0);
+      const uint64_t pdesc0 = smem_desc_k_sw128(sbase + kSmemP0, 0);
+      const uint64_t vdesc0 = smem_desc_mn_sw128(sbase + kSmemV0, 64 * 128, 1024);
       auto issue_s = [&](int j) -> bool {  // S[j&1] = Q K(j)^T, Q from TMEM
         const int kbuf = j % kKBufs, sb = j & 1;
-        if (!mbar_wait(&k_full[kbuf], (j / kKBufs) & 1, err, kErrTimeoutMma)) return false;
-        if (j >= 2 && !mbar_wait(&s_empty[sb], ((j >> 1) - 1) & 1, err, kErrTimeoutMma)) return false;
+        if (!__all_sync(kFull, mbar_wait(&k_full[kbuf], (j / kKBufs) & 1, err, kErrTimeoutMma))) return false;
+        if (j >= 2 && !__all_sync(kFull, mbar_wait(&s_empty[sb], ((j >> 1) - 1) & 1, err, kErrTimeoutMma)))
+          return false;
         fence_proxy_async_smem();
         tc_fence_after();
-        const uint32_t kb = sbase + kSmemK0 + kbuf * kKVBytes;
+        const uint64_t kd = kdesc0 + (uint64_t)((kbuf * kKVBytes) >> 4);
         const uint32_t d = tmem + (uint32_t)(sb * kKeyBlock);
 #pragma unroll
         for (int s = 0; s < 4; ++s)
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            tc_mma_bf16_ts(d, tmem + kTmemQ + (uint32_t)(32 * s + 8 * kk),
-                           smem_desc_k_sw128(kb + s * (64 * 128), kk * 32), idesc_s, (s | kk) != 0);
-        tc_commit(&s_full[sb]);
-        tc_commit(&k_empty[kbuf]);
+            tc_mma_bf16_ts_w(d, tmem + kTmemQ + (uint32_t)(32 * s + 8 * kk),
+                             kd + (uint64_t)((s * kSubTile + kk * 32) >> 4), idesc_s, (s | kk) != 0);
+        tc_commit_w(&s_full[sb]);
+        tc_commit_w(&k_empty[kbuf]);
         return true;
       };
       auto issue_pv = [&](int j) -> bool {  // O += P(j) V(j)
         const int vbuf = j % kVBufs, pb = j % kPBufs;
-        if (!mbar_wait(&p_full[pb], (j / kPBufs) & 1, err, kErrTimeoutMma)) return false;
-        if (!mbar_wait(&v_full[vbuf], (j / kVBufs) & 1, err, kErrTimeoutMma)) return false;
+        if (!__all_sync(kFull, mbar_wait(&p_full[pb], (j / kPBufs) & 1, err, kErrTimeoutMma))) return false;
+        if (!__all_sync(kFull, mbar_wait(&v_full[vbuf], (j / kVBufs) & 1, err, kErrTimeoutMma))) return false;
         fence_proxy_async_smem();
         tc_fence_after();
-        const uint32_t vb = sbase + kSmemV0 + vbuf * kKVBytes, pbase = sbase + kSmemP0 + pb * kPBytes;
+        const uint64_t pd = pdesc0 + (uint64_t)((pb * kPBytes) >> 4);
+        const uint64_t vd = vdesc0 + (uint64_t)((vbuf * kKVBytes) >> 4);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          tc_mma_bf16(tmem + kTmemO, smem_desc_k_sw128(pbase, kk * 32),
-                      smem_desc_mn_sw128(vb + kk * 2048, 64 * 128, 1024), idesc_o, (j | kk) != 0);
-        tc_commit(&pv_done[vbuf]);  // V buffer and P buffer free, O updated
+          tc_mma_bf16_w(tmem + kTmemO, pd + (uint64_t)((kk * 32) >> 4), vd + (uint64_t)((kk * 2048) >> 4), idesc_o,
+                        (j | kk) != 0);
+        tc_commit_w(&pv_done[vbuf]);  // V buffer and P buffer free, O updated
         return true;
       };
-      ok = mbar_wait(q_full, 0, err, kErrTimeoutMma);
+      ok = __all_sync(kFull, mbar_wait(q_full, 0, err, kErrTimeoutMma));
       tc_fence_after();
       if (ok) ok = issue_s(0);
       for (int j = 0; j < nb && ok; ++j) {
@@ -260,7 +294,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (ok) ok = issue_pv(j);
       }
       // every MMA issued (also after a failed wait) has finished before TMEM is freed
-      tc_commit(mma_done);
+      tc_commit_w(mma_done);
       mbar_wait(mma_done, 0, err, kErrTimeoutMma);
     }
     __syncwarp();
@@ -303,26 +337,26 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = __all_sync(0xffffffffu, mbar_wait(&s_full[sb], (j >> 1) & 1, err, kErrTimeoutEpilogue));
       if (!ok) break;
       tc_fence_after();
-      float sv[64];
-      {
-        float t0[32], t1[32];
-        tmem_ld_32x32b_x32(tmem + t_lane + sb * kKeyBlock, t0);
-        tmem_ld_32x32b_x32(tmem + t_lane + sb * kKeyBlock + 32, t1);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          sv[i] = t0[i];
-          sv[32 + i] = t1[i];
-        }
-      }
+      float sv[64];  // raw logits q.k of this row and block
+      tmem_ld_32x32b_x64(tmem + t_lane + sb * kKeyBlock, sv);
       tc_fence_before();
       mbar_arrive(&s_empty[sb]);
       const int kbase = (blk0 + j) * kKeyBlock;
       const int vis_lo = blk0 + j < nbp ? 0 : sfx_lo, vis_hi = blk0 + j < nbp ? nv : sfx_hi;
-      float bm = -INFINITY;
+      if (kbase < vis_lo || kbase + kKeyBlock > vis_hi) {  // some slot of the block is hidden from this row
 #pragma unroll
-      for (int i = 0; i < 64; ++i) {
-        sv[i] = (unsigned)(kbase + i - vis_lo) < (unsigned)(vis_hi - vis_lo) ? sv[i] * scale_l2 : -INFINITY;
-        bm = fmaxf(bm, sv[i]);
+        for (int i = 0; i < 64; ++i)
+          if ((unsigned)(kbase + i - vis_lo) >= (unsigned)(vis_hi - vis_lo)) sv[i] = -INFINITY;
+      }
+      float bm;
+      {  // block max in log2 units (the scale is positive); eight independent chains
+        float mx[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) mx[k] = sv[k];
+#pragma unroll
+        for (int i = 8; i < 64; ++i) mx[i & 7] = fmaxf(mx[i & 7], sv[i]);
+        bm = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])), fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+        bm *= scale_l2;
       }
       // Raise m_used (and rescale l, O) when this block's max exceeds it by more than
       // 2^8.  O lives in TMEM and tcgen05.ld/st are warp-collective, so the whole warp
@@ -357,19 +391,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         // no visible key seen yet <=> m_used = -inf <=> every sv is -inf: use 0 so that 2^(-inf) = 0
         const float mu = m_used == -INFINITY ? 0.f : m_used;
         uint8_t *prow = smem + kSmemP0 + pb * kPBytes;
+        float ls[4] = {0.f, 0.f, 0.f, 0.f};  // partial row sums (independent chains)
 #pragma unroll
         for (int cc = 0; cc < 8; ++cc) {
           uint32_t pk[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const int i0 = cc * 8 + 2 * e;
-            const float p0 = ex2_approx(sv[i0] - mu), p1 = ex2_approx(sv[i0 + 1] - mu);
-            l += p0 + p1;
+            const float p0 = ex2_approx(fmaf(sv[i0], scale_l2, -mu)), p1 = ex2_approx(fmaf(sv[i0 + 1], scale_l2, -mu));
+            ls[e] += p0 + p1;
             const __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
             pk[e] = *reinterpret_cast<const uint32_t *>(&h2);
           }
           *reinterpret_cast<uint4 *>(prow + sw128_off(tid, cc)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
         }
+        l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
       }
       fence_proxy_async_smem();
       mbar_arrive(&p_full[pb]);
@@ -492,11 +528,19 @@ size_t attn_tc_partial_floats(const Geo &g, int step0, int splits) {
 
 bool attn_tc_maps(CallPtrs &cp, int layers, int B, int P, const void *ks, const void *vs, uint64_t sfx_rows) {
   for (int l = 0; l < layers && P > 0; ++l)
-    if (!make_map(&cp.kv_map[0][l], cp.prefix_k[l], (uint64_t)B * P, kHeadDim, kHeadDim, 8) ||
-        !make_map(&cp.kv_map[1][l], cp.prefix_v[l], (uint64_t)B * P, kHeadDim, kHeadDim, 8))
+    for (int kv = 0; kv < 2; ++kv) {
+      const void *base = kv ? cp.prefix_v[l] : cp.prefix_k[l];
+      if (!make_map(&cp.kv_map[kv][l], base, (uint64_t)B * P, kHeadDim, kHeadDim, 8) ||
+          !make_map(&cp.kv_map64[kv][l], base, (uint64_t)B * P, kHeadDim, kHeadDim, 64))
+        return false;
+    }
+  for (int kv = 0; kv < 2; ++kv) {
+    const void *base = kv ? vs : ks;
+    if (!make_map(&cp.sfx_map[kv], base, sfx_rows, kHeadDim, kHeadDim, 8) ||
+        !make_map(&cp.sfx_map64[kv], base, sfx_rows, kHeadDim, kHeadDim, 64))
       return false;
-  return make_map(&cp.sfx_map[0], ks, sfx_rows, kHeadDim, kHeadDim, 8) &&
-         make_map(&cp.sfx_map[1], vs, sfx_rows, kHeadDim, kHeadDim, 8);
+  }
+  return true;
 }
 
 void launch_attention_tc(const bf16 *q, const bf16 *ks, const bf16 *vs, const CallPtrs *cp, int layer,

@@ -79,11 +79,54 @@ __device__ __forceinline__ float consumer_rstd(const EpiArgs &e, int r) {
   return 1.f;
 }
 
-// Epilogue of 32 consecutive output columns [n, n+32) of GEMM row r (`rs` from
-// consumer_rstd).  Returns the row's sum of squares over these columns for the
-// fused-norm producers, else 0.
+// Global operands of the epilogue of one 32-column chunk, loaded ahead of the chunk
+// (the residual row slice, bias, RoPE (cos, sin) pairs; norm gain in g).
+struct EpiIn {
+  float4 a[8];
+  float4 g[8];
+};
+
 template <int EPI>
-__device__ __forceinline__ float epilogue32(const EpiArgs &e, int r, int n, float (&v)[32], float rs) {
+__device__ __forceinline__ void epi_fetch(const EpiArgs &e, int r, int n, EpiIn &in) {
+  const int orow = e.out_row0 + r;
+  if constexpr (EPI == EPI_RESID_F32) {
+    const float4 *src = reinterpret_cast<const float4 *>(e.out_f32 + (size_t)orow * e.ldo + n);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) in.a[i] = src[i];
+  } else if constexpr (EPI == EPI_BIAS_F32 || EPI == EPI_VEC_SILU) {
+    const float4 *src = reinterpret_cast<const float4 *>(e.vec + n);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) in.a[i] = src[i];
+  } else if constexpr (EPI == EPI_QKV_ROPE) {
+    int b, j;
+    row_to_bj_tc(orow, e.B, e.H, b, j);
+    const int pos = e.nvalid[b] + j;
+#pragma unroll
+    for (int gi = 0; gi < 2; ++gi) {
+      const int gc = (n >> 4) + gi;
+      const int hd = gc >> 4, ib = (gc & 15) * 8;
+      if (hd < kHeads + 1) {
+        // (cos, sin) of fp32(pos) * inv_freq[i], tabulated per call (k_rope_table)
+        const float4 *tab = reinterpret_cast<const float4 *>(e.rope_tab + ((size_t)pos * (kHeadDim / 2) + ib) * 2);
+#pragma unroll
+        for (int w2 = 0; w2 < 4; ++w2) in.a[4 * gi + w2] = tab[w2];
+      }
+    }
+  }
+  if constexpr (EPI == EPI_RESID_F32 || EPI == EPI_BIAS_F32) {
+    if (e.gain) {
+      const float4 *gs = reinterpret_cast<const float4 *>(e.gain + n);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) in.g[i] = gs[i];
+    }
+  }
+}
+
+// Epilogue of 32 consecutive output columns [n, n+32) of GEMM row r (`rs` from
+// consumer_rstd, `in` from epi_fetch).  Returns the row's sum of squares over these
+// columns for the fused-norm producers, else 0.
+template <int EPI>
+__device__ __forceinline__ float epilogue32(const EpiArgs &e, int r, int n, float (&v)[32], float rs, const EpiIn &in) {
   const int orow = e.out_row0 + r;
   float ssq = 0.f;
   if constexpr (EPI == EPI_STORE_F32 || EPI == EPI_BIAS_F32 || EPI == EPI_RESID_F32) {
@@ -91,12 +134,9 @@ __device__ __forceinline__ float epilogue32(const EpiArgs &e, int r, int n, floa
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       float4 w = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
-      if constexpr (EPI == EPI_BIAS_F32) {
-        const float4 bb = reinterpret_cast<const float4 *>(e.vec + n)[i];
+      if constexpr (EPI == EPI_BIAS_F32 || EPI == EPI_RESID_F32) {
+        const float4 bb = in.a[i];  // bias, or the residual h
         w.x += bb.x; w.y += bb.y; w.z += bb.z; w.w += bb.w;
-      } else if constexpr (EPI == EPI_RESID_F32) {
-        const float4 old = dst[i];
-        w.x += old.x; w.y += old.y; w.z += old.z; w.w += old.w;
       }
       dst[i] = w;
       v[4 * i] = w.x; v[4 * i + 1] = w.y; v[4 * i + 2] = w.z; v[4 * i + 3] = w.w;
@@ -105,9 +145,16 @@ __device__ __forceinline__ float epilogue32(const EpiArgs &e, int r, int n, floa
       if (e.gain) {  // fused RMSNorm producer: bf16(h * (1 + g)) and sum of h^2
         float t[32];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          ssq = fmaf(v[i], v[i], ssq);
-          t[i] = v[i] * (1.0f + e.gain[n + i]);
+        for (int i = 0; i < 8; ++i) {
+          const float4 gg = in.g[i];
+          ssq = fmaf(v[4 * i], v[4 * i], ssq);
+          ssq = fmaf(v[4 * i + 1], v[4 * i + 1], ssq);
+          ssq = fmaf(v[4 * i + 2], v[4 * i + 2], ssq);
+          ssq = fmaf(v[4 * i + 3], v[4 * i + 3], ssq);
+          t[4 * i] = v[4 * i] * (1.0f + gg.x);
+          t[4 * i + 1] = v[4 * i + 1] * (1.0f + gg.y);
+          t[4 * i + 2] = v[4 * i + 2] * (1.0f + gg.z);
+          t[4 * i + 3] = v[4 * i + 3] * (1.0f + gg.w);
         }
         uint4 *xd = reinterpret_cast<uint4 *>(e.xn_out + (size_t)orow * kWidth + n);
 #pragma unroll
@@ -117,14 +164,17 @@ __device__ __forceinline__ float epilogue32(const EpiArgs &e, int r, int n, floa
   } else if constexpr (EPI == EPI_VEC_SILU) {
     float t[32];
 #pragma unroll
-    for (int i = 0; i < 32; ++i) t[i] = silu_f(v[i] + e.vec[n + i]);
+    for (int i = 0; i < 8; ++i) {
+      const float4 bb = in.a[i];
+      t[4 * i] = silu_f(v[4 * i] + bb.x);
+      t[4 * i + 1] = silu_f(v[4 * i + 1] + bb.y);
+      t[4 * i + 2] = silu_f(v[4 * i + 2] + bb.z);
+      t[4 * i + 3] = silu_f(v[4 * i + 3] + bb.w);
+    }
     uint4 *dst = reinterpret_cast<uint4 *>(e.out_bf16 + (size_t)orow * e.ldo + n);
 #pragma unroll
     for (int i = 0; i < 4; ++i) dst[i] = pack8_bf16(t + 8 * i);
   } else if constexpr (EPI == EPI_QKV_ROPE) {
-    int b, j;
-    row_to_bj_tc(orow, e.B, e.H, b, j);
-    const int pos = e.nvalid[b] + j;
 #pragma unroll
     for (int i = 0; i < 32; ++i) v[i] *= rs;
 #pragma unroll
@@ -138,12 +188,9 @@ __device__ __forceinline__ float epilogue32(const EpiArgs &e, int r, int n, floa
         hi[w] = v[16 * gi + 8 + w];
       }
       if (hd < kHeads + 1) {
-        // (cos, sin) of fp32(pos) * inv_freq[i], tabulated per call (k_rope_table)
-        const float4 *tab =
-            reinterpret_cast<const float4 *>(e.rope_tab + ((size_t)pos * (kHeadDim / 2) + ib) * 2);
 #pragma unroll
         for (int w2 = 0; w2 < 4; ++w2) {
-          const float4 t = tab[w2];  // (cos, sin) of pairs ib+2*w2, ib+2*w2+1
+          const float4 t = in.a[4 * gi + w2];  // (cos, sin) of pairs ib+2*w2, ib+2*w2+1
 #pragma unroll
           for (int h2 = 0; h2 < 2; ++h2) {
             const int w = 2 * w2 + h2;
@@ -286,11 +333,14 @@ __global__ void __launch_bounds__(128, 1)
     if (splits == 1) {
       float ssq = 0.f;
       const float rs = r < M ? consumer_rstd<EPI>(e, r) : 1.f;
-#pragma unroll 1
+      EpiIn in[2];
+      if (r < M) epi_fetch<EPI>(e, r, n0, in[0]);
+#pragma unroll
       for (int c = 0; c < BN; c += 32) {
+        if (c + 32 < BN && r < M) epi_fetch<EPI>(e, r, n0 + c + 32, in[((c >> 5) + 1) & 1]);
         float v[32];
         tmem_ld_32x32b_x32(tmem + t_lane + (uint32_t)c, v);
-        if (r < M) ssq += epilogue32<EPI>(e, r, n0 + c, v, rs);
+        if (r < M) ssq += epilogue32<EPI>(e, r, n0 + c, v, rs, in[(c >> 5) & 1]);
       }
       if (r < M) norm_partial_store<EPI>(e, r, n0, BN, gridDim.y * BN, ssq);
     } else {
@@ -332,7 +382,9 @@ __global__ void __launch_bounds__(128, 1)
                 v[4 * i] += t.x; v[4 * i + 1] += t.y; v[4 * i + 2] += t.z; v[4 * i + 3] += t.w;
               }
             }
-            ssq += epilogue32<EPI>(e, r, n0 + c, v, rs);
+            EpiIn in;
+            epi_fetch<EPI>(e, r, n0 + c, in);
+            ssq += epilogue32<EPI>(e, r, n0 + c, v, rs, in);
           }
           norm_partial_store<EPI>(e, r, n0, BN, gridDim.y * BN, ssq);
         }
@@ -467,19 +519,23 @@ __global__ void __launch_bounds__(192, 1)
     for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++ti) {
       const int a = ti % kAcc;
       const uint32_t around = ti / kAcc;
+      const int m0 = (t % mt) * 128, n0 = (t / mt) * BN;
+      const int r = m0 + q * 32 + lane;
+      // operands of the first chunk and the row's norm scale load while the MMAs run
+      const float rs = r < M ? consumer_rstd<EPI>(e, r) : 1.f;
+      EpiIn in[2];
+      if (r < M) epi_fetch<EPI>(e, r, n0, in[0]);
       const bool ok = mbar_wait(&acc_full[a], around & 1u, err, kErrTimeoutEpilogue);
       __syncwarp();
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
-      const int m0 = (t % mt) * 128, n0 = (t / mt) * BN;
-      const int r = m0 + q * 32 + lane;
       float ssq = 0.f;
-      const float rs = r < M ? consumer_rstd<EPI>(e, r) : 1.f;
-#pragma unroll 1
+#pragma unroll
       for (int c = 0; c < BN; c += 32) {
+        if (c + 32 < BN && r < M) epi_fetch<EPI>(e, r, n0 + c + 32, in[((c >> 5) + 1) & 1]);
         float v[32];
         tmem_ld_32x32b_x32(tmem + (uint32_t)(a * C::kTmemCols) + t_lane + (uint32_t)c, v);
-        if (r < M) ssq += epilogue32<EPI>(e, r, n0 + c, v, rs);
+        if (r < M) ssq += epilogue32<EPI>(e, r, n0 + c, v, rs, in[(c >> 5) & 1]);
       }
       if (r < M) norm_partial_store<EPI>(e, r, n0, BN, N, ssq);
       tc_fence_before();

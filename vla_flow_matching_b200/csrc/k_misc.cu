@@ -129,9 +129,10 @@ void launch_state_embed(const CallPtrs *cp, const TW *w, const float *b, int B, 
 }
 
 // Action tokens: out[i] = action_in_proj(x[i]) for every (sample, horizon) row.
-// Block (rows r0..r0+15, features 256*blockIdx.y..+255): each thread keeps the
-// weight row of its output feature in registers and reuses it for the 16 rows.
-constexpr int kActRows = 16;
+// Block (rows r0..r0+kActRows-1, features 256*blockIdx.y..+255): each thread keeps
+// the weight row of its output feature in registers (16-byte loads when the row
+// allows) and reuses it for the block's rows.
+constexpr int kActRows = 32;
 template <typename TW, typename T>
 __global__ void __launch_bounds__(256) k_action_in(const float *x, const TW *w, const float *bias, int rows, int A,
                                                     T *out) {
@@ -146,8 +147,21 @@ __global__ void __launch_bounds__(256) k_action_in(const float *x, const TW *w, 
   __syncthreads();
   const int n = blockIdx.y * 256 + threadIdx.x;
   float wr[64];
+  constexpr int kVec = 16 / sizeof(TW);  // elements per 16-byte load
+  if (A % kVec == 0) {
+    const uint4 *src = reinterpret_cast<const uint4 *>(w + (size_t)n * A);
 #pragma unroll
-  for (int i = 0; i < 64; ++i) wr[i] = i < A ? to_f32(w[(size_t)n * A + i]) : 0.f;
+    for (int q = 0; q < 64 / kVec; ++q) {
+      uint4 u = make_uint4(0, 0, 0, 0);
+      if (q * kVec < A) u = src[q];
+      const TW *e = reinterpret_cast<const TW *>(&u);
+#pragma unroll
+      for (int k = 0; k < kVec; ++k) wr[q * kVec + k] = q * kVec + k < A ? to_f32(e[k]) : 0.f;
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 64; ++i) wr[i] = i < A ? to_f32(w[(size_t)n * A + i]) : 0.f;
+  }
   const float bn = bias[n];
   for (int r = 0; r < kActRows && r0 + r < rows; ++r) {
     float acc = 0.f;
@@ -290,38 +304,54 @@ void launch_geglu(const float *raw, int row0, int rows, T *act, cudaStream_t s) 
 // Final RMSNorm of an action token, v = action_out_proj(.) in fp32, then the
 // Euler update x <- x + dt*v (`denoise_step` tail and `sample_actions`); the last
 // step also writes x_0.
+// Final norm, action_out_proj and the Euler update x <- x + dt * v (`denoise_step` /
+// `sample_actions` on the vllm-omni pi0 page) for kEulerRows action rows per block,
+// so each block reads the out-projection weights once for all of them (one row per
+// block when rows are few, for parallelism).  Per row the arithmetic and its order
+// do not depend on kEulerRows.
+template <int kEulerRows>
 __global__ void __launch_bounds__(256) k_final_euler(const float *h, Geo g, const float *gain, const float *w_out,
                                                       const float *b_out, float dt, float *x, const CallPtrs *cp,
                                                       int last) {
   pdl_wait();
   pdl_trigger();
-  __shared__ float y[kWidth];
-  __shared__ float red[8];
-  const int i = blockIdx.x;  // action row index b*H + (j-1)
-  const float *src = h + (size_t)(g.B + i) * kWidth;
-  float ss = 0.f;
-  for (int c = threadIdx.x; c < kWidth; c += blockDim.x) {
-    const float v = src[c];
-    y[c] = v;
-    ss += v * v;
-  }
+  __shared__ float y[kEulerRows][kWidth];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  ss = warp_sum(ss);
-  if (lane == 0) red[warp] = ss;
+  const int rows = g.B * g.H;
+  const int i0 = blockIdx.x * kEulerRows;  // action row index b*H + (j-1)
+  // normalised rows: warp w takes row i0 + w
+  if (warp < kEulerRows && i0 + warp < rows) {
+    const float *src = h + (size_t)(g.B + i0 + warp) * kWidth;
+    float ss = 0.f;
+    for (int c = lane; c < kWidth; c += 32) {
+      const float v = src[c];
+      y[warp][c] = v;
+      ss += v * v;
+    }
+    ss = warp_sum(ss);
+    const float inv = 1.0f / sqrtf(ss / (float)kWidth + kRmsEps);
+    for (int c = lane; c < kWidth; c += 32) y[warp][c] = (y[warp][c] * inv) * (1.0f + gain[c]);
+  }
   __syncthreads();
-  float tot = 0.f;
-  for (int w = 0; w < 8; ++w) tot += red[w];
-  const float inv = 1.0f / sqrtf(tot / (float)kWidth + kRmsEps);
-  for (int c = threadIdx.x; c < kWidth; c += blockDim.x) y[c] = (y[c] * inv) * (1.0f + gain[c]);
-  __syncthreads();
+  const int nr = min(kEulerRows, rows - i0);
   for (int a = warp; a < g.A; a += 8) {
     const float *wr = w_out + (size_t)a * kWidth;
-    float acc = 0.f;
-    for (int c = lane; c < kWidth; c += 32) acc = fmaf(wr[c], y[c], acc);
-    acc = warp_sum(acc);
-    if (lane == 0) {
-      const float v = acc + b_out[a];
-      const size_t xi = (size_t)i * g.A + a;
+    float acc[kEulerRows];
+#pragma unroll
+    for (int r = 0; r < kEulerRows; ++r) acc[r] = 0.f;
+    for (int c = lane; c < kWidth; c += 32) {
+      const float wv = wr[c];
+#pragma unroll
+      for (int r = 0; r < kEulerRows; ++r) acc[r] = fmaf(wv, y[r][c], acc[r]);
+    }
+#pragma unroll
+    for (int r = 0; r < kEulerRows; ++r) acc[r] = warp_sum(acc[r]);
+    if (lane < nr) {
+      float mine = acc[0];
+#pragma unroll
+      for (int r = 1; r < kEulerRows; ++r) mine = lane == r ? acc[r] : mine;
+      const float v = mine + b_out[a];
+      const size_t xi = (size_t)(i0 + lane) * g.A + a;
       const float xn = __fadd_rn(x[xi], __fmul_rn(dt, v));
       x[xi] = xn;
       if (last) cp->x0[xi] = xn;
@@ -331,7 +361,11 @@ __global__ void __launch_bounds__(256) k_final_euler(const float *h, Geo g, cons
 
 void launch_final_euler(const float *h, const Geo &g, const float *gain, const float *w_out, const float *b_out,
                         float dt, float *x, const CallPtrs *cp, int last, cudaStream_t s) {
-  launch_pdl(k_final_euler, g.B * g.H, 256, 0, s, h, g, gain, w_out, b_out, dt, x, cp, last);
+  const int rows = g.B * g.H;
+  if (rows >= 8 * 148)
+    launch_pdl(k_final_euler<8>, (rows + 7) / 8, 256, 0, s, h, g, gain, w_out, b_out, dt, x, cp, last);
+  else
+    launch_pdl(k_final_euler<1>, rows, 256, 0, s, h, g, gain, w_out, b_out, dt, x, cp, last);
 }
 
 __global__ void k_copy_x1(const CallPtrs *cp, int n, float *x) {

@@ -24,9 +24,11 @@ struct CallPtrs {
   // bf16 mode: TMA maps of the attention keys and values, [0] = K, [1] = V.
   // kv_map[.][l]: layer l's prefix tensor as B*P rows of 256 (encoded per call);
   // sfx_map[.]: the suffix K/V of all layers as one tensor of rows x 256.
-  // Boxes are 64 columns x 8 rows with the 128-byte swizzle.
+  // 128-byte swizzle; boxes of 64 columns x 8 rows, or x 64 rows for the *64 maps.
   CUtensorMap kv_map[2][kMaxDepth];
+  CUtensorMap kv_map64[2][kMaxDepth];
   CUtensorMap sfx_map[2];
+  CUtensorMap sfx_map64[2];
   const bf16 *prefix_k[kMaxDepth];
   const bf16 *prefix_v[kMaxDepth];
   const uint8_t *mask;
