@@ -514,7 +514,7 @@ int attn_tc_splits(const Geo &g, int step0) {
   const int ctas = mtiles * g.B;
   if (ctas >= 96) return 1;
   int splits = (148 + ctas - 1) / ctas;
-  const int max_split = (nblk + 1) / 2;  // at least two key blocks per split
+  const int max_split = (nblk + 3) / 4;  // at least four key blocks per split
   if (splits > max_split) splits = max_split;
   return splits < 1 ? 1 : splits;
 }
