@@ -9,6 +9,9 @@ and this module imports nothing from the product path.
 Source: the vllm-omni page "vllm_omni/diffusion/models/pi0/modeling_pi0.py"
 (an inference-only pi0 "math kernel"), cited below by function name, and the
 VersatIL ``GenerativeVLM`` page for the rotate-half RoPE and residual+FFN order.
+The solver and convention variants (time grid 0 -> 1, x-prediction, causal
+action mask) follow the Wall-X flow-matching page (its ODE integration of the
+sampler, ``use_x_pred`` and ``causal_action_attention_mask``).
 
 Precision follows that page: the expert runs in float32 (its Gemma config is
 built with ``dtype="float32"``), the timestep embedding is formed in float64 and
@@ -126,19 +129,26 @@ def linear(x, w, b=None):
 
 
 # --- masks and positions -----------------------------------------------------
-def suffix_visibility(prefix_valid: np.ndarray, horizon: int) -> np.ndarray:
+def suffix_visibility(prefix_valid: np.ndarray, horizon: int, causal_actions: bool = False) -> np.ndarray:
     """Boolean (B, T, P+T) mask of which key each suffix query may attend to.
 
     From ``denoise_step``/``embed_suffix``/``make_att_2d_masks``: prefix keys are
     visible to every suffix query iff valid; inside the suffix the AR flags are
     [1, 1, 0, ..., 0] and key j is visible to query i iff cumsum[j] <= cumsum[i]
     (all suffix tokens are non-padding).
+
+    ``causal_actions`` (the Wall-X ``causal_action_attention_mask``): the
+    suffix-to-suffix block is lower triangular, key j visible to query i iff
+    j <= i, so action token i sees the state and actions 0..i.
     """
     B, P = prefix_valid.shape
     T = horizon + 1
-    ar = np.array([1, 1] + [0] * (horizon - 1), dtype=np.int64)
-    cum = np.cumsum(ar)
-    suf = cum[None, :] <= cum[:, None]                      # [query, key]
+    if causal_actions:
+        suf = np.tril(np.ones((T, T), dtype=bool))          # [query, key]
+    else:
+        ar = np.array([1, 1] + [0] * (horizon - 1), dtype=np.int64)
+        cum = np.cumsum(ar)
+        suf = cum[None, :] <= cum[:, None]                  # [query, key]
     pre = np.broadcast_to(prefix_valid.astype(bool)[:, None, :], (B, T, P))
     return np.concatenate([pre, np.broadcast_to(suf, (B, T, T))], axis=2)
 
@@ -214,13 +224,13 @@ def embed_suffix(w, state, x_t, t, dtype):
     return np.concatenate([s_tok, act_tok], axis=1)
 
 
-def denoise_step(w, prefix_k, prefix_v, prefix_valid, state, x_t, t, dims, dtype):
+def denoise_step(w, prefix_k, prefix_v, prefix_valid, state, x_t, t, dims, dtype, causal_actions=False):
     """v_t for one Euler step (``denoise_step``): suffix through all expert layers,
     final RMSNorm, keep the last ``horizon`` tokens, action_out_proj."""
     n_heads, head_dim = dims
     H = x_t.shape[1]
     h = embed_suffix(w, state, x_t, t, dtype)
-    visible = suffix_visibility(prefix_valid, H)
+    visible = suffix_visibility(prefix_valid, H, causal_actions)
     pos = suffix_positions(prefix_valid, H)
     for layer, lw in enumerate(w["layers"]):
         h = expert_layer(h, lw, prefix_k[layer], prefix_v[layer], visible, pos,
@@ -236,15 +246,52 @@ def convert_weights(weights: dict, dtype) -> dict:
     return out
 
 
+def time_grid(num_steps: int, convention: str = "pi0"):
+    """Step times t_k (k < N, float32) and step sizes dt_k (float32).
+
+    "pi0" (``sample_actions``): t runs from 1 (noise) to 0, dt = -1/N taken as
+    float32, t_k = float32(1 + k*(-1/N)) with the product formed in float64.
+    "linspace" (the Wall-X sampler: ``torch.linspace(0, 1, N + 1)`` integrated
+    with a fixed-grid Euler step): t_k = float32(k/N), correctly rounded, and
+    dt_k = t_{k+1} - t_k in float32, so the noise sits at t = 0 and the action at t = 1.
+    """
+    if num_steps <= 0:
+        raise ValueError("num_steps must be positive")
+    if convention == "pi0":
+        dt_exact = -1.0 / num_steps
+        t = [np.float32(1.0 + k * dt_exact) for k in range(num_steps)]
+        dt = [np.float32(dt_exact)] * num_steps
+    elif convention == "linspace":
+        pts = [np.float32(k / num_steps) for k in range(num_steps + 1)]
+        t = pts[:-1]
+        dt = [np.float32(pts[k + 1] - pts[k]) for k in range(num_steps)]
+    else:
+        raise ValueError(f"unknown time grid {convention!r}")
+    return t, dt
+
+
+def output_to_velocity(out: np.ndarray, noise: np.ndarray, x_prediction: bool) -> np.ndarray:
+    """The network output read as the velocity (pi0), or as the clean action
+    x_hat with velocity x_hat - noise (the Wall-X ``use_x_pred`` branch)."""
+    return out - noise if x_prediction else out
+
+
 def sample_actions(weights: dict, prefix_k: Sequence[np.ndarray],
                    prefix_v: Sequence[np.ndarray], prefix_valid: np.ndarray,
                    state: np.ndarray, x1: np.ndarray, num_steps: int,
-                   num_heads: int = 8, dtype=np.float32) -> np.ndarray:
+                   num_heads: int = 8, dtype=np.float32, time_convention: str = "pi0",
+                   x_prediction: bool = False, causal_actions: bool = False) -> np.ndarray:
     """Euler integration from t = 1 (noise x_1) to t = 0 (``sample_actions``).
 
     dt = -1/num_steps; at step k the time is t = 1 + k*dt (stored as float32),
     v_t comes from :func:`denoise_step` and x <- x + dt*v_t (dt taken in the
     model dtype).  Returns x_0 with the shape of ``x1``.
+
+    Variants (the Wall-X page): ``time_convention="linspace"`` integrates from
+    t = 0 (noise) to 1 on the grid of :func:`time_grid`; ``x_prediction``
+    reads the network output as the clean action x_hat and uses the velocity
+    x_hat - x_1 (``use_x_pred``: prediction minus the noise); ``causal_actions``
+    makes the suffix attention lower triangular (:func:`suffix_visibility`).
 
     ``prefix_k``/``prefix_v``: per layer (B, 1, P, head_dim), already rotated,
     bf16 bits or floats.  ``prefix_valid``: (B, P), nonzero = valid key.
@@ -257,11 +304,12 @@ def sample_actions(weights: dict, prefix_k: Sequence[np.ndarray],
     head_dim = prefix_k[0].shape[-1]
     kp = [as_float(k, dtype)[:, 0] for k in prefix_k]
     vp = [as_float(v, dtype)[:, 0] for v in prefix_v]
-    dt_exact = -1.0 / num_steps
-    dt = dtype(dt_exact)
-    x = np.asarray(x1).astype(dtype)
+    ts, dts = time_grid(num_steps, time_convention)
+    noise = np.asarray(x1).astype(dtype)
+    x = noise.copy()
     for step in range(num_steps):
-        t = np.float32(1.0 + step * dt_exact)
-        v = denoise_step(w, kp, vp, prefix_valid, state, x, t, (num_heads, head_dim), dtype)
-        x = x + dt * v.astype(dtype)
+        v = denoise_step(w, kp, vp, prefix_valid, state, x, ts[step], (num_heads, head_dim), dtype,
+                         causal_actions).astype(dtype)
+        v = output_to_velocity(v, noise, x_prediction)
+        x = x + dtype(dts[step]) * v
     return x

@@ -66,22 +66,37 @@ def _temb(t, dim):
     return sins + coss
 
 
-def brute_sample(weights, prefix_k, prefix_v, mask, state, x1, num_steps, num_heads):
-    """weights: float arrays (nn.Linear layout); prefix_k/v: per layer (B,1,P,D) floats."""
+def brute_sample(weights, prefix_k, prefix_v, mask, state, x1, num_steps, num_heads, time_convention="pi0",
+                 x_prediction=False, causal_actions=False):
+    """weights: float arrays (nn.Linear layout); prefix_k/v: per layer (B,1,P,D) floats.
+
+    Variants (the Wall-X page): time_convention "linspace" steps t from 0 to 1 on
+    float32(k/N) with float32 differences as step sizes; x_prediction takes the
+    output as the clean action and moves along output - initial noise;
+    causal_actions lets suffix query i see suffix keys 0..i only."""
     W = _mat(weights["state_proj_w"])
     depth = len(weights["layers"])
     B = len(x1)
     H = len(x1[0])
     D = len(prefix_k[0][0][0][0])
     width = len(W)
+    np = __import__("numpy")
     dt = -1.0 / num_steps
+    if time_convention == "linspace":
+        grid = [float(np.float32(k / num_steps)) for k in range(num_steps + 1)]
     x = [[_vec(row) for row in x1[b]] for b in range(B)]
+    noise = [[_vec(row) for row in x1[b]] for b in range(B)]
     layers = [{k: (_mat(v) if getattr(v, "ndim", 1) == 2 else _vec(v)) for k, v in lw.items()}
               for lw in weights["layers"]]
     g = {k: (_mat(v) if getattr(v, "ndim", 1) == 2 else _vec(v))
          for k, v in weights.items() if k != "layers"}
     for step in range(num_steps):
-        t = float(__import__("numpy").float32(1.0 + step * dt))
+        if time_convention == "linspace":
+            t = grid[step]
+            h_step = float(np.float32(np.float32(grid[step + 1]) - np.float32(grid[step])))
+        else:
+            t = float(np.float32(1.0 + step * dt))
+            h_step = dt
         te = _temb(t, width)
         for b in range(B):
             n_valid = 0
@@ -108,7 +123,10 @@ def brute_sample(weights, prefix_k, prefix_v, mask, state, x1, num_steps, num_he
                 for i in range(T):
                     # keys this query may see: valid prefix, then the suffix block rule
                     keys = [(_vec(kp[p]), _vec(vp[p])) for p in valid_idx]
-                    suffix_keys = [0] if i == 0 else list(range(T))
+                    if causal_actions:
+                        suffix_keys = list(range(i + 1))
+                    else:
+                        suffix_keys = [0] if i == 0 else list(range(T))
                     keys += [(ks[j], vs[j]) for j in suffix_keys]
                     o = []
                     for hd in range(num_heads):
@@ -129,5 +147,7 @@ def brute_sample(weights, prefix_k, prefix_v, mask, state, x1, num_steps, num_he
             for j in range(H):
                 y = _rmsnorm(toks[1 + j], g["final_norm_w"])
                 vel = _matvec(g["action_out_w"], y, g["action_out_b"])
-                x[b][j] = [x[b][j][a] + dt * vel[a] for a in range(len(vel))]
+                if x_prediction:
+                    vel = [vel[a] - noise[b][j][a] for a in range(len(vel))]
+                x[b][j] = [x[b][j][a] + h_step * vel[a] for a in range(len(vel))]
     return x

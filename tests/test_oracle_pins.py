@@ -48,11 +48,11 @@ def full_width_small(depth=2, B=1, P=64, masked=10, horizon=50):
     return synth.make_inputs(wl)
 
 
-def run_oracle(inp, dtype=np.float32, weights=None, pk=None, pv=None):
+def run_oracle(inp, dtype=np.float32, weights=None, pk=None, pv=None, **variant):
     return O.sample_actions(weights if weights is not None else inp.weights,
                             pk if pk is not None else inp.prefix_k,
                             pv if pv is not None else inp.prefix_v,
-                            inp.mask, inp.state, inp.x1, inp.workload.num_steps, dtype=dtype)
+                            inp.mask, inp.state, inp.x1, inp.workload.num_steps, dtype=dtype, **variant)
 
 
 # --- timestep embedding ----------------------------------------------------------
@@ -294,6 +294,79 @@ def test_brute_force_sees_the_mask_hole():
     assert np.array_equal(a, b)
 
 
+# --- solver / convention variants (the Wall-X page) -------------------------------------
+VARIANTS = [dict(time_convention="linspace"), dict(x_prediction=True), dict(causal_actions=True),
+            dict(time_convention="linspace", x_prediction=True, causal_actions=True)]
+
+
+@pytest.mark.parametrize("variant", VARIANTS, ids=lambda v: "+".join(f"{k}={x}" for k, x in v.items()))
+def test_brute_force_float64_matches_variants(variant):
+    dims = synth.TINY_BRUTE_DIMS
+    w, pk, pv, mask, state, x1, steps = tiny_float_inputs(dims)
+    ref = np.array(brute_sample(w, pk, pv, mask, state, x1, steps, dims.num_heads, **variant))
+    ours = O.sample_actions(w, pk, pv, mask, state, x1, steps, num_heads=dims.num_heads, dtype=np.float64,
+                            **variant)
+    assert np.max(np.abs(ours - ref)) < 1e-11
+
+
+@pytest.mark.parametrize("steps", [1, 3, 10])
+def test_linspace_grid_runs_zero_to_one(steps):
+    """t_0 = 0, each t_k within fp32 rounding of k/N, and the float32 step sizes
+    are exact differences, so they add up to exactly +1 (the pi0 grid: -1)."""
+    ts, dts = O.time_grid(steps, "linspace")
+    assert ts[0] == 0.0 and len(ts) == len(dts) == steps
+    for k, t in enumerate(ts):
+        assert abs(float(t) - k / steps) <= 2.0 ** -24 * (k / steps)  # unit roundoff of fp32
+    assert math.fsum(float(d) for d in dts) == 1.0
+    ts_pi0, dts_pi0 = O.time_grid(steps, "pi0")
+    assert ts_pi0[0] == 1.0 and abs(math.fsum(float(d) for d in dts_pi0) + 1.0) < steps * 1e-7
+
+
+@pytest.mark.parametrize("steps", [1, 3, 10])
+def test_linspace_bias_only_outproj_moves_by_plus_b(steps):
+    inp = full_width_small()
+    inp = dataclasses.replace(inp, workload=dataclasses.replace(inp.workload, num_steps=steps))
+    w = dict(inp.weights)
+    b = np.random.default_rng(8).normal(0, 1, 32).astype(np.float32)
+    w["action_out_w"] = np.zeros((32, 1024), np.float32)
+    w["action_out_b"] = b
+    x0 = run_oracle(inp, weights=w, time_convention="linspace")
+    tol = steps * 1.2e-7 * (np.abs(inp.x1) + np.abs(b))
+    assert np.all(np.abs(x0 - (inp.x1 + b[None, None, :])) <= tol + 1e-30)
+
+
+@pytest.mark.parametrize("grid,expect", [("linspace", "b"), ("pi0", "2x1-b")])
+def test_x_prediction_with_a_constant_prediction(grid, expect):
+    """x_hat == b at every step: the velocity is b - x_1, so on the 0 -> 1 grid the
+    chunk lands on b and on the 1 -> 0 grid on x_1 - (b - x_1)."""
+    inp = full_width_small()
+    w = dict(inp.weights)
+    b = np.random.default_rng(12).normal(0, 1, 32).astype(np.float32)
+    w["action_out_w"] = np.zeros((32, 1024), np.float32)
+    w["action_out_b"] = b
+    x0 = run_oracle(inp, weights=w, time_convention=grid, x_prediction=True)
+    want = b[None, None, :] + 0 * inp.x1 if expect == "b" else 2 * inp.x1 - b[None, None, :]
+    steps = inp.workload.num_steps
+    assert np.all(np.abs(x0 - want) <= steps * 2.5e-7 * (np.abs(inp.x1) + np.abs(b)) + 1e-30)
+
+
+def test_causal_mask_first_action_ignores_later_actions():
+    """Under the causal action mask action 0 sees the prefix, the state and itself
+    only, so its whole trajectory is independent of the other actions' noise; with
+    the pi0 mask it is not."""
+    inp = full_width_small(horizon=6)
+    x1b = inp.x1.copy()
+    x1b[:, 1:] = np.random.default_rng(13).normal(0, 1, x1b[:, 1:].shape).astype(np.float32)
+    inp_b = dataclasses.replace(inp, x1=x1b)
+    a = run_oracle(inp, np.float64, causal_actions=True)
+    b = run_oracle(inp_b, np.float64, causal_actions=True)
+    assert np.max(np.abs(a[:, 0] - b[:, 0])) < 1e-12
+    assert np.max(np.abs(a[:, 1:] - b[:, 1:])) > 1e-3
+    a2 = run_oracle(inp, np.float64)
+    b2 = run_oracle(inp_b, np.float64)
+    assert np.max(np.abs(a2[:, 0] - b2[:, 0])) > 1e-6
+
+
 # --- planted mistakes: each must make a pin fail --------------------------------------
 def _mutations():
     def rope_sign(x, pos, dtype=np.float32):
@@ -308,32 +381,52 @@ def _mutations():
         h = dim // 2
         return np.concatenate([e[:, h:], e[:, :h]], axis=1)
 
-    def vis_state_sees_all(prefix_valid, horizon):
-        v = O.__dict__["_orig_suffix_visibility"](prefix_valid, horizon).copy()
+    def vis_state_sees_all(prefix_valid, horizon, causal_actions=False):
+        v = O.__dict__["_orig_suffix_visibility"](prefix_valid, horizon, causal_actions).copy()
         v[:, 0, :] = v[:, 1, :]
         return v
 
     def pos_off_by_one(prefix_valid, horizon):
         return O.__dict__["_orig_suffix_positions"](prefix_valid, horizon) + 1
 
+    def vis_causal_ignored(prefix_valid, horizon, causal_actions=False):
+        return O.__dict__["_orig_suffix_visibility"](prefix_valid, horizon, False)
+
+    def xpred_sign(out, noise, x_prediction):
+        return noise - out if x_prediction else out
+
+    def grid_reversed(num_steps, convention="pi0"):
+        t, dt = O.__dict__["_orig_time_grid"](num_steps, convention)
+        if convention == "linspace":
+            t = [np.float32(1.0) - x for x in t]
+        return t, dt
+
     def gelu_erf(x):
         import scipy.special
         return 0.5 * x * (1.0 + scipy.special.erf(x / math.sqrt(2.0)))
 
     return {
-        "apply_rope": rope_sign,
-        "rms_norm": rms_no_one,
-        "time_embedding": temb_swapped,
-        "suffix_visibility": vis_state_sees_all,
-        "suffix_positions": pos_off_by_one,
-        "gelu_tanh": gelu_erf,
+        # label: (oracle function replaced, mutant, variant the brute-force comparison runs)
+        "apply_rope": ("apply_rope", rope_sign, {}),
+        "rms_norm": ("rms_norm", rms_no_one, {}),
+        "time_embedding": ("time_embedding", temb_swapped, {}),
+        "suffix_visibility": ("suffix_visibility", vis_state_sees_all, {}),
+        "suffix_positions": ("suffix_positions", pos_off_by_one, {}),
+        "gelu_tanh": ("gelu_tanh", gelu_erf, {}),
+        "causal_mask_ignored": ("suffix_visibility", vis_causal_ignored, {"causal_actions": True}),
+        "x_prediction_sign": ("output_to_velocity", xpred_sign, {"x_prediction": True}),
+        "time_grid_reversed": ("time_grid", grid_reversed, {"time_convention": "linspace"}),
     }
 
 
-@pytest.mark.parametrize("name", sorted(_mutations()))
-def test_planted_mistakes_are_caught(name, monkeypatch):
-    fn = _mutations()[name]
+@pytest.mark.parametrize("label", sorted(_mutations()))
+def test_planted_mistakes_are_caught(label, monkeypatch):
+    name, fn, variant = _mutations()[label]
     monkeypatch.setitem(O.__dict__, "_orig_" + name, getattr(O, name))
     monkeypatch.setattr(O, name, fn)
-    ours, ref = _brute_and_oracle(np.float64)
-    assert np.max(np.abs(ours - ref)) > 1e-6, f"planted mistake in {name} went unnoticed"
+    dims = synth.TINY_BRUTE_DIMS
+    w, pk, pv, mask, state, x1, steps = tiny_float_inputs(dims)
+    ref = np.array(brute_sample(w, pk, pv, mask, state, x1, steps, dims.num_heads, **variant))
+    ours = O.sample_actions(w, pk, pv, mask, state, x1, steps, num_heads=dims.num_heads, dtype=np.float64,
+                            **variant)
+    assert np.max(np.abs(ours - ref)) > 1e-6, f"planted mistake {label} went unnoticed"
