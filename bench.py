@@ -123,7 +123,13 @@ def blas_threads():
     return os.cpu_count() or 1
 
 
-def time_oracle(wl, budget_s=12.0, max_reps=50):
+def variant_of(args):
+    """The solver / convention variant the run uses (oracle keyword arguments)."""
+    return dict(time_convention=args.time_grid, x_prediction=args.x_prediction,
+                causal_actions=args.causal_actions)
+
+
+def time_oracle(wl, budget_s=12.0, max_reps=50, variant=None):
     """The CPU oracle, as it stands, on bounded samples of the workload.
 
     Each repetition runs all Euler steps of one sample (one action chunk).
@@ -136,7 +142,7 @@ def time_oracle(wl, budget_s=12.0, max_reps=50):
         inp = synth.make_inputs(wl, samples=[b % wl.batch], weights=w)
         t0 = time.perf_counter()
         O.sample_actions(inp.weights, inp.prefix_k, inp.prefix_v, inp.mask, inp.state, inp.x1,
-                         wl.num_steps)
+                         wl.num_steps, **(variant or {}))
         t_total += time.perf_counter() - t0
         reps += 1
         b += 1
@@ -157,7 +163,7 @@ def run_reference(args, wl):
     def one(i):
         inp = inps[i % len(inps)]
         O.sample_actions(inp.weights, inp.prefix_k, inp.prefix_v, inp.mask, inp.state, inp.x1,
-                         wl.num_steps)
+                         wl.num_steps, **variant_of(args))
     for i in range(args.warmup):
         one(i)
     t0 = time.perf_counter()
@@ -185,6 +191,8 @@ def config_of(wl, args):
     return {"workload": wl.name, "batch": wl.batch, "prefix_len": wl.prefix_len,
             "num_steps": wl.num_steps, "depth": d.depth, "horizon": d.horizon,
             "action_dim": d.action_dim, "width": d.width, "precision": args.precision,
+            "time_grid": args.time_grid, "x_prediction": args.x_prediction,
+            "causal_actions": args.causal_actions,
             "l2": "inputs larger than L2: every Euler step streams the 629 MB of bf16 expert "
                   "weights (126 MB L2)"}
 
@@ -199,6 +207,10 @@ def main():
     ap.add_argument("--precision", default="bf16", choices=["bf16", "fp32"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile-steps", type=int, default=3)
+    # solver / convention variant (pi0x_set_variant); the default is pi0's own loop
+    ap.add_argument("--time-grid", default="pi0", choices=["pi0", "linspace"])
+    ap.add_argument("--x-prediction", action="store_true")
+    ap.add_argument("--causal-actions", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -227,6 +239,8 @@ def main():
     precision = pi0x.PI0X_BF16 if args.precision == "bf16" else pi0x.PI0X_FP32
     inp = synth.make_inputs(wl)
     sampler = pi0x.Sampler(wl.dims, inp.weights, precision)
+    sampler.set_variant(pi0x.PI0X_TIME_LINSPACE if args.time_grid == "linspace" else pi0x.PI0X_TIME_PI0,
+                        args.x_prediction, args.causal_actions)
     dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()
     pk = [dev(k.view(np.int16)) for k in inp.prefix_k]
     pv = [dev(v.view(np.int16)) for v in inp.prefix_v]
@@ -339,7 +353,7 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        v, desc, cores = time_oracle(wl)
+        v, desc, cores = time_oracle(wl, variant=variant_of(args))
         cpu = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc}
 
     if rank == 0:

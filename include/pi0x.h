@@ -131,6 +131,27 @@ int pi0x_sample(pi0x_handle *h, const void *const *prefix_k, const void *const *
  * of that call are invalid), PI0X_EDEVICE or PI0X_ECUDA.  Clears the word. */
 int pi0x_sync_status(pi0x_handle *h);
 
+/* ---- solver / convention variants --------------------------------------------
+ * The default is pi0's own loop (`sample_actions` / `denoise_step` on the
+ * vllm-omni pi0 page): t from 1 (noise) to 0 with dt = -1/N, the out-projection
+ * is the velocity, action tokens see each other.  pi0x_set_variant selects the
+ * conventions of the Wall-X flow-matching sampler instead, each independently:
+ *  - time_grid PI0X_TIME_LINSPACE: t from 0 (noise) to 1 on torch.linspace(0, 1,
+ *    N+1) integrated with a fixed-grid Euler step (its odeint call), taken as
+ *    t_k = fp32(k/N) correctly rounded, step size fp32(t_{k+1} - t_k);
+ *  - x_prediction = 1: the out-projection is the clean action x_hat and the
+ *    velocity is x_hat - x_1 (its use_x_pred branch: prediction minus noise);
+ *  - causal_actions = 1: action token i sees the prefix, the state and actions
+ *    0..i only (its causal_action_attention_mask, a lower-triangular suffix block).
+ * The setting applies to later pi0x_sample calls on the handle; changing it
+ * waits for the handle's last call and drops the cached graphs.
+ * Errors: PI0X_EINVAL for a null handle or a value out of range. */
+enum {
+  PI0X_TIME_PI0 = 0,      /* t: 1 -> 0, dt = -1/N */
+  PI0X_TIME_LINSPACE = 1  /* t: 0 -> 1 on fp32(k/N) */
+};
+int pi0x_set_variant(pi0x_handle *h, int time_grid, int x_prediction, int causal_actions);
+
 /* Number of kernels one pi0x_sample(B, P, num_steps) call launches (its own
  * kernels only, not memory copies), or -1 for invalid arguments. */
 long pi0x_launch_count(const pi0x_handle *h, int B, int P, int num_steps);

@@ -52,6 +52,7 @@ def test_null_arguments_are_rejected_without_a_gpu(lib):
     assert lib.pi0x_create(None, None, ctypes.byref(h)) == pi0x.PI0X_EINVAL
     assert lib.pi0x_sample(None, None, None, None, 1, 1, None, None, 1, None, None) == pi0x.PI0X_EINVAL
     assert lib.pi0x_sync_status(None) == pi0x.PI0X_EINVAL
+    assert lib.pi0x_set_variant(None, 0, 0, 0) == pi0x.PI0X_EINVAL
     assert lib.pi0x_launch_count(None, 1, 1, 1) == -1
     lib.pi0x_destroy(None)
 

@@ -21,7 +21,7 @@ constexpr int kAttnSmem = (kAttnKeys * (kHeadDim + 1) + kAttnKeys * kHeadDim + k
 template <typename T>
 __global__ void __launch_bounds__(128) k_attn_simt(const T *q, const T *ks, const T *vs, const CallPtrs *cp,
                                                     int layer, const int *nvalid, const int *vidx, Geo g,
-                                                    int step0, T *out) {
+                                                    int step0, int causal, T *out) {
   pdl_wait();
   pdl_trigger();
   extern __shared__ float sm[];
@@ -79,8 +79,12 @@ __global__ void __launch_bounds__(128) k_attn_simt(const T *q, const T *ks, cons
       const int qi = warp * 4 + qq, jq = qbase + qi;
       if (jq >= Tq) break;
       const bool state_q = step0 && jq == 0;
+      const int ja = step0 ? jq - 1 : jq;  // action index of an action query
+      // keys [prefix | state | actions]: the state query sees up to the state key, a
+      // causal action query up to its own action, other action queries all keys
+      const int last_key = state_q ? nv : (causal ? nv + 1 + ja : nkeys - 1);
       const int kk = k0 + lane;
-      const bool vis = kk < nkeys && (!state_q || kk <= nv);
+      const bool vis = kk < nkeys && kk <= last_key;
       float s = -INFINITY;
       if (vis) {
         const float *qv = Qs + qi * kHeadDim;
@@ -120,7 +124,7 @@ __global__ void __launch_bounds__(128) k_attn_simt(const T *q, const T *ks, cons
 
 template <typename T>
 void launch_attention(const T *q, const T *ks, const T *vs, const CallPtrs *cp, int layer, const int *nvalid,
-                      const int *vidx, const Geo &g, int step0, T *out, cudaStream_t s) {
+                      const int *vidx, const Geo &g, int step0, int causal, T *out, cudaStream_t s) {
   static bool attr_set = false;
   if (!attr_set) {
     cudaFuncSetAttribute(k_attn_simt<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, kAttnSmem);
@@ -128,12 +132,12 @@ void launch_attention(const T *q, const T *ks, const T *vs, const CallPtrs *cp, 
   }
   const int Tq = step0 ? g.H + 1 : g.H;
   dim3 grid(g.B, kHeads, (Tq + kAttnQ - 1) / kAttnQ);
-  launch_pdl(k_attn_simt<T>, grid, 128, kAttnSmem, s, q, ks, vs, cp, layer, nvalid, vidx, g, step0, out);
+  launch_pdl(k_attn_simt<T>, grid, 128, kAttnSmem, s, q, ks, vs, cp, layer, nvalid, vidx, g, step0, causal, out);
 }
 
 template void launch_attention<float>(const float *, const float *, const float *, const CallPtrs *, int,
-                                      const int *, const int *, const Geo &, int, float *, cudaStream_t);
+                                      const int *, const int *, const Geo &, int, int, float *, cudaStream_t);
 template void launch_attention<bf16>(const bf16 *, const bf16 *, const bf16 *, const CallPtrs *, int,
-                                     const int *, const int *, const Geo &, int, bf16 *, cudaStream_t);
+                                     const int *, const int *, const Geo &, int, int, bf16 *, cudaStream_t);
 
 }  // namespace pi0x

@@ -148,8 +148,8 @@ __device__ __forceinline__ void load_kv_tile(int blk, uint32_t tile, uint64_t *f
 
 __global__ void __launch_bounds__(kThreads, 1)
     k_attn_tc(const bf16 *q, const bf16 *ks, const bf16 *vs, const CallPtrs *cp, int layer, int sfx_row0,
-              const int *nvalid, const int *vidx, Geo g, int step0, int blocks_per_split, bf16 *out, float *part_o,
-              float *part_ml, unsigned *err) {
+              const int *nvalid, const int *vidx, Geo g, int step0, int causal, int blocks_per_split, bf16 *out,
+              float *part_o, float *part_ml, unsigned *err) {
   pdl_wait();
   pdl_trigger();
   if (*(volatile unsigned *)err != 0) return;
@@ -306,8 +306,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     int tok = 0;
     if (row_ok) tok = step0 ? (jq == 0 ? b : g.B + b * g.H + jq - 1) : g.B + b * g.H + jq;
     const bool state_q = step0 && jq == 0;
-    // visible suffix slots: the action keys (not for the state query) and the state key
-    const int sfx_lo = nbp * kKeyBlock + (state_q ? g.H : 0), sfx_hi = nbp * kKeyBlock + g.H + 1;
+    const int ja = step0 ? jq - 1 : jq;  // action index of an action query
+    // Visible suffix slots (actions at base + 0..H-1, the state at base + H): the
+    // state query sees the state slot only; an action query sees all of them, or
+    // under the causal action mask actions 0..ja plus the state slot.
+    const int sfx_base = nbp * kKeyBlock;
+    const int sfx_lo = sfx_base + (state_q ? g.H : 0);
+    const int sfx_hi = state_q ? sfx_base + g.H + 1 : (causal ? sfx_base + ja + 1 : sfx_base + g.H + 1);
+    const int sfx_state = sfx_base + g.H;
     const uint32_t t_lane = (uint32_t)(warp * 32) << 16;
     const float scale_l2 = 0.0625f * kLog2e;
 
@@ -342,11 +348,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       mbar_arrive(&s_empty[sb]);
       const int kbase = (blk0 + j) * kKeyBlock;
-      const int vis_lo = blk0 + j < nbp ? 0 : sfx_lo, vis_hi = blk0 + j < nbp ? nv : sfx_hi;
+      const bool pre_blk = blk0 + j < nbp;
+      const int vis_lo = pre_blk ? 0 : sfx_lo, vis_hi = pre_blk ? nv : sfx_hi;
+      const int vis_st = pre_blk ? -1 : sfx_state;  // also visible (the range may end before it)
       if (kbase < vis_lo || kbase + kKeyBlock > vis_hi) {  // some slot of the block is hidden from this row
 #pragma unroll
         for (int i = 0; i < 64; ++i)
-          if ((unsigned)(kbase + i - vis_lo) >= (unsigned)(vis_hi - vis_lo)) sv[i] = -INFINITY;
+          if ((unsigned)(kbase + i - vis_lo) >= (unsigned)(vis_hi - vis_lo) && kbase + i != vis_st) sv[i] = -INFINITY;
       }
       float bm;
       {  // block max in log2 units (the scale is positive); eight independent chains
@@ -544,8 +552,8 @@ bool attn_tc_maps(CallPtrs &cp, int layers, int B, int P, const void *ks, const 
 }
 
 void launch_attention_tc(const bf16 *q, const bf16 *ks, const bf16 *vs, const CallPtrs *cp, int layer,
-                         int sfx_row0, const int *nvalid, const int *vidx, const Geo &g, int step0, int splits,
-                         bf16 *out, float *part, unsigned *err, cudaStream_t s) {
+                         int sfx_row0, const int *nvalid, const int *vidx, const Geo &g, int step0, int causal,
+                         int splits, bf16 *out, float *part, unsigned *err, cudaStream_t s) {
   cudaFuncSetAttribute(k_attn_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemTotal);
   const int Tq = step0 ? g.H + 1 : g.H;
   const int mtiles = (kHeads * Tq + kRowsPerCta - 1) / kRowsPerCta;
@@ -554,8 +562,8 @@ void launch_attention_tc(const bf16 *q, const bf16 *ks, const bf16 *vs, const Ca
   float *part_o = part;
   float *part_ml = splits > 1 ? part + (size_t)g.B * splits * mtiles * kRowsPerCta * kHeadDim : nullptr;
   dim3 grid(mtiles, splits, g.B);
-  launch_pdl(k_attn_tc, grid, kThreads, kSmemTotal, s, q, ks, vs, cp, layer, sfx_row0, nvalid, vidx, g, step0, bps,
-             out, part_o, part_ml, err);
+  launch_pdl(k_attn_tc, grid, kThreads, kSmemTotal, s, q, ks, vs, cp, layer, sfx_row0, nvalid, vidx, g, step0,
+             causal, bps, out, part_o, part_ml, err);
   if (splits > 1) {
     dim3 cg((kHeads * Tq + 7) / 8, g.B);
     launch_pdl(k_attn_combine, cg, 256, 0, s, part_o, part_ml, g, step0, splits, mtiles * kRowsPerCta, out);

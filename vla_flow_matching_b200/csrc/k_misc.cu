@@ -52,13 +52,15 @@ void launch_prep_mask(const CallPtrs *cp, int B, int P, int *nvalid, int *vidx, 
 // (`create_sinusoidal_pos_embedding`, min period 4e-3, max period 4).  The result
 // is the same for every sample and action token, so it is formed once per call.
 template <typename TW>
-__global__ void __launch_bounds__(256) k_time_vec(const TW *wt, const float *bias, int num_steps, float *tvec) {
+__global__ void __launch_bounds__(256) k_time_vec(const TW *wt, const float *bias, int num_steps, int linspace,
+                                                   float *tvec) {
   pdl_wait();
   pdl_trigger();
   __shared__ float temb[kWidth];
   const int k = blockIdx.x;
+  // step time: pi0 grid fp32(1 + k*(-1/N)); linspace grid fp32(k/N) (correctly rounded)
   const double dt = -1.0 / (double)num_steps;
-  const float t = (float)(1.0 + (double)k * dt);
+  const float t = linspace ? (float)((double)k / (double)num_steps) : (float)(1.0 + (double)k * dt);
   constexpr int half = kWidth / 2;
   for (int i = threadIdx.x; i < half; i += blockDim.x) {
     const double frac = (double)i / (double)(half - 1);
@@ -80,8 +82,8 @@ __global__ void __launch_bounds__(256) k_time_vec(const TW *wt, const float *bia
 }
 
 template <typename TW>
-void launch_time_vec(const TW *w_time, const float *bias, int num_steps, float *tvec, cudaStream_t s) {
-  launch_pdl(k_time_vec<TW>, dim3(num_steps, kWidth / 32), 256, 0, s, w_time, bias, num_steps, tvec);
+void launch_time_vec(const TW *w_time, const float *bias, int num_steps, int linspace, float *tvec, cudaStream_t s) {
+  launch_pdl(k_time_vec<TW>, dim3(num_steps, kWidth / 32), 256, 0, s, w_time, bias, num_steps, linspace, tvec);
 }
 
 // State token: h[b] = state_proj(state[b]) (`embed_suffix`).  With `gain` set it
@@ -312,7 +314,7 @@ void launch_geglu(const float *raw, int row0, int rows, T *act, cudaStream_t s) 
 template <int kEulerRows>
 __global__ void __launch_bounds__(256) k_final_euler(const float *h, Geo g, const float *gain, const float *w_out,
                                                       const float *b_out, float dt, float *x, const CallPtrs *cp,
-                                                      int last) {
+                                                      int last, int x_pred) {
   pdl_wait();
   pdl_trigger();
   __shared__ float y[kEulerRows][kWidth];
@@ -350,8 +352,9 @@ __global__ void __launch_bounds__(256) k_final_euler(const float *h, Geo g, cons
       float mine = acc[0];
 #pragma unroll
       for (int r = 1; r < kEulerRows; ++r) mine = lane == r ? acc[r] : mine;
-      const float v = mine + b_out[a];
       const size_t xi = (size_t)(i0 + lane) * g.A + a;
+      float v = mine + b_out[a];
+      if (x_pred) v -= cp->x1[xi];  // output is the clean action: velocity = x_hat - noise
       const float xn = __fadd_rn(x[xi], __fmul_rn(dt, v));
       x[xi] = xn;
       if (last) cp->x0[xi] = xn;
@@ -360,12 +363,12 @@ __global__ void __launch_bounds__(256) k_final_euler(const float *h, Geo g, cons
 }
 
 void launch_final_euler(const float *h, const Geo &g, const float *gain, const float *w_out, const float *b_out,
-                        float dt, float *x, const CallPtrs *cp, int last, cudaStream_t s) {
+                        float dt, float *x, const CallPtrs *cp, int last, int x_pred, cudaStream_t s) {
   const int rows = g.B * g.H;
   if (rows >= 8 * 148)
-    launch_pdl(k_final_euler<8>, (rows + 7) / 8, 256, 0, s, h, g, gain, w_out, b_out, dt, x, cp, last);
+    launch_pdl(k_final_euler<8>, (rows + 7) / 8, 256, 0, s, h, g, gain, w_out, b_out, dt, x, cp, last, x_pred);
   else
-    launch_pdl(k_final_euler<1>, rows, 256, 0, s, h, g, gain, w_out, b_out, dt, x, cp, last);
+    launch_pdl(k_final_euler<1>, rows, 256, 0, s, h, g, gain, w_out, b_out, dt, x, cp, last, x_pred);
 }
 
 __global__ void k_copy_x1(const CallPtrs *cp, int n, float *x) {
@@ -385,8 +388,8 @@ __global__ void k_delay(unsigned long long ns) {
 void launch_delay_ns(unsigned long long ns, cudaStream_t s) { k_delay<<<1, 1, 0, s>>>(ns); }
 
 // ---- explicit instantiations ----
-template void launch_time_vec<float>(const float *, const float *, int, float *, cudaStream_t);
-template void launch_time_vec<bf16>(const bf16 *, const float *, int, float *, cudaStream_t);
+template void launch_time_vec<float>(const float *, const float *, int, int, float *, cudaStream_t);
+template void launch_time_vec<bf16>(const bf16 *, const float *, int, int, float *, cudaStream_t);
 template void launch_state_embed<float>(const CallPtrs *, const float *, const float *, int, int, float *,
                                         cudaStream_t, const float *, bf16 *, float *, int);
 template void launch_state_embed<bf16>(const CallPtrs *, const bf16 *, const float *, int, int, float *,

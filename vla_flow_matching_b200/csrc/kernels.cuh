@@ -126,7 +126,7 @@ inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, siz
 // ---- misc kernels (k_misc.cu) ----
 void launch_prep_mask(const CallPtrs *cp, int B, int P, int *nvalid, int *vidx, cudaStream_t s);
 template <typename TW>
-void launch_time_vec(const TW *w_time, const float *bias, int num_steps, float *tvec, cudaStream_t s);
+void launch_time_vec(const TW *w_time, const float *bias, int num_steps, int linspace, float *tvec, cudaStream_t s);
 template <typename TW>
 void launch_state_embed(const CallPtrs *cp, const TW *w, const float *b, int B, int S, float *h, cudaStream_t s,
                         const float *gain = nullptr, bf16 *xn = nullptr, float *ss = nullptr, int ss_ld = 0);
@@ -139,8 +139,9 @@ void launch_rope_qkv(const float *raw, int row0, int rows, const Geo &g, const i
                      T *q, T *ks, T *vs, cudaStream_t s);
 template <typename T>
 void launch_geglu(const float *raw, int row0, int rows, T *act, cudaStream_t s);
+// x_pred: the out-projection is the clean action; velocity = it - cp->x1.
 void launch_final_euler(const float *h, const Geo &g, const float *gain, const float *w_out, const float *b_out,
-                        float dt, float *x, const CallPtrs *cp, int last, cudaStream_t s);
+                        float dt, float *x, const CallPtrs *cp, int last, int x_pred, cudaStream_t s);
 void launch_copy_x1(const CallPtrs *cp, int n, float *x, cudaStream_t s);
 void launch_delay_ns(unsigned long long ns, cudaStream_t s);
 void launch_rope_table(const float *inv_freq, int npos, float *tab, cudaStream_t s);
@@ -148,7 +149,7 @@ void launch_rope_table(const float *inv_freq, int npos, float *tab, cudaStream_t
 // ---- attention (k_attn.cu) ----
 template <typename T>
 void launch_attention(const T *q, const T *ks, const T *vs, const CallPtrs *cp, int layer, const int *nvalid,
-                      const int *vidx, const Geo &g, int step0, T *out, cudaStream_t s);
+                      const int *vidx, const Geo &g, int step0, int causal, T *out, cudaStream_t s);
 
 // tcgen05 attention (k_attn_tc.cu); `part` holds attn_tc_partial_floats() floats
 // when splits > 1.
@@ -162,9 +163,10 @@ size_t attn_tc_partial_floats(const Geo &g, int step0, int splits);
 // pointer that is not 16-byte aligned).
 bool attn_tc_maps(CallPtrs &cp, int layers, int B, int P, const void *ks, const void *vs, uint64_t sfx_rows);
 // ks / vs: this layer's suffix rows, which start at row `sfx_row0` of cp->sfx_map.
+// causal: the causal action mask (action query i sees actions 0..i and the state).
 void launch_attention_tc(const bf16 *q, const bf16 *ks, const bf16 *vs, const CallPtrs *cp, int layer,
-                         int sfx_row0, const int *nvalid, const int *vidx, const Geo &g, int step0, int splits,
-                         bf16 *out, float *part, unsigned *err, cudaStream_t s);
+                         int sfx_row0, const int *nvalid, const int *vidx, const Geo &g, int step0, int causal,
+                         int splits, bf16 *out, float *part, unsigned *err, cudaStream_t s);
 bool make_map(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols, uint64_t pitch, uint32_t box_rows);
 
 // Text for pi0x_last_error() (this thread).

@@ -119,7 +119,8 @@ extern "C" int pi0x_attention_noalloc(const void *q, const void *ks, const void 
   if (e == cudaSuccess) e = cudaMemsetAsync(d_err, 0, sizeof(unsigned), s);
   if (e == cudaSuccess) {
     launch_prep_mask(d_cp, B, P, nvalid, vidx, s);
-    launch_attention_tc((const bf16 *)q, (const bf16 *)ks, (const bf16 *)vs, d_cp, 0, 0, nvalid, vidx, g, step0, splits,
+    launch_attention_tc((const bf16 *)q, (const bf16 *)ks, (const bf16 *)vs, d_cp, 0, 0, nvalid, vidx, g, step0, 0,
+                        splits,
                         (bf16 *)out, part, d_err, s);
     e = cudaGetLastError();
   }

@@ -142,6 +142,8 @@ struct pi0x_handle {
   unsigned *d_err = nullptr;
   cudaStream_t last_stream = nullptr;  // stream of the last call (NULL = legacy default)
   bool called = false;
+  // solver / convention variant (pi0x_set_variant)
+  int time_grid = PI0X_TIME_PI0, x_pred = 0, causal = 0;
   cudaStream_t cap = nullptr;   // capture stream (graphs are launched on the caller's stream)
   struct Graph {
     int B, P, N, prof;
@@ -422,7 +424,14 @@ int enqueue_loop(pi0x_handle *h, int B, int P, int N, cudaStream_t s) {
   const int H = c.horizon, A = c.action_dim, L = c.depth;
   Geo g{B, H, A, c.state_dim, P, B + B * H};
   const int R = g.R, BH = B * H;
-  const float dt = (float)(-1.0 / (double)N);
+  // step sizes: the pi0 grid steps by fp32(-1/N); the linspace grid by the fp32
+  // difference of consecutive fp32(k/N)
+  const bool linspace = h->time_grid == PI0X_TIME_LINSPACE;
+  auto step_dt = [&](int k) -> float {
+    if (!linspace) return (float)(-1.0 / (double)N);
+    const float t0 = (float)((double)k / (double)N), t1 = (float)((double)(k + 1) / (double)N);
+    return t1 - t0;
+  };
   const bool tc = h->bf16;
   T *xn = (T *)ws.xn, *q = (T *)ws.q, *att = (T *)ws.att, *act = (T *)ws.act;
   T *aemb = (T *)ws.a_emb, *uemb = (T *)ws.u_emb;
@@ -443,7 +452,7 @@ int enqueue_loop(pi0x_handle *h, int B, int P, int N, cudaStream_t s) {
   };
 
   RUN(PI0X_K_PREP, launch_prep_mask(h->d_ptrs, B, P, ws.nvalid, ws.vidx, s));
-  RUN(PI0X_K_PREP, launch_time_vec<T>((const T *)h->tin_t, h->tin_b, N, ws.tvec, s));
+  RUN(PI0X_K_PREP, launch_time_vec<T>((const T *)h->tin_t, h->tin_b, N, linspace ? 1 : 0, ws.tvec, s));
   RUN(PI0X_K_PREP, launch_copy_x1(h->d_ptrs, BH * A, ws.xw, s));
   if (tc) RUN(PI0X_K_PREP, launch_rope_table(h->inv_freq, P + H + 1, ws.rope_tab, s));
 
@@ -507,10 +516,11 @@ int enqueue_loop(pi0x_handle *h, int B, int P, int N, cudaStream_t s) {
       if (tc) {
         const int splits = attn_tc_splits(g, step0);
         RUN(PI0X_K_ATTN, launch_attention_tc((const bf16 *)q, (const bf16 *)ks, (const bf16 *)vs, h->d_ptrs, l,
-                                             l * R, ws.nvalid, ws.vidx, g, step0, splits, (bf16 *)att, ws.part,
-                                             h->d_err, s));
+                                             l * R, ws.nvalid, ws.vidx, g, step0, h->causal, splits, (bf16 *)att,
+                                             ws.part, h->d_err, s));
       } else {
-        RUN(PI0X_K_ATTN, launch_attention<T>(q, ks, vs, h->d_ptrs, l, ws.nvalid, ws.vidx, g, step0, att, s));
+        RUN(PI0X_K_ATTN, launch_attention<T>(q, ks, vs, h->d_ptrs, l, ws.nvalid, ws.vidx, g, step0, h->causal, att,
+                                             s));
       }
       GemmOut o_res{ws.h, kWidth, row0, nullptr};
       EpiArgs eres = ebase;
@@ -556,7 +566,8 @@ int enqueue_loop(pi0x_handle *h, int B, int P, int N, cudaStream_t s) {
                                 kWidth, kMlp, EPI_RESID_F32, o_res, s));
       }
     }
-    RUN(PI0X_K_FINAL, launch_final_euler(ws.h, g, h->fnorm, h->aout_w, h->aout_b, dt, ws.xw, h->d_ptrs, k == N - 1, s));
+    RUN(PI0X_K_FINAL, launch_final_euler(ws.h, g, h->fnorm, h->aout_w, h->aout_b, step_dt(k), ws.xw, h->d_ptrs,
+                                         k == N - 1, h->x_pred, s));
   }
   CK(cudaGetLastError());
   return PI0X_OK;
@@ -679,11 +690,11 @@ int pi0x_debug_attention(const void *q, const void *ks, const void *vs, const vo
   if (e == cudaSuccess) {
     launch_prep_mask(d_cp, B, P, nvalid, vidx, s);
     if (impl == 0) {
-      launch_attention<bf16>((const bf16 *)q, (const bf16 *)ks, (const bf16 *)vs, d_cp, 0, nvalid, vidx, g, step0,
+      launch_attention<bf16>((const bf16 *)q, (const bf16 *)ks, (const bf16 *)vs, d_cp, 0, nvalid, vidx, g, step0, 0,
                              (bf16 *)out, s);
     } else {
       const int splits = impl == 2 ? 1 : attn_tc_splits(g, step0);
-      launch_attention_tc((const bf16 *)q, (const bf16 *)ks, (const bf16 *)vs, d_cp, 0, 0, nvalid, vidx, g, step0,
+      launch_attention_tc((const bf16 *)q, (const bf16 *)ks, (const bf16 *)vs, d_cp, 0, 0, nvalid, vidx, g, step0, 0,
                           splits, (bf16 *)out, part, err, s);
     }
     e = cudaGetLastError();
@@ -935,6 +946,20 @@ int pi0x_sync_status(pi0x_handle *h) {
     g_last_error = "device error word 0x" + std::to_string(err);
     return (err & (kErrTimeoutProducer | kErrTimeoutMma | kErrTimeoutEpilogue)) ? PI0X_ETIMEOUT : PI0X_EDEVICE;
   }
+  return PI0X_OK;
+}
+
+int pi0x_set_variant(pi0x_handle *h, int time_grid, int x_prediction, int causal_actions) {
+  if (!h || (time_grid != PI0X_TIME_PI0 && time_grid != PI0X_TIME_LINSPACE) || x_prediction < 0 ||
+      x_prediction > 1 || causal_actions < 0 || causal_actions > 1)
+    return PI0X_EINVAL;
+  if (time_grid == h->time_grid && x_prediction == h->x_pred && causal_actions == h->causal) return PI0X_OK;
+  // the captured graphs bake the variant in: let in-flight calls finish, then drop them
+  if (h->called) CK(cudaStreamSynchronize(h->last_stream));
+  drop_graphs(h);
+  h->time_grid = time_grid;
+  h->x_pred = x_prediction;
+  h->causal = causal_actions;
   return PI0X_OK;
 }
 

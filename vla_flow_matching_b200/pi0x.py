@@ -21,7 +21,12 @@ PI0X_DTYPE_BF16, PI0X_DTYPE_F32 = 0, 1
 #: Every symbol include/pi0x.h declares.
 EXPORTED = ["pi0x_create", "pi0x_sample", "pi0x_sync_status", "pi0x_launch_count",
             "pi0x_status_string", "pi0x_last_error", "pi0x_destroy", "pi0x_version",
-            "pi0x_debug_gemm_bf16", "pi0x_debug_attention", "pi0x_profile_enable", "pi0x_profile_read"]
+            "pi0x_debug_gemm_bf16", "pi0x_debug_attention", "pi0x_profile_enable", "pi0x_profile_read",
+            "pi0x_set_variant"]
+
+#: time grids of pi0x_set_variant
+PI0X_TIME_PI0 = 0
+PI0X_TIME_LINSPACE = 1
 
 #: kernel classes of pi0x_profile_read
 K_CLASSES = ["prep", "embed", "gemm", "norm", "rope", "attn", "geglu", "final"]
@@ -78,6 +83,8 @@ def load() -> ctypes.CDLL:
                                 ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int,
                                 ctypes.c_void_p, ctypes.c_void_p]
     lib.pi0x_sample.restype = ctypes.c_int
+    lib.pi0x_set_variant.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int]
+    lib.pi0x_set_variant.restype = ctypes.c_int
     lib.pi0x_sync_status.argtypes = [ctypes.c_void_p]
     lib.pi0x_sync_status.restype = ctypes.c_int
     lib.pi0x_launch_count.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int]
@@ -202,6 +209,12 @@ class Sampler:
                                      int(num_steps), _ptr(x0), ctypes.c_void_p(stream)),
                "pi0x_sample")
         return x0
+
+    def set_variant(self, time_grid: int = PI0X_TIME_PI0, x_prediction: bool = False,
+                    causal_actions: bool = False):
+        """Solver / convention variant for later calls (see pi0x_set_variant)."""
+        _check(self._lib.pi0x_set_variant(self._h, int(time_grid), int(bool(x_prediction)),
+                                          int(bool(causal_actions))), "pi0x_set_variant")
 
     def profile(self, on: bool = True):
         _check(self._lib.pi0x_profile_enable(self._h, int(on)), "pi0x_profile_enable")
