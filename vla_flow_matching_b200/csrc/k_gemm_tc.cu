@@ -79,15 +79,27 @@ __device__ __forceinline__ float consumer_rstd(const EpiArgs &e, int r) {
   return 1.f;
 }
 
-// Global operands of the epilogue of one 32-column chunk, loaded ahead of the chunk
-// (the residual row slice, bias, RoPE (cos, sin) pairs; norm gain in g).
+// Global operands of the epilogue of one 32-column chunk, loaded ahead of the chunk:
+// the residual row slice, the bias, or the RoPE (cos, sin) pairs.  (The norm gain is
+// the same for every row and is read from L1 when used.)
+constexpr int kEpiAhead = 2;  // chunks loaded ahead of the one in process
 struct EpiIn {
   float4 a[8];
-  float4 g[8];
 };
 
+// RoPE position of output row `orow` (EPI_QKV_ROPE), once per tile.
 template <int EPI>
-__device__ __forceinline__ void epi_fetch(const EpiArgs &e, int r, int n, EpiIn &in) {
+__device__ __forceinline__ int epi_pos(const EpiArgs &e, int orow) {
+  if constexpr (EPI == EPI_QKV_ROPE) {
+    int b, j;
+    row_to_bj_tc(orow, e.B, e.H, b, j);
+    return e.nvalid[b] + j;
+  }
+  return 0;
+}
+
+template <int EPI>
+__device__ __forceinline__ void epi_fetch(const EpiArgs &e, int r, int n, int pos, EpiIn &in) {
   const int orow = e.out_row0 + r;
   if constexpr (EPI == EPI_RESID_F32) {
     const float4 *src = reinterpret_cast<const float4 *>(e.out_f32 + (size_t)orow * e.ldo + n);
@@ -98,9 +110,6 @@ __device__ __forceinline__ void epi_fetch(const EpiArgs &e, int r, int n, EpiIn 
 #pragma unroll
     for (int i = 0; i < 8; ++i) in.a[i] = src[i];
   } else if constexpr (EPI == EPI_QKV_ROPE) {
-    int b, j;
-    row_to_bj_tc(orow, e.B, e.H, b, j);
-    const int pos = e.nvalid[b] + j;
 #pragma unroll
     for (int gi = 0; gi < 2; ++gi) {
       const int gc = (n >> 4) + gi;
@@ -113,13 +122,8 @@ __device__ __forceinline__ void epi_fetch(const EpiArgs &e, int r, int n, EpiIn 
       }
     }
   }
-  if constexpr (EPI == EPI_RESID_F32 || EPI == EPI_BIAS_F32) {
-    if (e.gain) {
-      const float4 *gs = reinterpret_cast<const float4 *>(e.gain + n);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) in.g[i] = gs[i];
-    }
-  }
+  (void)pos;
+  (void)orow;
 }
 
 // Epilogue of 32 consecutive output columns [n, n+32) of GEMM row r (`rs` from
@@ -146,7 +150,7 @@ __device__ __forceinline__ float epilogue32(const EpiArgs &e, int r, int n, floa
         float t[32];
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-          const float4 gg = in.g[i];
+          const float4 gg = reinterpret_cast<const float4 *>(e.gain + n)[i];
           ssq = fmaf(v[4 * i], v[4 * i], ssq);
           ssq = fmaf(v[4 * i + 1], v[4 * i + 1], ssq);
           ssq = fmaf(v[4 * i + 2], v[4 * i + 2], ssq);
@@ -333,14 +337,19 @@ __global__ void __launch_bounds__(128, 1)
     if (splits == 1) {
       float ssq = 0.f;
       const float rs = r < M ? consumer_rstd<EPI>(e, r) : 1.f;
-      EpiIn in[2];
-      if (r < M) epi_fetch<EPI>(e, r, n0, in[0]);
+      const int pos = r < M ? epi_pos<EPI>(e, e.out_row0 + r) : 0;
+      EpiIn in[kEpiAhead + 1];
+#pragma unroll
+      for (int c = 0; c < kEpiAhead * 32 && c < BN; c += 32)
+        if (r < M) epi_fetch<EPI>(e, r, n0 + c, pos, in[c >> 5]);
 #pragma unroll
       for (int c = 0; c < BN; c += 32) {
-        if (c + 32 < BN && r < M) epi_fetch<EPI>(e, r, n0 + c + 32, in[((c >> 5) + 1) & 1]);
+        const int ci = c >> 5;
+        if (c + kEpiAhead * 32 < BN && r < M)
+          epi_fetch<EPI>(e, r, n0 + c + kEpiAhead * 32, pos, in[(ci + kEpiAhead) % (kEpiAhead + 1)]);
         float v[32];
         tmem_ld_32x32b_x32(tmem + t_lane + (uint32_t)c, v);
-        if (r < M) ssq += epilogue32<EPI>(e, r, n0 + c, v, rs, in[(c >> 5) & 1]);
+        if (r < M) ssq += epilogue32<EPI>(e, r, n0 + c, v, rs, in[ci % (kEpiAhead + 1)]);
       }
       if (r < M) norm_partial_store<EPI>(e, r, n0, BN, gridDim.y * BN, ssq);
     } else {
@@ -383,7 +392,7 @@ __global__ void __launch_bounds__(128, 1)
               }
             }
             EpiIn in;
-            epi_fetch<EPI>(e, r, n0 + c, in);
+            epi_fetch<EPI>(e, r, n0 + c, epi_pos<EPI>(e, e.out_row0 + r), in);
             ssq += epilogue32<EPI>(e, r, n0 + c, v, rs, in);
           }
           norm_partial_store<EPI>(e, r, n0, BN, gridDim.y * BN, ssq);
@@ -523,8 +532,11 @@ __global__ void __launch_bounds__(192, 1)
       const int r = m0 + q * 32 + lane;
       // operands of the first chunk and the row's norm scale load while the MMAs run
       const float rs = r < M ? consumer_rstd<EPI>(e, r) : 1.f;
-      EpiIn in[2];
-      if (r < M) epi_fetch<EPI>(e, r, n0, in[0]);
+      const int pos = r < M ? epi_pos<EPI>(e, e.out_row0 + r) : 0;
+      EpiIn in[kEpiAhead + 1];
+#pragma unroll
+      for (int c = 0; c < kEpiAhead * 32 && c < BN; c += 32)
+        if (r < M) epi_fetch<EPI>(e, r, n0 + c, pos, in[c >> 5]);
       const bool ok = mbar_wait(&acc_full[a], around & 1u, err, kErrTimeoutEpilogue);
       __syncwarp();
       if (!__all_sync(0xffffffffu, ok)) break;
@@ -532,10 +544,12 @@ __global__ void __launch_bounds__(192, 1)
       float ssq = 0.f;
 #pragma unroll
       for (int c = 0; c < BN; c += 32) {
-        if (c + 32 < BN && r < M) epi_fetch<EPI>(e, r, n0 + c + 32, in[((c >> 5) + 1) & 1]);
+        const int ci = c >> 5;
+        if (c + kEpiAhead * 32 < BN && r < M)
+          epi_fetch<EPI>(e, r, n0 + c + kEpiAhead * 32, pos, in[(ci + kEpiAhead) % (kEpiAhead + 1)]);
         float v[32];
         tmem_ld_32x32b_x32(tmem + (uint32_t)(a * C::kTmemCols) + t_lane + (uint32_t)c, v);
-        if (r < M) ssq += epilogue32<EPI>(e, r, n0 + c, v, rs, in[(c >> 5) & 1]);
+        if (r < M) ssq += epilogue32<EPI>(e, r, n0 + c, v, rs, in[ci % (kEpiAhead + 1)]);
       }
       if (r < M) norm_partial_store<EPI>(e, r, n0, BN, N, ssq);
       tc_fence_before();
