@@ -140,7 +140,7 @@ __global__ void __launch_bounds__(256) k_action_in(const float *x, const TW *w, 
                                                     T *out) {
   pdl_wait();
   pdl_trigger();
-  __shared__ float xv[kActRows][64];
+  __shared__ __align__(16) float xv[kActRows][64];
   const int r0 = blockIdx.x * kActRows;
   for (int e = threadIdx.x; e < kActRows * A; e += blockDim.x) {
     const int r = e / A, i = e % A;
@@ -167,9 +167,16 @@ __global__ void __launch_bounds__(256) k_action_in(const float *x, const TW *w, 
   const float bn = bias[n];
   for (int r = 0; r < kActRows && r0 + r < rows; ++r) {
     float acc = 0.f;
+    const float4 *xr = reinterpret_cast<const float4 *>(xv[r]);  // 16-byte shared loads (broadcast)
 #pragma unroll
-    for (int i = 0; i < 64; ++i)
-      if (i < A) acc = fmaf(wr[i], xv[r][i], acc);
+    for (int i4 = 0; i4 < 16; ++i4) {
+      if (4 * i4 >= A) break;
+      const float4 xq = xr[i4];
+      const float xs[4] = {xq.x, xq.y, xq.z, xq.w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        if (4 * i4 + k < A) acc = fmaf(wr[4 * i4 + k], xs[k], acc);
+    }
     out[(size_t)(r0 + r) * kWidth + n] = from_f32<T>(acc + bn);
   }
 }
@@ -317,7 +324,7 @@ __global__ void __launch_bounds__(256) k_final_euler(const float *h, Geo g, cons
                                                       int last, int x_pred) {
   pdl_wait();
   pdl_trigger();
-  __shared__ float y[kEulerRows][kWidth];
+  __shared__ __align__(16) float y[kEulerRows][kWidth];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int rows = g.B * g.H;
   const int i0 = blockIdx.x * kEulerRows;  // action row index b*H + (j-1)
@@ -337,14 +344,21 @@ __global__ void __launch_bounds__(256) k_final_euler(const float *h, Geo g, cons
   __syncthreads();
   const int nr = min(kEulerRows, rows - i0);
   for (int a = warp; a < g.A; a += 8) {
-    const float *wr = w_out + (size_t)a * kWidth;
+    const float4 *wr = reinterpret_cast<const float4 *>(w_out + (size_t)a * kWidth);
     float acc[kEulerRows];
 #pragma unroll
     for (int r = 0; r < kEulerRows; ++r) acc[r] = 0.f;
-    for (int c = lane; c < kWidth; c += 32) {
-      const float wv = wr[c];
+    // lane takes columns 4*lane + 128*k .. +3 (16-byte loads of weights and rows)
+    for (int c4 = lane; c4 < kWidth / 4; c4 += 32) {
+      const float4 wv = wr[c4];
 #pragma unroll
-      for (int r = 0; r < kEulerRows; ++r) acc[r] = fmaf(wv, y[r][c], acc[r]);
+      for (int r = 0; r < kEulerRows; ++r) {
+        const float4 yv = reinterpret_cast<const float4 *>(y[r])[c4];
+        acc[r] = fmaf(wv.x, yv.x, acc[r]);
+        acc[r] = fmaf(wv.y, yv.y, acc[r]);
+        acc[r] = fmaf(wv.z, yv.z, acc[r]);
+        acc[r] = fmaf(wv.w, yv.w, acc[r]);
+      }
     }
 #pragma unroll
     for (int r = 0; r < kEulerRows; ++r) acc[r] = warp_sum(acc[r]);
