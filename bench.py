@@ -123,6 +123,24 @@ def blas_threads():
     return os.cpu_count() or 1
 
 
+def slowest_rank_ms(ms, dist, device="cuda"):
+    """The device time of the slowest rank: every rank passes its own CUDA-event time
+    and all take the same collective step (a MAX all-reduce); without a process
+    group the time is returned as is."""
+    if dist is None:
+        return ms
+    import torch
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world, batch, calls, ms):
+    """Whole-job chunks/s: every rank (one GPU) runs `calls` calls of `batch`
+    samples (replicas with a fixed per-GPU batch), all done in `ms`."""
+    return world * batch * calls / (ms / 1000.0)
+
+
 def variant_of(args):
     """The solver / convention variant the run uses (oracle keyword arguments)."""
     return dict(time_convention=args.time_grid, x_prediction=args.x_prediction,
@@ -273,13 +291,9 @@ def main():
         dist.barrier()
     clocks = sample_clocks_stop(clk, local) if clk else None
     sampler.sync()
-    ms = e0.elapsed_time(e1)
-    if dist is not None:
-        t = torch.tensor([ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = slowest_rank_ms(e0.elapsed_time(e1), dist)
     ms_per = ms / args.steps
-    value = world * B * args.steps / (ms / 1000.0)
+    value = job_throughput(world, B, args.steps, ms)
     if rank == 0:
         print(f"[bench] {wl.name} {args.precision}: {1000 * ms_per:.1f} us per call, "
               f"{value:.1f} {UNIT}", file=sys.stderr, flush=True)
@@ -303,12 +317,8 @@ def main():
         sampler.sample(hk, hv, hm, hs, hx, N, x0=hx0, stream=sid)
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1)
-    if dist is not None:
-        t = torch.tensor([e2e_ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e_value = world * B * e2e_steps / (e2e_ms / 1000.0)
+    e2e_ms = slowest_rank_ms(e0.elapsed_time(e1), dist)
+    e2e_value = job_throughput(world, B, e2e_steps, e2e_ms)
 
     # ---- per-kernel device time from the profiling graph (same workload) ----
     sampler.profile(True)
