@@ -2,7 +2,8 @@
 //
 // Computes, per sample and per query head, softmax(q . K^T / sqrt(256) + mask) . V
 // over the valid prefix keys, the state key and the action keys (`_attend` with the
-// block mask of `denoise_step` on the vllm-omni pi0 page).  The 8 query heads share
+// block mask of `denoise_step` on the vllm-omni pi0 page, or with the Wall-X page's
+// causal action mask: action i sees actions 0..i).  The 8 query heads share
 // the one KV head, so a CTA takes 128 query rows (token-major: row = token*8 + head)
 // of one sample against the sample's keys, in blocks of 64 key slots.
 //
@@ -18,10 +19,12 @@
 //    P = 2^(s - m) with an online softmax, writes P (bf16) to shared memory, and
 //    rescales O in TMEM when the running max grows by more than 2^8 (rare).
 //  * warp 4 / warp 5: K / V loader into 3-deep rings of 128-byte-swizzled tiles.  A
-//    run of 8 slots whose keys are consecutive rows of one tensor is one TMA box per
-//    64 dims; other runs are copied row by row with cp.async.
-//  * warp 6 lane 0: tcgen05.mma issuer: S(j+1) before PV(j), so the softmax of block
-//    j+1 overlaps the P.V of block j.
+//    block whose 64 slots are consecutive rows of one tensor is one 64-row TMA box
+//    per 64 dims; otherwise each such run of 8 slots is an 8-row box, and other runs
+//    are copied row by row with cp.async.
+//  * warp 6: tcgen05.mma issuer (the whole warp runs the loop, one elected lane
+//    issues): S(j+1) before PV(j), so the softmax of block j+1 overlaps the P.V of
+//    block j.
 // All hand-offs are mbarriers (TMA transaction bytes, cp.async completion, tcgen05
 // commits, thread arrivals) and every wait is bounded.  O / l at the end
 // normalises.  With split-KV (small batches) every split writes O/l and (m, l) and
