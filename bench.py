@@ -373,7 +373,8 @@ def main():
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": args.precision, "data": "synthetic (seeded numpy PCG64, bf16-rounded N(0,0.02) "
                                                "weights, N(0,1) prefix K/V, state, noise)",
-            "config": config_of(wl, args), "parallelism": f"replicas x{world} (batch per GPU fixed)",
+            "config": dict(config_of(wl, args), parallelism=f"replicas x{world} (batch per GPU fixed)"),
+            "parallelism": f"replicas x{world} (batch per GPU fixed)",
             "gpu_launches": sampler.launch_count(B, wl.prefix_len, N) * args.steps,
             "clocks": clocks,
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
