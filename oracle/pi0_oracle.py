@@ -246,25 +246,28 @@ def convert_weights(weights: dict, dtype) -> dict:
     return out
 
 
-def time_grid(num_steps: int, convention: str = "pi0"):
-    """Step times t_k (k < N, float32) and step sizes dt_k (float32).
+def time_grid(num_steps: int, convention: str = "pi0", dtype=np.float32):
+    """Step times t_k (k < N; float32, the value the time embedding receives) and
+    step sizes dt_k (in the model dtype).
 
-    "pi0" (``sample_actions``): t runs from 1 (noise) to 0, dt = -1/N taken as
-    float32, t_k = float32(1 + k*(-1/N)) with the product formed in float64.
-    "linspace" (the Wall-X sampler: ``torch.linspace(0, 1, N + 1)`` integrated
-    with a fixed-grid Euler step): t_k = float32(k/N), correctly rounded, and
-    dt_k = t_{k+1} - t_k in float32, so the noise sits at t = 0 and the action at t = 1.
+    "pi0" (``sample_actions``): t runs from 1 (noise) to 0; t_k = float32(1 + k*(-1/N))
+    with the product formed in float64, dt = -1/N (a Python double) taken in the
+    model dtype.
+    "linspace" (the Wall-X sampler: ``torch.linspace(0, 1, N + 1)`` in the model
+    dtype, integrated with a fixed-grid Euler step): grid points dtype(k/N),
+    correctly rounded, dt_k = their difference in the model dtype, and t_k =
+    float32(k/N), so the noise sits at t = 0 and the action at t = 1.
     """
     if num_steps <= 0:
         raise ValueError("num_steps must be positive")
     if convention == "pi0":
         dt_exact = -1.0 / num_steps
         t = [np.float32(1.0 + k * dt_exact) for k in range(num_steps)]
-        dt = [np.float32(dt_exact)] * num_steps
+        dt = [dtype(dt_exact)] * num_steps
     elif convention == "linspace":
-        pts = [np.float32(k / num_steps) for k in range(num_steps + 1)]
-        t = pts[:-1]
-        dt = [np.float32(pts[k + 1] - pts[k]) for k in range(num_steps)]
+        pts = [dtype(k / num_steps) for k in range(num_steps + 1)]
+        t = [np.float32(k / num_steps) for k in range(num_steps)]
+        dt = [dtype(pts[k + 1] - pts[k]) for k in range(num_steps)]
     else:
         raise ValueError(f"unknown time grid {convention!r}")
     return t, dt
@@ -304,7 +307,7 @@ def sample_actions(weights: dict, prefix_k: Sequence[np.ndarray],
     head_dim = prefix_k[0].shape[-1]
     kp = [as_float(k, dtype)[:, 0] for k in prefix_k]
     vp = [as_float(v, dtype)[:, 0] for v in prefix_v]
-    ts, dts = time_grid(num_steps, time_convention)
+    ts, dts = time_grid(num_steps, time_convention, dtype)
     noise = np.asarray(x1).astype(dtype)
     x = noise.copy()
     for step in range(num_steps):

@@ -70,8 +70,8 @@ def brute_sample(weights, prefix_k, prefix_v, mask, state, x1, num_steps, num_he
                  x_prediction=False, causal_actions=False):
     """weights: float arrays (nn.Linear layout); prefix_k/v: per layer (B,1,P,D) floats.
 
-    Variants (the Wall-X page): time_convention "linspace" steps t from 0 to 1 on
-    float32(k/N) with float32 differences as step sizes; x_prediction takes the
+    Variants (the Wall-X page): time_convention "linspace" steps t from 0 to 1 on the
+    grid k/N (the time embedding sees float32(k/N)); x_prediction takes the
     output as the clean action and moves along output - initial noise;
     causal_actions lets suffix query i see suffix keys 0..i only."""
     W = _mat(weights["state_proj_w"])
@@ -83,7 +83,7 @@ def brute_sample(weights, prefix_k, prefix_v, mask, state, x1, num_steps, num_he
     np = __import__("numpy")
     dt = -1.0 / num_steps
     if time_convention == "linspace":
-        grid = [float(np.float32(k / num_steps)) for k in range(num_steps + 1)]
+        grid = [k / num_steps for k in range(num_steps + 1)]
     x = [[_vec(row) for row in x1[b]] for b in range(B)]
     noise = [[_vec(row) for row in x1[b]] for b in range(B)]
     layers = [{k: (_mat(v) if getattr(v, "ndim", 1) == 2 else _vec(v)) for k, v in lw.items()}
@@ -92,8 +92,8 @@ def brute_sample(weights, prefix_k, prefix_v, mask, state, x1, num_steps, num_he
          for k, v in weights.items() if k != "layers"}
     for step in range(num_steps):
         if time_convention == "linspace":
-            t = grid[step]
-            h_step = float(np.float32(np.float32(grid[step + 1]) - np.float32(grid[step])))
+            t = float(np.float32(grid[step]))
+            h_step = grid[step + 1] - grid[step]
         else:
             t = float(np.float32(1.0 + step * dt))
             h_step = dt

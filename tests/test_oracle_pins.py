@@ -294,6 +294,34 @@ def test_brute_force_sees_the_mask_hole():
     assert np.array_equal(a, b)
 
 
+# --- edge shapes against the float64 brute force --------------------------------------
+EDGE_CASES = {
+    # name: (horizon, P, mask rows (1 = valid), steps)
+    "horizon_1": (1, 5, [[1, 1, 0, 1, 1], [1, 1, 1, 1, 0]], 2),
+    "no_valid_prefix": (3, 4, [[0, 0, 0, 0], [1, 0, 1, 1]], 2),
+    "one_position_prefix": (3, 1, [[1], [0]], 3),
+    "single_step": (3, 5, [[1, 1, 1, 1, 1], [1, 0, 0, 0, 0]], 1),
+}
+
+
+@pytest.mark.parametrize("variant", [{}, VARIANTS_ALL := dict(time_convention="linspace", x_prediction=True,
+                                                            causal_actions=True)],
+                         ids=["pi0", "variants"])
+@pytest.mark.parametrize("case", sorted(EDGE_CASES))
+def test_brute_force_float64_matches_edge_shapes(case, variant):
+    H, P, rows, steps = EDGE_CASES[case]
+    dims = dataclasses.replace(synth.TINY_BRUTE_DIMS, horizon=H)
+    w, pk, pv, _, state, x1, _ = tiny_float_inputs(dims, B=2, P=max(P, 2), n_masked=(0,))
+    pk = [k[:, :, :P] for k in pk]
+    pv = [v[:, :, :P] for v in pv]
+    mask = np.array(rows, np.uint8)
+    ref = np.array(brute_sample(w, pk, pv, mask, state, x1, steps, dims.num_heads, **variant))
+    ours = O.sample_actions(w, pk, pv, mask, state, x1, steps, num_heads=dims.num_heads, dtype=np.float64,
+                            **variant)
+    assert ours.shape == (2, H, dims.action_dim)
+    assert np.max(np.abs(ours - ref)) < 1e-11
+
+
 # --- solver / convention variants (the Wall-X page) -------------------------------------
 VARIANTS = [dict(time_convention="linspace"), dict(x_prediction=True), dict(causal_actions=True),
             dict(time_convention="linspace", x_prediction=True, causal_actions=True)]
@@ -395,8 +423,8 @@ def _mutations():
     def xpred_sign(out, noise, x_prediction):
         return noise - out if x_prediction else out
 
-    def grid_reversed(num_steps, convention="pi0"):
-        t, dt = O.__dict__["_orig_time_grid"](num_steps, convention)
+    def grid_reversed(num_steps, convention="pi0", dtype=np.float32):
+        t, dt = O.__dict__["_orig_time_grid"](num_steps, convention, dtype)
         if convention == "linspace":
             t = [np.float32(1.0) - x for x in t]
         return t, dt
