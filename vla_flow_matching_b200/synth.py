@@ -131,10 +131,13 @@ def weight_shapes(d: ExpertDims) -> Dict[str, tuple]:
 
 
 def f32_to_bf16_bits(x: np.ndarray) -> np.ndarray:
-    """Round fp32 to bf16 (nearest, ties to even); returns the uint16 bit pattern."""
+    """Round fp32 to bf16 (nearest, ties to even); returns the uint16 bit pattern.
+    NaN stays NaN (quiet, sign kept); overflow rounds to infinity."""
     u = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32)
     rounded = u + (np.uint32(0x7FFF) + ((u >> np.uint32(16)) & np.uint32(1)))
-    return (rounded >> np.uint32(16)).astype(np.uint16)
+    out = (rounded >> np.uint32(16)).astype(np.uint16)
+    nan = (u & np.uint32(0x7FFFFFFF)) > np.uint32(0x7F800000)
+    return np.where(nan, ((u >> np.uint32(16)) | np.uint32(0x0040)).astype(np.uint16), out)
 
 
 def bf16_bits_to_f32(bits: np.ndarray) -> np.ndarray:
