@@ -215,6 +215,117 @@ def config_of(wl, args):
                   "weights (126 MB L2)"}
 
 
+def hbm_bytes(wl):
+    """Compulsory HBM bytes of one call: every weight of the expert and of the
+    suffix embedding / out-projection read once per Euler step (bf16 matrices; the
+    fp32 out-projection, biases and norm gains), plus the valid prefix K/V of every
+    layer read once per step."""
+    d, N = wl.dims, wl.num_steps
+    W, F, Q, Dh, L, A = d.width, d.mlp_dim, d.num_heads * d.head_dim, d.head_dim, d.depth, d.action_dim
+    per_layer = 2 * (W * (Q + 2 * Dh) + W * Q + 2 * F * W + W * F) + 4 * 2 * W
+    embed = 2 * (W * A + 2 * W * W + W * W) + 4 * (4 * W) + 4 * (A * W + A + W)
+    n = synth.make_mask(wl).sum(axis=1).astype(np.int64)
+    kv = int(n.sum()) * L * Dh * 2 * 2
+    return N * (L * per_layer + embed + kv)
+
+
+def roofline_of(wl, kernel_ms, call_ms):
+    """Roofline of the kernel class with the most device time.
+
+    The class's time per call is its share of the profiled (serialised, one event
+    pair per kernel) device time times the graph-timed call, so it can never exceed
+    the call.  Work per call is algorithmic: the loop kernel (every step of a small
+    batch) moves the call's compulsory HBM bytes and runs all of its FLOPs; the GEMM
+    class moves its weights and operands (``algorithmic_work``)."""
+    pk_, src = peaks()
+    total = sum(kernel_ms.values())
+    dom = max(kernel_ms, key=kernel_ms.get)
+    t_ms = call_ms * kernel_ms[dom] / total
+    gbytes, gflops, aflops = algorithmic_work(wl)
+    if dom == "loop":
+        byt, flo, name = hbm_bytes(wl), gflops + aflops, "k_loop (persistent: every Euler step of the call)"
+    elif dom == "attn":
+        n = synth.make_mask(wl).sum(axis=1).astype(np.int64)
+        byt = int(n.sum()) * wl.dims.depth * wl.dims.head_dim * 4 * wl.num_steps
+        flo, name = aflops, "k_attn_tc (masked MQA attention)"
+    else:
+        byt, flo, name = gbytes, gflops, "k_gemm_tc (all expert and time-MLP Linears)"
+    ridge = pk_["bf16_tflops"] * 1e12 / (pk_["hbm_gbs"] * 1e9)
+    if flo / byt < ridge:
+        bound, peak, unit, psrc = "hbm", pk_["hbm_gbs"], "GB/s", f"{src} hbm_gbs"
+        ach, whole = byt / (t_ms / 1e3) / 1e9, hbm_bytes(wl) / (call_ms / 1e3) / 1e9
+    else:
+        bound, unit, psrc = "tensor", "TFLOP/s", f"{src} bf16_tflops_sustained"
+        peak = pk_.get("bf16_tflops_sustained", pk_["bf16_tflops"])
+        ach, whole = flo / (t_ms / 1e3) / 1e12, (gflops + aflops) / (call_ms / 1e3) / 1e12
+    traffic = TRAFFIC.get((wl.name, dom))
+    return {"kernel": name, "bound": bound, "achieved": ach, "peak": peak, "unit": unit, "frac": ach / peak,
+            "traffic": traffic, "peak_source": psrc, "kernel_ms_per_call": t_ms,
+            "kernel_share_of_profile": kernel_ms[dom] / total,
+            "whole_call": {"achieved": whole, "frac": whole / peak},
+            "algorithmic_per_call": {"bytes": byt, "flops": flo, "hbm_bytes": hbm_bytes(wl),
+                                     "gemm_bytes": gbytes, "gemm_flops": gflops, "attn_flops": aflops}}
+
+
+# DRAM bytes (read + write) per launch of the dominant kernel from an ncu capture of
+# the same build, keyed by (workload, kernel class); None when not captured.
+TRAFFIC = {}
+
+
+def measure(wl, args, sampler, inp, rank, dist, clocks_on):
+    """Device-timed throughput of whole calls on one workload (inputs resident)."""
+    import torch
+    dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()
+    pk = [dev(k.view(np.int16)) for k in inp.prefix_k]
+    pv = [dev(v.view(np.int16)) for v in inp.prefix_v]
+    mask, state, x1 = dev(inp.mask), dev(inp.state), dev(inp.x1)
+    x0 = torch.empty_like(x1)
+    stream = torch.cuda.current_stream()
+    sid = stream.cuda_stream
+    N = wl.num_steps
+    steps = args.steps if wl.name == args.workload else max(5, min(args.steps, 20))
+
+    def call():
+        sampler.sample(pk, pv, mask, state, x1, N, x0=x0, stream=sid)
+
+    for _ in range(args.warmup):
+        call()
+    sampler.sync()
+    clk = sample_clocks_start() if (rank == 0 and clocks_on) else None
+    time.sleep(0.3 if clk else 0)
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        call()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    clocks = sample_clocks_stop(clk, int(os.environ.get("LOCAL_RANK", "0"))) if clk else None
+    sampler.sync()
+    ms = slowest_rank_ms(e0.elapsed_time(e1), dist)
+    # per-kernel-class device time of the same call shape (serialised profile)
+    sampler.profile(True)
+    acc = {}
+    for _ in range(max(1, args.profile_steps)):
+        call()
+        for kname, (n, t) in sampler.profile_read().items():
+            a = acc.setdefault(kname, [0, 0.0])
+            a[0] += n
+            a[1] += t
+    sampler.profile(False)
+    sampler.sync()
+    ps = max(1, args.profile_steps)
+    kernel_ms = {k: v[1] / ps for k, v in acc.items() if v[0] > 0}
+    launches = {k: v[0] // ps for k, v in acc.items() if v[0] > 0}
+    out = {"ms": ms, "steps": steps, "clocks": clocks, "kernel_ms": kernel_ms, "launches": launches,
+           "tensors": (pk, pv, mask, state, x1, x0, sid)}
+    return out
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__)
     ap.add_argument("--gpus", type=int, default=1)
@@ -224,6 +335,8 @@ def main():
     ap.add_argument("--workload", default="full_b1", choices=sorted(synth.WORKLOADS))
     ap.add_argument("--precision", default="bf16", choices=["bf16", "fp32"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-by-workload", action="store_true",
+                    help="skip the per-workload lines (short_b8, full_b32, full_b128) of a 1-GPU run")
     ap.add_argument("--profile-steps", type=int, default=3)
     # solver / convention variant (pi0x_set_variant); the default is pi0's own loop
     ap.add_argument("--time-grid", default="pi0", choices=["pi0", "linspace"])
@@ -232,6 +345,12 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if args.gpus != world:
+        print(f"bench.py: --gpus {args.gpus} needs {args.gpus} ranks (WORLD_SIZE={world}); launch it with "
+              f"python -m torch.distributed.run --nproc-per-node {args.gpus} bench.py --gpus {args.gpus}",
+              file=sys.stderr)
+        return 2
     wl = synth.WORKLOADS[args.workload]
     if args.impl == "reference":
         return run_reference(args, wl)
@@ -239,7 +358,6 @@ def main():
     import torch
     from vla_flow_matching_b200 import build, pi0x
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     torch.cuda.set_device(local)
@@ -255,45 +373,21 @@ def main():
         dist.barrier()
 
     precision = pi0x.PI0X_BF16 if args.precision == "bf16" else pi0x.PI0X_FP32
+    variant = (pi0x.PI0X_TIME_LINSPACE if args.time_grid == "linspace" else pi0x.PI0X_TIME_PI0,
+               args.x_prediction, args.causal_actions)
+
+    def sampler_for(w, inp):
+        s = pi0x.Sampler(w.dims, inp.weights, precision)
+        s.set_variant(*variant)
+        return s
+
     inp = synth.make_inputs(wl)
-    sampler = pi0x.Sampler(wl.dims, inp.weights, precision)
-    sampler.set_variant(pi0x.PI0X_TIME_LINSPACE if args.time_grid == "linspace" else pi0x.PI0X_TIME_PI0,
-                        args.x_prediction, args.causal_actions)
-    dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()
-    pk = [dev(k.view(np.int16)) for k in inp.prefix_k]
-    pv = [dev(v.view(np.int16)) for v in inp.prefix_v]
-    mask, state, x1 = dev(inp.mask), dev(inp.state), dev(inp.x1)
-    x0 = torch.empty_like(x1)
-    stream = torch.cuda.current_stream()
-    sid = stream.cuda_stream
+    sampler = sampler_for(wl, inp)
     B, N = wl.batch, wl.num_steps
-
-    def call():
-        sampler.sample(pk, pv, mask, state, x1, N, x0=x0, stream=sid)
-
-    for _ in range(args.warmup):
-        call()
-    sampler.sync()
-
-    # ---- timed region: K whole calls, device-timed, max over ranks ----
-    clk = sample_clocks_start() if rank == 0 else None
-    time.sleep(0.3 if clk else 0)
-    torch.cuda.synchronize()
-    if dist is not None:
-        dist.barrier()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(args.steps):
-        call()
-    e1.record(stream)
-    torch.cuda.synchronize()
-    if dist is not None:
-        dist.barrier()
-    clocks = sample_clocks_stop(clk, local) if clk else None
-    sampler.sync()
-    ms = slowest_rank_ms(e0.elapsed_time(e1), dist)
-    ms_per = ms / args.steps
-    value = job_throughput(world, B, args.steps, ms)
+    r = measure(wl, args, sampler, inp, rank, dist, clocks_on=True)
+    ms, steps = r["ms"], r["steps"]
+    ms_per = ms / steps
+    value = job_throughput(world, B, steps, ms)
     if rank == 0:
         print(f"[bench] {wl.name} {args.precision}: {1000 * ms_per:.1f} us per call, "
               f"{value:.1f} {UNIT}", file=sys.stderr, flush=True)
@@ -306,12 +400,15 @@ def main():
     hx0 = torch.empty(inp.x1.shape, dtype=torch.float32).pin_memory()
     h2d = sum(t.numel() * t.element_size() for t in hk + hv + [hm, hs, hx])
     d2h = hx0.numel() * 4
+    sid = r["tensors"][-1]
+    stream = torch.cuda.current_stream()
     e2e_steps = max(3, min(args.steps, 50))
     for _ in range(3):
         sampler.sample(hk, hv, hm, hs, hx, N, x0=hx0, stream=sid)
     torch.cuda.synchronize()
     if dist is not None:
         dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(e2e_steps):
         sampler.sample(hk, hv, hm, hs, hx, N, x0=hx0, stream=sid)
@@ -319,47 +416,38 @@ def main():
     torch.cuda.synchronize()
     e2e_ms = slowest_rank_ms(e0.elapsed_time(e1), dist)
     e2e_value = job_throughput(world, B, e2e_steps, e2e_ms)
-
-    # ---- per-kernel device time from the profiling graph (same workload) ----
-    sampler.profile(True)
-    acc = {}
-    for _ in range(max(1, args.profile_steps)):
-        call()
-        for kname, (n, t) in sampler.profile_read().items():
-            a = acc.setdefault(kname, [0, 0.0])
-            a[0] += n
-            a[1] += t
-    sampler.profile(False)
     sampler.sync()
     if rank == 0:
         print("[bench] per-call kernel ms (launches): " + ", ".join(
-            f"{k}={v[1] / max(1, args.profile_steps):.3f} ({v[0] // max(1, args.profile_steps)})"
-            for k, v in acc.items()), file=sys.stderr, flush=True)
+            f"{k}={v:.3f} ({r['launches'][k]})" for k, v in r["kernel_ms"].items()), file=sys.stderr, flush=True)
+    launches_per_call = sampler.launch_count(B, wl.prefix_len, N)
+    roof = roofline_of(wl, r["kernel_ms"], ms_per) if rank == 0 else None
+    clocks = r["clocks"]
+    del r
+    sampler.close()
 
-    roofline = None
-    kernel_ms = {}
-    if rank == 0:
-        pk_, src = peaks()
-        byt, flo, att = algorithmic_work(wl)
-        n_g, t_g = acc["gemm"]
-        t_g_per_call = t_g / max(1, args.profile_steps)
-        kernel_ms = {k: round(v[1] / max(1, args.profile_steps), 4) for k, v in acc.items()}
-        ridge = pk_["bf16_tflops"] * 1e12 / (pk_["hbm_gbs"] * 1e9)
-        if flo / byt < ridge:
-            achieved = byt / (t_g_per_call / 1000) / 1e9
-            roofline = {"kernel": "k_gemm_tc (all expert and time-MLP Linears)", "bound": "hbm",
-                        "achieved": achieved, "peak": pk_["hbm_gbs"], "unit": "GB/s",
-                        "frac": achieved / pk_["hbm_gbs"], "traffic": None,
-                        "peak_source": f"{src} hbm_gbs"}
-        else:
-            achieved = flo / (t_g_per_call / 1000) / 1e12
-            peak = pk_.get("bf16_tflops_sustained", pk_["bf16_tflops"])
-            roofline = {"kernel": "k_gemm_tc (all expert and time-MLP Linears)", "bound": "tensor",
-                        "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                        "frac": achieved / peak, "traffic": None,
-                        "peak_source": f"{src} bf16_tflops_sustained"}
-        roofline["launches_per_call"] = n_g // max(1, args.profile_steps)
-        roofline["algorithmic_per_call"] = {"gemm_bytes": byt, "gemm_flops": flo, "attn_flops": att}
+    # ---- the other workloads of the metric (B = 8, 32, 128), device-timed, 1 GPU ----
+    by_workload = {}
+    if world == 1 and not args.no_by_workload and args.workload == "full_b1":
+        for name in ("short_b8", "full_b32", "full_b128"):
+            w2 = synth.WORKLOADS[name]
+            inp2 = synth.make_inputs(w2)
+            s2 = sampler_for(w2, inp2)
+            r2 = measure(w2, args, s2, inp2, rank, None, clocks_on=True)
+            mp = r2["ms"] / r2["steps"]
+            by_workload[name] = {
+                "batch": w2.batch, "prefix_len": w2.prefix_len, "num_steps": w2.num_steps,
+                "horizon": w2.dims.horizon, "value": w2.batch * r2["steps"] / (r2["ms"] / 1000.0), "unit": UNIT,
+                "ms_per_step": mp, "us_per_chunk": 1000 * mp, "steps": r2["steps"],
+                "gpu_launches": s2.launch_count(w2.batch, w2.prefix_len, w2.num_steps) * r2["steps"],
+                "clocks": r2["clocks"], "roofline": roofline_of(w2, r2["kernel_ms"], mp),
+                "profiled_kernel_ms_per_call": {k: round(v, 4) for k, v in r2["kernel_ms"].items()},
+            }
+            print(f"[bench] {name}: {1000 * mp:.1f} us per call, "
+                  f"{by_workload[name]['value']:.1f} {UNIT}", file=sys.stderr, flush=True)
+            del r2, inp2
+            s2.close()
+            torch.cuda.empty_cache()
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -368,21 +456,20 @@ def main():
 
     if rank == 0:
         line = {
-            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": steps,
             "warmup": args.warmup, "ms_per_step": ms_per, "us_per_chunk": 1000 * ms_per,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": args.precision, "data": "synthetic (seeded numpy PCG64, bf16-rounded N(0,0.02) "
                                                "weights, N(0,1) prefix K/V, state, noise)",
             "config": dict(config_of(wl, args), parallelism=f"replicas x{world} (batch per GPU fixed)"),
             "parallelism": f"replicas x{world} (batch per GPU fixed)",
-            "gpu_launches": sampler.launch_count(B, wl.prefix_len, N) * args.steps,
+            "gpu_launches": launches_per_call * steps,
             "clocks": clocks,
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "steps": e2e_steps},
-            "roofline": roofline, "kernel_ms_per_call": kernel_ms, "cpu_baseline": cpu,
+            "roofline": roof, "cpu_baseline": cpu, "by_workload": by_workload or None,
         }
         print(json.dumps(line), flush=True)
-    sampler.close()
     if dist is not None:
         dist.barrier()
         dist.destroy_process_group()

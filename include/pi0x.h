@@ -153,7 +153,10 @@ enum {
 int pi0x_set_variant(pi0x_handle *h, int time_grid, int x_prediction, int causal_actions);
 
 /* Number of kernels one pi0x_sample(B, P, num_steps) call launches (its own
- * kernels only, not memory copies), or -1 for invalid arguments. */
+ * kernels only, not memory copies), or -1 for invalid arguments.  In bf16 mode a
+ * batch whose rows fit one 128-row tile (B * (horizon + 1) <= 128) runs every
+ * Euler step in one persistent kernel after five small set-up kernels; larger
+ * batches run one kernel per projection, attention and small step. */
 long pi0x_launch_count(const pi0x_handle *h, int B, int P, int num_steps);
 
 /* ---- per-kernel-class device timing ------------------------------------------
@@ -172,7 +175,8 @@ enum {
   PI0X_K_ATTN = 5,   /* masked MQA attention */
   PI0X_K_GEGLU = 6,  /* gated GELU(tanh) */
   PI0X_K_FINAL = 7,  /* final norm + action out-proj + Euler update */
-  PI0X_K_COUNT = 8
+  PI0X_K_LOOP = 8,   /* the persistent small-batch loop kernel (every step of a call) */
+  PI0X_K_COUNT = 9
 };
 int pi0x_profile_enable(pi0x_handle *h, int on);
 int pi0x_profile_read(pi0x_handle *h, int kclass, long *launches, double *total_ms);

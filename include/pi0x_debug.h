@@ -6,6 +6,8 @@
 #ifndef PI0X_DEBUG_H
 #define PI0X_DEBUG_H
 
+#include "pi0x.h"
+
 #ifdef __cplusplus
 extern "C" {
 #endif
@@ -37,27 +39,53 @@ int pi0x_debug_attention(const void *q, const void *ks, const void *vs, const vo
 
 /* The same attention as pi0x_debug_attention with impl 1 (tcgen05, split-KV as the
  * sampler chooses), for callers that cannot allocate device memory while they run
- * — e.g. a robot control loop that must never stall in cudaMalloc, or an
- * application whose device memory is owned by its own pool.  It calls no
- * cudaMalloc/cudaFree and no allocating library routine: all its scratch (a call
- * table, an error word, the valid-prefix index list and the split-KV partials)
- * lives in one static device array of 32 MiB inside libpi0x, which every GPU that
- * loads the library holds until the process exits.  The pages have no counterpart
- * to this entry point; it is a deployment variant of the `_attend` step.
+ * — e.g. a robot control loop that must never stall in cudaMalloc (it can block
+ * for milliseconds and synchronises the device), or an application whose device
+ * memory is owned by its own pool.  It calls no cudaMalloc/cudaFree and no
+ * allocating library routine: all its scratch (a call table, an error word, the
+ * valid-prefix index list and the split-KV partials) lives in one static device
+ * array of 32 MiB inside libpi0x, which every GPU that loads the library holds
+ * until the process exits.  The paper has no counterpart to this entry point.
  *
  * Arguments as for pi0x_debug_attention.  Returns PI0X_EINVAL when the problem's
- * scratch (4 B per prefix position per sample plus the split-KV partials,
- * 4 B x 258 per query row per split, at most 32.1 MB) does not fit in the 32 MiB;
- * the pi0 workloads up to B = 8 fit.  The first call on each device looks up the device
- * address of the array (cudaGetSymbolAddress, with that device current); make that
- * first call before any stream capture.  Every call clears the error word it uses;
- * the array keeps the contents of the last call.  All calls share the one array,
- * so calls that overlap on the GPU (other streams, other host threads) race.
- * Synchronous: returns after `stream` has finished the work, with PI0X_ETIMEOUT if
- * a bounded device wait gave up. */
+ * scratch does not fit in the 32 MiB: 4 B per prefix position per sample for the
+ * index list, plus the split-KV partials (4 B x 258 per query row per split; split-KV
+ * is used only for fewer than 96 row tiles and keeps tiles x splits <= 219, i.e.
+ * at most 28.9 MB); the pi0 workloads up to B = 8 fit.  The first call on each
+ * device looks up the device address of the array (cudaGetSymbolAddress, with that
+ * device current).  Every call clears the error word it uses; the array keeps the
+ * contents of the last call.  All calls share the one array, so calls that overlap
+ * on the GPU (other streams, other host threads) race.  Synchronous: it waits for
+ * `stream` and copies the error word to the host, so it cannot be captured into a
+ * CUDA graph.  Returns PI0X_ETIMEOUT if a bounded device wait gave up, PI0X_ECUDA
+ * for a CUDA error (text in pi0x_last_error). */
 int pi0x_attention_noalloc(const void *q, const void *ks, const void *vs, const void *prefix_k,
                            const void *prefix_v, const void *mask, int B, int H, int P, int step0, void *out,
                            void *stream);
+
+/* 1 if pi0x_sample(h, B, ...) runs the persistent small-batch loop kernel (bf16
+ * mode, B * (horizon + 1) <= 128, a device that can co-schedule one CTA per SM),
+ * else 0 (also for a NULL handle). */
+int pi0x_uses_loop(const pi0x_handle *h, int B);
+
+/* enable = 0: later pi0x_sample calls on `h` run every batch on the multi-kernel
+ * path (one kernel per projection, attention and small step), so that tests can
+ * compare it with the persistent loop at the same small batch; enable = 1 (the
+ * default) restores the choice pi0x_uses_loop describes.  Waits for the handle's
+ * last call and drops its cached graphs.  PI0X_EINVAL for a NULL handle or another
+ * value. */
+int pi0x_debug_set_loop(pi0x_handle *h, int enable);
+
+/* Failure-path test hook of the persistent loop.  The next pi0x_sample call on `h`
+ * that runs the loop kernel makes stage `stage` of the call (0 = the first stage of
+ * Euler step 0; a GEMM stage is needed to take effect) wait on a done-counter that
+ * nothing raises, with every wait of that call bounded by `wait_ns` nanoseconds
+ * instead of the default 200 ms.  The wait gives up, the kernel's other waits see
+ * the error word and return, and pi0x_sync_status then reports PI0X_ETIMEOUT; the
+ * call's x0 is invalid.  Later calls run normally (every call starts from zeroed
+ * counters).  Returns PI0X_EINVAL for a NULL handle, a negative stage or a zero
+ * limit. */
+int pi0x_debug_loop_stall(pi0x_handle *h, int stage, unsigned long long wait_ns);
 
 #ifdef __cplusplus
 }

@@ -81,8 +81,9 @@ def test_tiny_workload_variants(name, precision):
 
 # Full size in bf16: the combinations whose x_0 is the noise plus the integrated
 # velocity, like the pi0 loop's.  With x-prediction on the 0 -> 1 grid x_0 is the
-# network's own last prediction, so the relative L2 measures the bf16 network error
-# itself (1.4 % on full_b1, max|dx0| 0.009): that combination is held to the fp32 bar.
+# average of the network's predictions, so the relative L2 measures the bf16 network
+# error itself (1.4 % on full_b1, max|dx0| 0.009): that combination is held to the
+# fp32 bar in fp32 mode and to max|dx0| (2 % relative guard) in bf16 below.
 BF16_FULL = {
     "full_b1": dict(time_convention="linspace", causal_actions=True),
     "short_b8": dict(x_prediction=True, causal_actions=True),
@@ -106,9 +107,25 @@ def test_full_size_all_variants_fp32():
     s.close()
 
 
+def test_x_prediction_linspace_full_b1_fp32():
+    """Linspace grid + x-prediction + causal mask at full_b1 in fp32 mode, held to the
+    fp32 bar.  Same kernels and control flow as the bf16 run below, so a pass here
+    says the bf16 relative-L2 excess is bf16 rounding of the network, not a logic error."""
+    wl = synth.WORKLOADS["full_b1"]
+    inp = synth.make_inputs(wl)
+    s = _sampler(wl, 1, VARIANTS["all"])
+    check(run_gpu(s, inp), _oracle(inp, VARIANTS["all"]), 1, "full_b1 all variants")
+    s.close()
+
+
 def test_x_prediction_linspace_full_b1_bf16_max_error():
     """The x-prediction / 0 -> 1 combination at full size in bf16, held to the max|dx0|
-    bar; its relative L2 is reported by the assertion message when it grows."""
+    bar with a 2 % relative-L2 guard: with x-prediction on the 0 -> 1 grid the noise
+    cancels (the step sizes sum to 1), so x_0 is the average of the network's
+    predictions rather than the noise plus a small correction, and its relative L2
+    measures the bf16 error of the network itself (1.4 % measured).
+    The fp32 run of the same combination above meets the 1e-4 bar, which rules out a
+    logic error."""
     wl = synth.WORKLOADS["full_b1"]
     inp = synth.make_inputs(wl)
     s = _sampler(wl, 0, VARIANTS["all"])

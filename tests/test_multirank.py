@@ -71,3 +71,17 @@ def test_reference_arm_other_ranks_exit_without_work(monkeypatch, capsys):
                               causal_actions=False, precision="bf16")
     assert bench.run_reference(args, synth.WORKLOADS["tiny"]) == 0
     assert capsys.readouterr().out == ""
+
+
+def test_bench_refuses_a_gpu_count_without_that_many_ranks():
+    """`bench.py --gpus N` must run as N ranks; run alone it exits non-zero
+    instead of timing one GPU under an N-GPU label."""
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = dict(os.environ)
+    env.pop("WORLD_SIZE", None)
+    r = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--gpus", "4", "--steps", "1",
+                        "--warmup", "3"], capture_output=True, text=True, env=env, timeout=120)
+    assert r.returncode != 0 and "--nproc-per-node 4" in r.stderr
+    assert r.stdout.strip() == ""

@@ -130,6 +130,72 @@ def test_rope_matches_transformers():
     assert np.allclose(qo[:, :2], qt[0].numpy()[:, :2], atol=1e-6)
 
 
+# --- bf16 widening of weights and prefix K/V -------------------------------------
+def _torch_bf16_to_f32(bits: np.ndarray) -> np.ndarray:
+    """torch's own bf16 -> float32 conversion of uint16 bit patterns."""
+    return torch.from_numpy(bits.view(np.int16).copy()).view(torch.bfloat16).float().numpy()
+
+
+def _widening_agrees_with_torch(widen) -> bool:
+    """Every one of the 65536 bf16 bit patterns widens to torch's float32 value,
+    bit for bit (so +0 / -0, subnormals and infinities too); NaN patterns stay NaN."""
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    ref = _torch_bf16_to_f32(bits)
+    with np.errstate(invalid="ignore"):   # signalling-NaN patterns
+        got = np.asarray(widen(bits, np.float32))
+        wide = np.asarray(widen(bits, np.float64))
+    if got.dtype != np.float32 or got.shape != ref.shape:
+        return False
+    nan = np.isnan(ref)
+    if not np.array_equal(np.isnan(got), nan):
+        return False
+    if not np.array_equal(got[~nan].view(np.uint32), ref[~nan].view(np.uint32)):
+        return False
+    return wide.dtype == np.float64 and np.array_equal(wide[~nan], ref[~nan].astype(np.float64))
+
+
+def test_bf16_widening_matches_torch_on_every_bit_pattern():
+    # the vllm-omni page casts the bf16 prefix cache to the expert's dtype before the
+    # attention (`_compute_layer_suffix_only`); weights enter the float32 model the same way
+    assert _widening_agrees_with_torch(O.as_float)
+    f = np.array([1.5, -2.25], np.float32)
+    assert O.as_float(f, np.float64).dtype == np.float64 and np.array_equal(O.as_float(f, np.float32), f)
+
+
+@pytest.mark.parametrize("mutant", ["int16_value", "no_shift", "shift_15", "byteswap"])
+def test_bf16_widening_pin_catches_planted_mistakes(mutant):
+    """Plausible widening mistakes, each of which the pin above must reject."""
+    def int16_value(a, dtype):          # sign-extending int16 view taken as a number
+        return np.asarray(a).view(np.int16).astype(dtype)
+
+    def no_shift(a, dtype):             # bits placed in the low half of the float32
+        return np.asarray(a).astype(np.uint32).view(np.float32).astype(dtype)
+
+    def shift_15(a, dtype):
+        return (np.asarray(a).astype(np.uint32) << np.uint32(15)).view(np.float32).astype(dtype)
+
+    def byteswap(a, dtype):
+        return (np.asarray(a).byteswap().astype(np.uint32) << np.uint32(16)).view(np.float32).astype(dtype)
+
+    fn = {"int16_value": int16_value, "no_shift": no_shift, "shift_15": shift_15, "byteswap": byteswap}[mutant]
+    assert not _widening_agrees_with_torch(fn)
+
+
+def test_convert_weights_widens_every_array():
+    dims = dataclasses.replace(synth.ExpertDims(), depth=2)
+    w = synth.make_weights(dims, seed=5)
+    for dtype in (np.float32, np.float64):
+        c = O.convert_weights(w, dtype)
+        assert set(c) == set(w)
+        assert len(c["layers"]) == len(w["layers"])
+        pairs = [(c[k], w[k]) for k in w if k != "layers"]
+        pairs += [(cl[k], wl[k]) for cl, wl in zip(c["layers"], w["layers"]) for k in wl]
+        assert len(pairs) == len(synth.WEIGHT_ORDER + synth.TAIL_ORDER) + 2 * len(synth.LAYER_ORDER)
+        for got, bits in pairs:
+            assert bits.dtype == np.uint16 and got.dtype == dtype and got.shape == bits.shape
+            assert np.array_equal(got, _torch_bf16_to_f32(bits).astype(dtype))
+
+
 # --- RMSNorm, activations ----------------------------------------------------------
 def test_rms_norm_unit_rms_and_gain():
     rng = np.random.default_rng(3)

@@ -27,6 +27,7 @@ enum : unsigned {
   kErrTimeoutMma = 1u << 1,
   kErrTimeoutEpilogue = 1u << 2,
   kErrBadLaunch = 1u << 3,
+  kErrTimeoutFlag = 1u << 4,   // a wait on another CTA's done-counter
 };
 
 constexpr unsigned long long kWaitLimitNs = 200000000ull;  // 200 ms

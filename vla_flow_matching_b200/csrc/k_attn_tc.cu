@@ -554,6 +554,17 @@ bool attn_tc_maps(CallPtrs &cp, int layers, int B, int P, const void *ks, const 
   return true;
 }
 
+bool loop_attn_maps(CallPtrs &cp, int layers, int B, int P, const void *ks, const void *vs, uint64_t sfx_rows) {
+  for (int l = 0; l < layers && P > 0; ++l)
+    for (int kv = 0; kv < 2; ++kv) {
+      const void *base = kv ? cp.prefix_v[l] : cp.prefix_k[l];
+      if (!make_map(&cp.kv_map32[kv][l], base, (uint64_t)B * P, kHeadDim, kHeadDim, 32)) return false;
+    }
+  for (int kv = 0; kv < 2; ++kv)
+    if (!make_map(&cp.sfx_map32[kv], kv ? vs : ks, sfx_rows, kHeadDim, kHeadDim, 32)) return false;
+  return true;
+}
+
 void launch_attention_tc(const bf16 *q, const bf16 *ks, const bf16 *vs, const CallPtrs *cp, int layer,
                          int sfx_row0, const int *nvalid, const int *vidx, const Geo &g, int step0, int causal,
                          int splits, bf16 *out, float *part, unsigned *err, cudaStream_t s) {

@@ -92,7 +92,7 @@ void launch_time_vec(const TW *w_time, const float *bias, int num_steps, int lin
 template <typename TW>
 __global__ void __launch_bounds__(256) k_state_embed(const CallPtrs *cp, const TW *w, const float *bias, int S,
                                                       float *h, const float *gain, bf16 *xn, float *ss,
-                                                      int ss_ld) {
+                                                      int ss_ld, int nslots) {
   pdl_wait();
   pdl_trigger();
   __shared__ float sv[64];
@@ -115,19 +115,19 @@ __global__ void __launch_bounds__(256) k_state_embed(const CallPtrs *cp, const T
     ssq = warp_sum(ssq);
     if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ssq;
     __syncthreads();
-    if (threadIdx.x < kNormSlots) {
+    for (int t = threadIdx.x; t < nslots; t += blockDim.x) {
       float tot = 0.f;
-      if (threadIdx.x == 0)
+      if (t == 0)
         for (int i = 0; i < 8; ++i) tot += red[i];
-      ss[(size_t)threadIdx.x * ss_ld + b] = tot;
+      ss[(size_t)t * ss_ld + b] = tot;
     }
   }
 }
 
 template <typename TW>
 void launch_state_embed(const CallPtrs *cp, const TW *w, const float *b, int B, int S, float *h, cudaStream_t s,
-                        const float *gain, bf16 *xn, float *ss, int ss_ld) {
-  launch_pdl(k_state_embed<TW>, B, 256, 0, s, cp, w, b, S, h, gain, xn, ss, ss_ld);
+                        const float *gain, bf16 *xn, float *ss, int ss_ld, int nslots) {
+  launch_pdl(k_state_embed<TW>, B, 256, 0, s, cp, w, b, S, h, gain, xn, ss, ss_ld, nslots);
 }
 
 // Action tokens: out[i] = action_in_proj(x[i]) for every (sample, horizon) row.
@@ -405,9 +405,9 @@ void launch_delay_ns(unsigned long long ns, cudaStream_t s) { k_delay<<<1, 1, 0,
 template void launch_time_vec<float>(const float *, const float *, int, int, float *, cudaStream_t);
 template void launch_time_vec<bf16>(const bf16 *, const float *, int, int, float *, cudaStream_t);
 template void launch_state_embed<float>(const CallPtrs *, const float *, const float *, int, int, float *,
-                                        cudaStream_t, const float *, bf16 *, float *, int);
+                                        cudaStream_t, const float *, bf16 *, float *, int, int);
 template void launch_state_embed<bf16>(const CallPtrs *, const bf16 *, const float *, int, int, float *,
-                                       cudaStream_t, const float *, bf16 *, float *, int);
+                                       cudaStream_t, const float *, bf16 *, float *, int, int);
 template void launch_action_in<float, float>(const float *, const float *, const float *, int, int, float *,
                                              cudaStream_t);
 template void launch_action_in<bf16, bf16>(const float *, const bf16 *, const float *, int, int, bf16 *,

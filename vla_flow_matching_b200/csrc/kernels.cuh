@@ -29,6 +29,9 @@ struct CallPtrs {
   CUtensorMap kv_map64[2][kMaxDepth];
   CUtensorMap sfx_map[2];
   CUtensorMap sfx_map64[2];
+  // 32-row boxes of the same tensors (the persistent small-batch loop's 32-key blocks)
+  CUtensorMap kv_map32[2][kMaxDepth];
+  CUtensorMap sfx_map32[2];
   const bf16 *prefix_k[kMaxDepth];
   const bf16 *prefix_v[kMaxDepth];
   const uint8_t *mask;
@@ -129,7 +132,8 @@ template <typename TW>
 void launch_time_vec(const TW *w_time, const float *bias, int num_steps, int linspace, float *tvec, cudaStream_t s);
 template <typename TW>
 void launch_state_embed(const CallPtrs *cp, const TW *w, const float *b, int B, int S, float *h, cudaStream_t s,
-                        const float *gain = nullptr, bf16 *xn = nullptr, float *ss = nullptr, int ss_ld = 0);
+                        const float *gain = nullptr, bf16 *xn = nullptr, float *ss = nullptr, int ss_ld = 0,
+                        int nslots = kNormSlots);
 template <typename TW, typename T>
 void launch_action_in(const float *x, const TW *w, const float *b, int rows, int A, T *out, cudaStream_t s);
 template <typename T>
@@ -162,6 +166,8 @@ size_t attn_tc_partial_floats(const Geo &g, int step0, int splits);
 // and cp.sfx_map over `sfx_rows` rows at ks / vs.  False if an encode fails (e.g. a
 // pointer that is not 16-byte aligned).
 bool attn_tc_maps(CallPtrs &cp, int layers, int B, int P, const void *ks, const void *vs, uint64_t sfx_rows);
+// The 32-row-box maps (kv_map32, sfx_map32) of the same tensors.
+bool loop_attn_maps(CallPtrs &cp, int layers, int B, int P, const void *ks, const void *vs, uint64_t sfx_rows);
 // ks / vs: this layer's suffix rows, which start at row `sfx_row0` of cp->sfx_map.
 // causal: the causal action mask (action query i sees actions 0..i and the state).
 void launch_attention_tc(const bf16 *q, const bf16 *ks, const bf16 *vs, const CallPtrs *cp, int layer,
@@ -180,6 +186,7 @@ void launch_gemm_simt(const float *A, int lda, const float *Bw, int ldb, int M, 
 // Weight operand of a tcgen05 GEMM: tensor maps with 64-row and wide boxes.
 struct TcWeight {
   CUtensorMap tm64, tm_wide;
+  CUtensorMap tm16;  // 64 x 16 boxes (the persistent small-batch loop)
   int N = 0, K = 0, bn_wide = 128;
   const CUtensorMap &map(int bn) const { return bn == 64 ? tm64 : tm_wide; }
 };
@@ -188,5 +195,109 @@ TcPlan plan_gemm_tc(int M, int N, int K);
 size_t gemm_tc_partial_floats(int M, int N, const TcPlan &p);
 void launch_gemm_tc(int epi, const CUtensorMap &tmA, const CUtensorMap &tmB, const TcPlan &p, int a_row0, int M,
                     int N, int K, const EpiArgs &e, unsigned *err, cudaStream_t s);
+
+// ---- persistent small-batch loop (k_loop.cu) -----------------------------------
+// One cooperative launch runs every Euler step of a call when every step's rows fit
+// one 128-row MMA tile (B * (H + 1) <= 128): one CTA per SM, the steps' stages in
+// program order, each stage waiting on the done-counter of the one before it.
+//
+// Stages of one Euler step (index i within the step):
+//   0 ACTION_IN, 1 TIN (action-time MLP in + SiLU), 2 TOUT (MLP out -> h, layer-0 norm
+//   inputs), then per layer QKV, ATTN, [COMBINE when attention is split], O, GU, DOWN,
+//   and last EULER (final norm, out-projection, x += dt v).
+enum LoopKind : int {
+  LK_ACTION_IN = 0, LK_TIN = 1, LK_TOUT = 2, LK_QKV = 3, LK_ATTN = 4, LK_COMBINE = 5,
+  LK_O = 6, LK_GU = 7, LK_DOWN = 8, LK_EULER = 9
+};
+constexpr int kLoopMaxRows = 128;
+constexpr int kLoopNormSlots = 64;   // fused-norm partial sums: one slot per 16-column group
+constexpr int kLoopKeyBlock = 32;    // attention key block of the loop kernel
+constexpr int kLoopMinGrid = 128;    // GEMM units stay <= 64 columns wide
+
+__host__ __device__ inline int loop_layer_stages(int attn_splits) { return attn_splits > 1 ? 6 : 5; }
+__host__ __device__ inline int loop_stages_per_step(int L, int attn_splits) {
+  return 3 + L * loop_layer_stages(attn_splits) + 1;
+}
+// Kind and layer of stage i of a step.
+__host__ __device__ inline void loop_stage(int i, int L, int attn_splits, int &kind, int &layer) {
+  layer = 0;
+  if (i < 3) {
+    kind = i;
+    return;
+  }
+  const int ls = loop_layer_stages(attn_splits);
+  const int j = i - 3;
+  if (j >= L * ls) {
+    kind = LK_EULER;
+    layer = L - 1;
+    return;
+  }
+  layer = j / ls;
+  int sub = j % ls;
+  if (ls == 5 && sub >= 2) ++sub;  // no COMBINE stage
+  switch (sub) {
+    case 0: kind = LK_QKV; break;
+    case 1: kind = LK_ATTN; break;
+    case 2: kind = LK_COMBINE; break;
+    case 3: kind = LK_O; break;
+    case 4: kind = LK_GU; break;
+    default: kind = LK_DOWN; break;
+  }
+}
+
+// GEMM stage plan: N columns in 16-column groups, split over `nchunks` contiguous
+// chunks (<= 64 columns each) and `splits` equal K ranges; unit u = chunk * splits + split.
+struct LoopGemm {
+  int N, K, splits, nchunks;
+};
+__host__ __device__ inline LoopGemm loop_gemm_plan(int kind, int grid) {
+  LoopGemm p{1024, 1024, 1, 1};
+  switch (kind) {
+    case LK_QKV: p.N = kQkvDim; break;
+    case LK_O: p.K = kQDim; p.splits = 2; break;
+    case LK_GU: p.N = 2 * kMlp; break;
+    case LK_DOWN: p.K = kMlp; p.splits = 4; break;
+    default: break;
+  }
+  const int G = p.N / 16, per = grid / p.splits;
+  p.nchunks = G < per ? G : per;
+  return p;
+}
+__host__ __device__ inline bool loop_is_gemm(int kind) {
+  return kind == LK_TIN || kind == LK_TOUT || kind == LK_QKV || kind == LK_O || kind == LK_GU || kind == LK_DOWN;
+}
+
+struct LoopArgs {
+  int B, H, A, S, P, R, L, N;
+  int linspace, x_pred, causal;
+  int grid;
+  int attn_splits, attn_bps;   // split-KV: splits per query tile, 32-key blocks per split
+  int box_rows;                // activation TMA box rows (64 or 128)
+  int ss_ld;
+  int debug_stall_stage;       // >= 0: that stage waits on a counter nothing raises (tests)
+  unsigned long long wait_ns;  // time limit of every wait
+  float *h, *ss_a, *ss_m, *gpart, *tvec, *xw, *part_o, *part_ml;
+  bf16 *xn, *q, *ks, *vs, *att, *act, *aemb, *uemb;
+  int *counters, *done;
+  const int *nvalid, *vidx;
+  const float *rope_tab;
+  const CallPtrs *cp;
+  unsigned *err;
+  const bf16 *ain_w;
+  const float *ain_b, *tout_b, *aout_w, *aout_b, *fnorm;
+  const float *in_norm[kMaxDepth], *post_norm[kMaxDepth];
+  // tensor maps in device memory: weights (64 x 16 boxes) and activations
+  const CUtensorMap *m_tin, *m_tout;
+  const CUtensorMap *m_qkv[kMaxDepth], *m_o[kMaxDepth], *m_gu[kMaxDepth], *m_down[kMaxDepth];
+  const CUtensorMap *m_xn, *m_att, *m_act, *m_aemb, *m_uemb;
+};
+
+// Split-KV plan of the loop attention (splits per query tile, key blocks per split).
+void loop_attn_plan(int B, int H, int P, int grid, int &splits, int &bps);
+size_t loop_smem_bytes();
+// CTAs of the loop kernel on `dev` (one per SM), or 0 if it cannot run there.
+int loop_max_grid(int dev);
+// Enqueue the loop kernel (cooperative launch) on `s`.
+cudaError_t launch_loop(const LoopArgs &a, cudaStream_t s);
 
 }  // namespace pi0x

@@ -26,8 +26,10 @@
 namespace pi0x {
 namespace {
 
-// 32 MiB: split-KV uses at most 243 row tiles x splits (attn_tc_splits), i.e. at most
-// 243 x 128 rows x 258 floats = 32.1 MB of partials, plus the valid-index list.
+// 32 MiB.  Split-KV runs only while row tiles x batch < 96 and then uses
+// ceil(148 / tiles) splits (attn_tc_splits), so tiles x splits <= 73 x 3 = 219 and the
+// partials take at most 219 x 128 rows x 258 floats = 28.9 MB; the valid-index list
+// (4 B per prefix position per sample) and the call table share the rest.
 constexpr size_t kScratchBytes = size_t(32) << 20;
 __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
 
@@ -128,8 +130,13 @@ extern "C" int pi0x_attention_noalloc(const void *q, const void *ks, const void 
   unsigned w = 0;
   if (e == cudaSuccess) e = cudaMemcpy(&w, d_err, sizeof(w), cudaMemcpyDeviceToHost);
   if (e != cudaSuccess) {
+    set_last_error((std::string("pi0x_attention_noalloc: ") + cudaGetErrorString(e)).c_str());
     cudaGetLastError();
     return e == cudaErrorMemoryAllocation ? PI0X_ENOMEM : PI0X_ECUDA;
   }
-  return w ? PI0X_ETIMEOUT : PI0X_OK;
+  if (w) {
+    set_last_error(("pi0x_attention_noalloc: device error word 0x" + std::to_string(w)).c_str());
+    return PI0X_ETIMEOUT;
+  }
+  return PI0X_OK;
 }

@@ -111,6 +111,11 @@ struct Workspace {
   int *counters; // split-K per-tile arrival counters
   float *ss_a, *ss_m;  // fused RMSNorm partial sums of squares, kNormSlots x ss_ld (bf16 mode)
   int ss_ld = 0;
+  // persistent small-batch loop (bf16 mode): 64-slot norm sums, stage done-counters,
+  // activation tensor maps in device memory ([i][0] = 64-row, [i][1] = 128-row boxes)
+  float *ss64_a = nullptr, *ss64_m = nullptr;
+  int *done = nullptr;
+  CUtensorMap *d_amaps = nullptr;
   float *rope_tab;     // (cos, sin) per position and pair (bf16 mode)
   void *xn, *q, *ks, *vs, *att, *act, *a_emb, *u_emb;
   // host-input staging (device side), allocated lazily
@@ -137,6 +142,14 @@ struct pi0x_handle {
   LayerW layer[kMaxDepth];
   // weight-side tensor maps + tile widths (bf16 mode)
   TcWeight g_tin, g_tout, g_qkv[kMaxDepth], g_o[kMaxDepth], g_gu[kMaxDepth], g_down[kMaxDepth];
+  // 16-row-box weight maps in device memory for the persistent loop: tin, tout, then
+  // per layer qkv, o, gu, down
+  CUtensorMap *d_wmaps = nullptr;
+  int loop_grid = 0;          // CTAs of the persistent loop (0: the loop cannot launch here)
+  bool loop_direct = false;   // the cooperative launch could not be captured: launch it directly
+  bool loop_off = false;      // pi0x_debug_set_loop(h, 0): small batches take the multi-kernel path
+  int dbg_stall = -1;         // next call's loop waits on a counter nothing raises at this stage
+  unsigned long long dbg_wait_ns = 0;
   Workspace ws;
   CallPtrs *d_ptrs = nullptr;
   unsigned *d_err = nullptr;
@@ -240,7 +253,8 @@ int build_weight_maps(pi0x_handle *h) {
     g.N = N;
     g.K = K;
     g.bn_wide = plan_gemm_tc(1 << 20, N, K).bn;
-    return make_map(&g.tm64, w, N, K, K, 64) && make_map(&g.tm_wide, w, N, K, K, g.bn_wide);
+    return make_map(&g.tm64, w, N, K, K, 64) && make_map(&g.tm_wide, w, N, K, K, g.bn_wide) &&
+           make_map(&g.tm16, w, N, K, K, 16);
   };
   bool ok = mk(h->g_tin, h->tin_a, kWidth, kWidth) && mk(h->g_tout, h->tout_w, kWidth, kWidth);
   for (int l = 0; l < L && ok; ++l) {
@@ -251,6 +265,17 @@ int build_weight_maps(pi0x_handle *h) {
     g_last_error = "cuTensorMapEncodeTiled failed for a weight operand";
     return PI0X_ECUDA;
   }
+  std::vector<CUtensorMap> maps;
+  maps.push_back(h->g_tin.tm16);
+  maps.push_back(h->g_tout.tm16);
+  for (int l = 0; l < L; ++l) {
+    maps.push_back(h->g_qkv[l].tm16);
+    maps.push_back(h->g_o[l].tm16);
+    maps.push_back(h->g_gu[l].tm16);
+    maps.push_back(h->g_down[l].tm16);
+  }
+  CK(cudaMalloc(&h->d_wmaps, maps.size() * sizeof(CUtensorMap)));
+  CK(cudaMemcpy(h->d_wmaps, maps.data(), maps.size() * sizeof(CUtensorMap), cudaMemcpyHostToDevice));
   return PI0X_OK;
 }
 
@@ -307,6 +332,13 @@ int ensure_workspace(pi0x_handle *h, int B, int P, int N) {
   // split-KV partials: splits*mtiles*B stays below 96 + 148 CTAs (attn_tc_splits)
   const size_t part_floats = h->bf16 ? (size_t)256 * 128 * (kHeadDim + 2) : 0;
   add(4 * part_floats);
+  // persistent loop: 64-slot norm sums (two sets), one done-counter per stage, maps
+  const size_t ss64_floats = h->bf16 ? (size_t)kLoopNormSlots * Rp : 0;
+  const size_t done_ints = h->bf16 ? (size_t)nN * loop_stages_per_step(L, 2) : 0;
+  add(4 * ss64_floats);
+  add(4 * ss64_floats);
+  add(4 * done_ints);
+  add(h->bf16 ? 10 * sizeof(CUtensorMap) : 0);
   void *base = nullptr;
   CK(cudaMalloc(&base, bytes));
   ws.arena.base = static_cast<uint8_t *>(base);
@@ -332,6 +364,10 @@ int ensure_workspace(pi0x_handle *h, int B, int P, int N) {
   ws.a_emb = ws.arena.take(es * Rp * kWidth);
   ws.u_emb = ws.arena.take(es * Rp * kWidth);
   ws.part = (float *)ws.arena.take(4 * part_floats);
+  ws.ss64_a = (float *)ws.arena.take(4 * ss64_floats);
+  ws.ss64_m = (float *)ws.arena.take(4 * ss64_floats);
+  ws.done = (int *)ws.arena.take(4 * done_ints);
+  ws.d_amaps = h->bf16 ? (CUtensorMap *)ws.arena.take(10 * sizeof(CUtensorMap)) : nullptr;
   CK(cudaMemset(base, 0, bytes));
   ws.B = nB;
   ws.P = nP;
@@ -347,6 +383,13 @@ int ensure_workspace(pi0x_handle *h, int B, int P, int N) {
       g_last_error = "cuTensorMapEncodeTiled failed for an activation operand";
       return PI0X_ECUDA;
     }
+    const ActMap *am[5] = {&ws.m_xn, &ws.m_att, &ws.m_act, &ws.m_aemb, &ws.m_uemb};
+    CUtensorMap dm[10];
+    for (int i = 0; i < 5; ++i) {
+      dm[2 * i] = am[i]->m64;
+      dm[2 * i + 1] = am[i]->m128;
+    }
+    CK(cudaMemcpy(ws.d_amaps, dm, sizeof(dm), cudaMemcpyHostToDevice));
   }
   return PI0X_OK;
 }
@@ -451,6 +494,9 @@ int enqueue_loop(pi0x_handle *h, int B, int P, int N, cudaStream_t s) {
     launch_gemm_tc(epi, am.get(p.a_rows), w.map(p.bn), p, a_row0, M, w.N, w.K, e, h->d_err, s);
   };
 
+  // Cross-CTA arrival counters start every call at zero, also after a call whose
+  // bounded waits gave up part-way (a memset node of the graph).
+  if (tc) CK(cudaMemsetAsync(ws.counters, 0, 4 * 1024, s));
   RUN(PI0X_K_PREP, launch_prep_mask(h->d_ptrs, B, P, ws.nvalid, ws.vidx, s));
   RUN(PI0X_K_PREP, launch_time_vec<T>((const T *)h->tin_t, h->tin_b, N, linspace ? 1 : 0, ws.tvec, s));
   RUN(PI0X_K_PREP, launch_copy_x1(h->d_ptrs, BH * A, ws.xw, s));
@@ -573,6 +619,112 @@ int enqueue_loop(pi0x_handle *h, int B, int P, int N, cudaStream_t s) {
   return PI0X_OK;
 }
 
+// ---- the Euler loop of a small batch: one persistent kernel ------------------------
+bool use_loop(const pi0x_handle *h, int B) {
+  return h->bf16 && !h->loop_off && h->loop_grid >= kLoopMinGrid && (long)B * (h->cfg.horizon + 1) <= kLoopMaxRows;
+}
+
+int enqueue_persistent(pi0x_handle *h, int B, int P, int N, cudaStream_t s, int stall_stage,
+                       unsigned long long wait_ns) {
+  Marker mk{h, s};
+  if (h->prof_on) h->prof_marks.clear();
+  Workspace &ws = h->ws;
+  const pi0x_config &c = h->cfg;
+  const int H = c.horizon, L = c.depth, R = B + B * H;
+  int splits = 1, bps = 1;
+  loop_attn_plan(B, H, P, h->loop_grid, splits, bps);
+  const int qps0 = (kHeads * (H + 1) + 127) / 128;
+  const size_t units0 = (size_t)B * qps0 * splits;
+  if (units0 > 256) {
+    g_last_error = "persistent loop: too many attention units for the partial buffer";
+    return PI0X_EUNSUPPORTED;
+  }
+  const int spp = loop_stages_per_step(L, splits);
+  CK(cudaMemsetAsync(ws.counters, 0, 4 * 1024, s));
+  CK(cudaMemsetAsync(ws.done, 0, 4 * (size_t)N * spp, s));
+  RUN(PI0X_K_PREP, launch_prep_mask(h->d_ptrs, B, P, ws.nvalid, ws.vidx, s));
+  RUN(PI0X_K_PREP, launch_time_vec<bf16>((const bf16 *)h->tin_t, h->tin_b, N,
+                                         h->time_grid == PI0X_TIME_LINSPACE ? 1 : 0, ws.tvec, s));
+  RUN(PI0X_K_PREP, launch_copy_x1(h->d_ptrs, B * H * c.action_dim, ws.xw, s));
+  RUN(PI0X_K_PREP, launch_rope_table(h->inv_freq, P + H + 1, ws.rope_tab, s));
+  RUN(PI0X_K_EMBED, launch_state_embed<bf16>(h->d_ptrs, (const bf16 *)h->state_w, h->state_b, B, c.state_dim,
+                                             ws.h, s, h->layer[0].in_norm, (bf16 *)ws.xn, ws.ss64_a, ws.ss_ld,
+                                             kLoopNormSlots));
+  LoopArgs a;
+  memset(&a, 0, sizeof(a));
+  a.B = B;
+  a.H = H;
+  a.A = c.action_dim;
+  a.S = c.state_dim;
+  a.P = P;
+  a.R = R;
+  a.L = L;
+  a.N = N;
+  a.linspace = h->time_grid == PI0X_TIME_LINSPACE;
+  a.x_pred = h->x_pred;
+  a.causal = h->causal;
+  a.grid = h->loop_grid;
+  a.attn_splits = splits;
+  a.attn_bps = bps;
+  a.box_rows = R <= 64 ? 64 : 128;
+  a.ss_ld = ws.ss_ld;
+  a.debug_stall_stage = stall_stage;
+  a.wait_ns = wait_ns;
+  a.h = ws.h;
+  a.ss_a = ws.ss64_a;
+  a.ss_m = ws.ss64_m;
+  a.gpart = ws.gpart;
+  a.tvec = ws.tvec;
+  a.xw = ws.xw;
+  a.part_o = ws.part;
+  a.part_ml = ws.part + units0 * 128 * kHeadDim;
+  a.xn = (bf16 *)ws.xn;
+  a.q = (bf16 *)ws.q;
+  a.ks = (bf16 *)ws.ks;
+  a.vs = (bf16 *)ws.vs;
+  a.att = (bf16 *)ws.att;
+  a.act = (bf16 *)ws.act;
+  a.aemb = (bf16 *)ws.a_emb;
+  a.uemb = (bf16 *)ws.u_emb;
+  a.counters = ws.counters;
+  a.done = ws.done;
+  a.nvalid = ws.nvalid;
+  a.vidx = ws.vidx;
+  a.rope_tab = ws.rope_tab;
+  a.cp = h->d_ptrs;
+  a.err = h->d_err;
+  a.ain_w = (const bf16 *)h->ain_w;
+  a.ain_b = h->ain_b;
+  a.tout_b = h->tout_b;
+  a.aout_w = h->aout_w;
+  a.aout_b = h->aout_b;
+  a.fnorm = h->fnorm;
+  for (int l = 0; l < L; ++l) {
+    a.in_norm[l] = h->layer[l].in_norm;
+    a.post_norm[l] = h->layer[l].post_norm;
+    a.m_qkv[l] = h->d_wmaps + 2 + 4 * l;
+    a.m_o[l] = h->d_wmaps + 3 + 4 * l;
+    a.m_gu[l] = h->d_wmaps + 4 + 4 * l;
+    a.m_down[l] = h->d_wmaps + 5 + 4 * l;
+  }
+  a.m_tin = h->d_wmaps;
+  a.m_tout = h->d_wmaps + 1;
+  const int box = a.box_rows == 128 ? 1 : 0;
+  a.m_xn = ws.d_amaps + 0 + box;
+  a.m_att = ws.d_amaps + 2 + box;
+  a.m_act = ws.d_amaps + 4 + box;
+  a.m_aemb = ws.d_amaps + 6 + box;
+  a.m_uemb = ws.d_amaps + 8 + box;
+  RUN(PI0X_K_LOOP, CK(launch_loop(a, s)));
+  CK(cudaGetLastError());
+  return PI0X_OK;
+}
+
+int enqueue_call(pi0x_handle *h, int B, int P, int N, cudaStream_t s) {
+  if (use_loop(h, B)) return enqueue_persistent(h, B, P, N, s, -1, kWaitLimitNs);
+  return h->bf16 ? enqueue_loop<bf16>(h, B, P, N, s) : enqueue_loop<float>(h, B, P, N, s);
+}
+
 // The whole call (all Euler steps) as one CUDA graph per (B, P, N, profiling),
 // captured on the handle's own stream and launched on the caller's.  Every
 // caller-owned pointer reaches the kernels through the device table d_ptrs, so a
@@ -586,7 +738,7 @@ int get_graph(pi0x_handle *h, int B, int P, int N, cudaGraphExec_t *out) {
     }
   cudaGraph_t graph = nullptr;
   CK(cudaStreamBeginCapture(h->cap, cudaStreamCaptureModeThreadLocal));
-  int st = h->bf16 ? enqueue_loop<bf16>(h, B, P, N, h->cap) : enqueue_loop<float>(h, B, P, N, h->cap);
+  int st = enqueue_call(h, B, P, N, h->cap);
   cudaError_t e = cudaStreamEndCapture(h->cap, &graph);
   if (st) {
     if (graph) cudaGraphDestroy(graph);
@@ -842,6 +994,7 @@ int pi0x_create(const pi0x_config *cfg, const pi0x_weights *w, pi0x_handle **out
     st = build_weight_maps(h);
     if (st) return fail(st);
   }
+  if (h->bf16) h->loop_grid = loop_max_grid(dev);
   e = cudaMalloc(&h->d_ptrs, sizeof(CallPtrs));
   if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&h->cap, cudaStreamNonBlocking);
   if (e == cudaSuccess) e = cudaMalloc(&h->d_err, sizeof(unsigned));
@@ -911,7 +1064,8 @@ int pi0x_sample(pi0x_handle *h, const void *const *prefix_k, const void *const *
   cp.x1 = (const float *)tmp;
   const bool x0_host = !is_device_ptr(x0);
   cp.x0 = x0_host ? ws.st_x : x0;  // staged x1 is consumed before x0 is written
-  if (h->bf16 && !attn_tc_maps(cp, L, B, P, ws.ks, ws.vs, (uint64_t)L * (B + (size_t)B * H))) {
+  if (h->bf16 && (!attn_tc_maps(cp, L, B, P, ws.ks, ws.vs, (uint64_t)L * (B + (size_t)B * H)) ||
+                  (use_loop(h, B) && !loop_attn_maps(cp, L, B, P, ws.ks, ws.vs, (uint64_t)L * (B + (size_t)B * H))))) {
     g_last_error = "pi0x_sample: cuTensorMapEncodeTiled failed for the prefix K/V (pointers must be 16-byte aligned)";
     return PI0X_EINVAL;
   }
@@ -922,13 +1076,29 @@ int pi0x_sample(pi0x_handle *h, const void *const *prefix_k, const void *const *
     // call, so the kernels then run back to back as they do in the graph.
     const long n = pi0x_launch_count(h, B, P, num_steps);
     launch_delay_ns((unsigned long long)(20000 * n + 2000000), s);
-    st = h->bf16 ? enqueue_loop<bf16>(h, B, P, num_steps, s) : enqueue_loop<float>(h, B, P, num_steps, s);
+    st = enqueue_call(h, B, P, num_steps, s);
+    if (st) return st;
+  } else if (use_loop(h, B) && (h->dbg_stall >= 0 || h->loop_direct)) {
+    // direct launches: a test's stalled call, or a driver that cannot capture the
+    // cooperative launch into a graph
+    const int stall = h->dbg_stall;
+    const unsigned long long limit = stall >= 0 ? h->dbg_wait_ns : kWaitLimitNs;
+    h->dbg_stall = -1;
+    st = enqueue_persistent(h, B, P, num_steps, s, stall, limit);
     if (st) return st;
   } else {
     cudaGraphExec_t exec = nullptr;
     st = get_graph(h, B, P, num_steps, &exec);
-    if (st) return st;
-    CK(cudaGraphLaunch(exec, s));
+    if (st && use_loop(h, B)) {
+      // the cooperative launch could not be captured: launch the loop directly from now on
+      h->loop_direct = true;
+      g_last_error.clear();
+      st = enqueue_persistent(h, B, P, num_steps, s, -1, kWaitLimitNs);
+      if (st) return st;
+    } else {
+      if (st) return st;
+      CK(cudaGraphLaunch(exec, s));
+    }
   }
   if (x0_host) CK(cudaMemcpyAsync(x0, ws.st_x, 4 * (size_t)B * H * A, cudaMemcpyDeviceToHost, s));
   h->last_stream = s;
@@ -944,7 +1114,8 @@ int pi0x_sync_status(pi0x_handle *h) {
   if (err) {
     cudaMemset(h->d_err, 0, sizeof(unsigned));
     g_last_error = "device error word 0x" + std::to_string(err);
-    return (err & (kErrTimeoutProducer | kErrTimeoutMma | kErrTimeoutEpilogue)) ? PI0X_ETIMEOUT : PI0X_EDEVICE;
+    return (err & (kErrTimeoutProducer | kErrTimeoutMma | kErrTimeoutEpilogue | kErrTimeoutFlag)) ? PI0X_ETIMEOUT
+                                                                                                 : PI0X_EDEVICE;
   }
   return PI0X_OK;
 }
@@ -960,6 +1131,24 @@ int pi0x_set_variant(pi0x_handle *h, int time_grid, int x_prediction, int causal
   h->time_grid = time_grid;
   h->x_pred = x_prediction;
   h->causal = causal_actions;
+  return PI0X_OK;
+}
+
+int pi0x_debug_loop_stall(pi0x_handle *h, int stage, unsigned long long wait_ns) {
+  if (!h || stage < 0 || wait_ns == 0) return PI0X_EINVAL;
+  h->dbg_stall = stage;
+  h->dbg_wait_ns = wait_ns;
+  return PI0X_OK;
+}
+
+int pi0x_uses_loop(const pi0x_handle *h, int B) { return h && B >= 1 && use_loop(h, B) ? 1 : 0; }
+
+int pi0x_debug_set_loop(pi0x_handle *h, int enable) {
+  if (!h || enable < 0 || enable > 1) return PI0X_EINVAL;
+  if (h->loop_off == !enable) return PI0X_OK;
+  if (h->called) CK(cudaStreamSynchronize(h->last_stream));
+  drop_graphs(h);
+  h->loop_off = !enable;
   return PI0X_OK;
 }
 
@@ -989,6 +1178,8 @@ int pi0x_profile_read(pi0x_handle *h, int kclass, long *launches, double *total_
 long pi0x_launch_count(const pi0x_handle *h, int B, int P, int num_steps) {
   if (!h || B < 1 || P < 0 || num_steps < 1) return -1;
   const long L = h->cfg.depth, H = h->cfg.horizon;
+  // persistent loop: mask prep, time-MLP half, x_1 copy, RoPE table, state embed, loop
+  if (use_loop(h, B)) return 6;
   Geo g{B, (int)H, h->cfg.action_dim, h->cfg.state_dim, P, B + B * (int)H};
   long n = 3 + 1 + (h->bf16 ? 1 : 0);  // mask prep, time-MLP half, x_1 copy; state embed; RoPE table
   for (int k = 0; k < num_steps; ++k) {
@@ -1004,14 +1195,15 @@ long pi0x_launch_count(const pi0x_handle *h, int B, int P, int num_steps) {
 
 void pi0x_destroy(pi0x_handle *h) {
   if (!h) return;
+  // the handle's work runs on the stream of its calls (the capture stream only records)
   if (h->called) cudaStreamSynchronize(h->last_stream);
-  cudaDeviceSynchronize();
   drop_graphs(h);
   for (cudaEvent_t ev : h->prof_ev) cudaEventDestroy(ev);
   if (h->cap) cudaStreamDestroy(h->cap);
   free_workspace(h->ws);
   if (h->ws.stage.base) cudaFree(h->ws.stage.base);
   if (h->warena.base) cudaFree(h->warena.base);
+  if (h->d_wmaps) cudaFree(h->d_wmaps);
   if (h->d_ptrs) cudaFree(h->d_ptrs);
   if (h->d_err) cudaFree(h->d_err);
   delete h;

@@ -22,14 +22,15 @@ PI0X_DTYPE_BF16, PI0X_DTYPE_F32 = 0, 1
 EXPORTED = ["pi0x_create", "pi0x_sample", "pi0x_sync_status", "pi0x_launch_count",
             "pi0x_status_string", "pi0x_last_error", "pi0x_destroy", "pi0x_version",
             "pi0x_debug_gemm_bf16", "pi0x_debug_attention", "pi0x_profile_enable", "pi0x_profile_read",
-            "pi0x_set_variant"]
+            "pi0x_set_variant", "pi0x_attention_noalloc", "pi0x_uses_loop", "pi0x_debug_loop_stall",
+            "pi0x_debug_set_loop"]
 
 #: time grids of pi0x_set_variant
 PI0X_TIME_PI0 = 0
 PI0X_TIME_LINSPACE = 1
 
 #: kernel classes of pi0x_profile_read
-K_CLASSES = ["prep", "embed", "gemm", "norm", "rope", "attn", "geglu", "final"]
+K_CLASSES = ["prep", "embed", "gemm", "norm", "rope", "attn", "geglu", "final", "loop"]
 
 
 class Pi0xError(RuntimeError):
@@ -103,6 +104,14 @@ def load() -> ctypes.CDLL:
     lib.pi0x_debug_gemm_bf16.restype = ctypes.c_int
     lib.pi0x_debug_attention.argtypes = [ctypes.c_void_p] * 6 + [ctypes.c_int] * 5 + [ctypes.c_void_p] * 2
     lib.pi0x_debug_attention.restype = ctypes.c_int
+    lib.pi0x_attention_noalloc.argtypes = [ctypes.c_void_p] * 6 + [ctypes.c_int] * 4 + [ctypes.c_void_p] * 2
+    lib.pi0x_attention_noalloc.restype = ctypes.c_int
+    lib.pi0x_uses_loop.argtypes = [ctypes.c_void_p, ctypes.c_int]
+    lib.pi0x_uses_loop.restype = ctypes.c_int
+    lib.pi0x_debug_loop_stall.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_ulonglong]
+    lib.pi0x_debug_loop_stall.restype = ctypes.c_int
+    lib.pi0x_debug_set_loop.argtypes = [ctypes.c_void_p, ctypes.c_int]
+    lib.pi0x_debug_set_loop.restype = ctypes.c_int
     lib.pi0x_profile_enable.argtypes = [ctypes.c_void_p, ctypes.c_int]
     lib.pi0x_profile_enable.restype = ctypes.c_int
     lib.pi0x_profile_read.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.POINTER(ctypes.c_long),
@@ -149,6 +158,15 @@ def debug_attention(q, ks, vs, prefix_k, prefix_v, mask, B, H, P, step0, out, im
     return out
 
 
+def attention_noalloc(q, ks, vs, prefix_k, prefix_v, mask, B, H, P, step0, out, stream: int = 0):
+    """The same attention through pi0x_attention_noalloc (no device allocation;
+    scratch in the library's static device array)."""
+    _check(load().pi0x_attention_noalloc(_ptr(q), _ptr(ks), _ptr(vs), _ptr(prefix_k), _ptr(prefix_v), _ptr(mask),
+                                         B, H, P, int(step0), _ptr(out), ctypes.c_void_p(stream)),
+           "pi0x_attention_noalloc")
+    return out
+
+
 class Sampler:
     """A pi0x handle: expert weights on the device plus the loop's workspace.
 
@@ -184,6 +202,18 @@ class Sampler:
 
     def launch_count(self, B: int, P: int, num_steps: int) -> int:
         return int(self._lib.pi0x_launch_count(self._h, B, P, num_steps))
+
+    def uses_loop(self, B: int) -> bool:
+        """True if calls with batch B run the persistent small-batch loop kernel."""
+        return bool(self._lib.pi0x_uses_loop(self._h, int(B)))
+
+    def debug_set_loop(self, enable: bool):
+        """Allow (True, default) or forbid (False) the persistent loop (see pi0x_debug.h)."""
+        _check(self._lib.pi0x_debug_set_loop(self._h, int(bool(enable))), "pi0x_debug_set_loop")
+
+    def debug_loop_stall(self, stage: int, wait_ns: int):
+        """Make the next loop call stall at `stage` (test hook, see pi0x_debug.h)."""
+        _check(self._lib.pi0x_debug_loop_stall(self._h, int(stage), int(wait_ns)), "pi0x_debug_loop_stall")
 
     def sample(self, prefix_k: Sequence, prefix_v: Sequence, mask, state, x1, num_steps: int,
                x0=None, stream: Optional[int] = None):
