@@ -64,8 +64,8 @@ int pi0x_attention_noalloc(const void *q, const void *ks, const void *vs, const 
                            void *stream);
 
 /* 1 if pi0x_sample(h, B, ...) runs the persistent small-batch loop kernel (bf16
- * mode, B * (horizon + 1) <= 128, a device that can co-schedule one CTA per SM),
- * else 0 (also for a NULL handle). */
+ * mode, B * (horizon + 1) <= 128, action_dim <= 32 and a multiple of 4, a device
+ * that can co-schedule one CTA per SM), else 0 (also for a NULL handle). */
 int pi0x_uses_loop(const pi0x_handle *h, int B);
 
 /* enable = 0: later pi0x_sample calls on `h` run every batch on the multi-kernel
@@ -78,9 +78,9 @@ int pi0x_debug_set_loop(pi0x_handle *h, int enable);
 
 /* Failure-path test hook of the persistent loop.  The next pi0x_sample call on `h`
  * that runs the loop kernel makes stage `stage` of the call (0 = the first stage of
- * Euler step 0; a GEMM stage is needed to take effect) wait on a done-counter that
- * nothing raises, with every wait of that call bounded by `wait_ns` nanoseconds
- * instead of the default 200 ms.  The wait gives up, the kernel's other waits see
+ * Euler step 0, in program order) wait on a done-counter that nothing raises, with
+ * every wait of that call bounded by `wait_ns` nanoseconds instead of the default
+ * 200 ms.  The wait gives up, the kernel's other waits see
  * the error word and return, and pi0x_sync_status then reports PI0X_ETIMEOUT; the
  * call's x0 is invalid.  Later calls run normally (every call starts from zeroed
  * counters).  Returns PI0X_EINVAL for a NULL handle, a negative stage or a zero

@@ -26,7 +26,9 @@ def _sampler(dims, seed):
     from vla_flow_matching_b200 import build, pi0x
     _torch()
     build.build()
-    return pi0x.Sampler(dims, synth.make_weights(dims, seed), pi0x.PI0X_BF16)
+    s = pi0x.Sampler(dims, synth.make_weights(dims, seed), pi0x.PI0X_BF16)
+    assert s.uses_loop(1), pi0x.load().pi0x_last_error().decode()
+    return s
 
 
 @pytest.mark.parametrize("name", ["tiny", "full_b1", "short_b8"])
@@ -53,7 +55,7 @@ def test_only_batches_that_fit_one_tile_use_the_loop():
     assert s.uses_loop(1) and s.uses_loop(2)          # 51 and 102 rows
     assert not s.uses_loop(3) and not s.uses_loop(32)  # 153 and 1632 rows
     assert s.launch_count(1, 816, 10) == 6
-    assert s.launch_count(32, 816, 10) > 100
+    assert s.launch_count(32, 816, 10) > 50       # one kernel per projection, attention, small step
     s.close()
 
 
@@ -69,12 +71,11 @@ def test_loop_two_samples_ragged_prefix(masked, hole):
     s.close()
 
 
-@pytest.mark.parametrize("stage", [1, 9], ids=["first_gemm", "layer1_qkv"])
+@pytest.mark.parametrize("stage", [1, 9], ids=["step0_mlp_out", "step0_layer1"])
 def test_stalled_stage_times_out_and_next_call_is_exact(stage):
-    """Stage 1 is the action-time MLP GEMM of step 0; stage 9 the QKV of layer 1 of
-    step 0 (three stages per step before the layers, six per layer with split
-    attention), so attention units of layer 0 and every CTA's later waits are in
-    flight when the error word is raised."""
+    """Stage 1 is the action-time MLP output GEMM of step 0; stage 9 lies in layer 1
+    of step 0, so layer 0's units and every CTA's later waits are in flight when the
+    error word is raised."""
     from vla_flow_matching_b200 import pi0x
     torch = _torch()
     wl = small_wl(B=1, P=77, steps=2, depth=2)

@@ -127,6 +127,24 @@ __device__ __forceinline__ void tma_load_2d(uint32_t smem_dst, const CUtensorMap
       : "memory");
 }
 
+// 1-D bulk copy of `bytes` (multiple of 16, both addresses 16-byte aligned) from
+// global memory into this CTA's shared memory, completion counted on `bar`.
+__device__ __forceinline__ void bulk_load(uint32_t smem_dst, const void *gsrc, uint32_t bytes, uint64_t *bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   smem_dst),
+               "l"(gsrc), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
+}
+
+// Offset (elements) of element (r, k) of a bf16 matrix stored as "tiled K-blocks":
+// for each 64-column K-block a tile of `rb` rows x 128 bytes in the 128-byte-swizzled
+// K-major layout the tensor cores read (16-byte chunk c of row r at chunk c ^ (r % 8)).
+// A K-block tile is contiguous, so one bulk copy into a 1024-byte-aligned shared
+// buffer gives an MMA operand.
+__host__ __device__ __forceinline__ size_t tiled_off(int r, int k, int rb) {
+  return ((size_t)((k >> 6) * rb + r) << 6) + (size_t)((((k >> 3) & 7) ^ (r & 7)) << 3) + (size_t)(k & 7);
+}
+
 // ---- tcgen05 -----------------------------------------------------------------
 __device__ __forceinline__ void tmem_alloc(uint32_t *smem_slot, uint32_t ncols) {
   asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(smem_slot)),
@@ -312,6 +330,14 @@ __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.lau
 __device__ __forceinline__ float gelu_tanh_f(float x) {
   const float k = 0.7978845608028654f;  // sqrt(2/pi)
   return 0.5f * x * (1.0f + tanhf(k * (x + 0.044715f * x * x * x)));
+}
+// GeGLU's tanh form with the SFU tanh (PTX tanh.approx.f32, relative error about
+// 2^-11): for products that are stored in bf16 (relative step 2^-8) right after.
+__device__ __forceinline__ float gelu_tanh_fast(float x) {
+  const float k = 0.7978845608028654f;  // sqrt(2/pi)
+  float t;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(k * (x + 0.044715f * x * x * x)));
+  return 0.5f * x * (1.0f + t);
 }
 __device__ __forceinline__ float silu_f(float x) { return x / (1.0f + expf(-x)); }
 // 2^x with the SFU instruction (PTX ex2.approx, relative error about 2^-22; 2^-inf = 0),

@@ -4,115 +4,157 @@
 // activation bytes, and a layer is a chain of five dependent contractions (QKV,
 // attention, O-proj, gate/up, down) whose weights do not depend on the activations.
 // One cooperative launch with one CTA per SM runs every stage of every Euler step of
-// the call (`sample_actions` / `denoise_step` / `_compute_layer_suffix_only` on the
-// vllm-omni pi0 page) in program order:
+// the call (`sample_actions` / `denoise_step` / `embed_suffix` /
+// `_compute_layer_suffix_only` on the vllm-omni pi0 page) in program order:
 //
-//   per step: ACTION_IN, TIN (action-time MLP in + SiLU), TOUT (MLP out -> residual
-//   stream, layer-0 norm inputs), then per layer QKV (+ RoPE), ATTN (split-KV masked
-//   MQA), COMBINE (merge of the splits), O (+ residual), GU (gate/up + GeGLU), DOWN
-//   (+ residual, next norm inputs), and last EULER (final norm, out-projection,
-//   x += dt v).
+//   per step TIN (action-time MLP input), TOUT (MLP output -> residual stream,
+//   layer-0 norm inputs), per layer QKV (+ RoPE), ATTN (masked MQA, one CTA per
+//   128-row query tile), O (+ residual), GU (gate/up + GeGLU), DOWN (+ residual,
+//   next norm inputs), and last XOUT (final norm, out-projection, x += dt v).
 //
-// Stage s of a CTA starts when the done-counter of stage s-1 (global memory, one per
-// stage of the call, zeroed before the launch) reaches the number of work items that
-// stage releases; every counter only grows, so the order of arrivals never matters.
-// A stage's results are released with a gpu-scope fence before the counter
-// increment and acquired with ld.acquire by the consumers (plus a proxy fence before
-// TMA reads them).
+// The action-time MLP input `mlp_in([action_in(x); temb])` is evaluated as
+// silu(w_xa x + tvec[k]) with w_xa = W_in[:, :W] W_action_in and the bias
+// W_in[:, :W] b_action_in folded into tvec (products formed once, in float64, at
+// pi0x_create): the same linear map with the action embedding not materialised,
+// which turns a K = 1024 contraction into a K = action_dim one per row.
+//
+// Stage s of a CTA starts when the done-counter of stage s-1 (global memory, one
+// per stage of the call, zeroed before the launch) reaches the number of work
+// items that stage releases; counters only grow, so arrival order never matters.
+// One poller (lane 0 of the V-loader warp) waits on the counters and opens a
+// shared-memory gate for the other roles.  Work items release with a gpu-scope red.release after a CTA
+// barrier over the threads that stored their results.
 //
 // Roles (256 threads):
-//   warp 0   weight TMA producer: streams this CTA's weight tiles of every stage, in
-//            program order, into a 15-slot ring.  Weights are inputs, so it runs ahead
-//            of the activations across stage boundaries, bounded only by the ring.
-//   warp 1   tcgen05.mma issuer (GEMM units, and S = Q K^T / O += P V of attention).
-//   warp 2   activation TMA loader of GEMM units; K loader of attention units.
-//   warp 3   V loader of attention units.
+//   warp 0    weight producer (lanes 0 and 1, alternate K-blocks): streams this CTA's
+//             weight K-blocks of every stage, in program order, into a 5-slot ring of
+//             16 KB.  Weights are inputs, so it runs ahead of the activations across
+//             stage boundaries, bounded only by the ring.
+//   warp 1    tcgen05.mma issuer (GEMM units; S = Q K^T and O += P V of attention).
+//   warp 2    activation loader of GEMM units; K loader of attention units.
+//   warp 3    poller of the stage done-counters (lane 0), V loader of attention units.
 //   warps 4-7 epilogues (TMEM lane quarter = warp % 4), the softmax of attention
-//            units, and the small stages (ACTION_IN, COMBINE, EULER).
+//             units and the row-wise stages (TIN, COMBINE, XOUT).
 //
-// GEMM units: the N columns of a Linear are cut into contiguous chunks of whole
-// 16-column groups (<= 64 columns) and the K range into `splits` parts; the
-// accumulator (M = 128 rows x chunk) lives in TMEM columns 448..511.  With split-K
-// every unit stores its fp32 partial tile and the last unit of a chunk to arrive
-// (counter) adds the partials in split order -- the result does not depend on timing
-// -- and runs the epilogue.  Epilogues are those of the multi-kernel path: SiLU +
-// time vector, bias, residual add with the fused RMSNorm producer (bf16 h*(1+g) and
-// per-16-column sums of squares), RoPE at position n_b + j with q/k/v stores, GeGLU.
+// GEMM units: the weight is the MMA's M side.  128 weight rows (output features) form
+// an m-tile and the call's rows, rounded up to 16 tokens, are N, so one tcgen05.mma
+// does 128 x N x 16 of useful work (on B200 each MMA costs its issuing warp about
+// 200 cycles whatever N is, so a small batch wants few, wide MMAs).  The K range of
+// every m-tile is split over ksplit CTAs (ksplit = grid / m-tiles, at most one per
+// K-block), so every Linear streams its weight through nearly every SM.  Each unit
+// stores its fp32 partial tile (token-major), raises its m-tile's counter, waits for
+// the other splits and adds a slice of the tokens over all splits in split order (the
+// result does not depend on timing), then runs the epilogue for that slice: bias or
+// residual with the fused RMSNorm producer (bf16 h*(1+g), per-m-tile sums of h^2),
+// RoPE at position n_b + j with q/k/v stores, or GeGLU.
 //
-// Shared memory: a weight ring (15 x 8 KB) and region X (96 KB) that holds either the
-// activation ring of a GEMM unit (4 x 16 KB) or the K/V rings (2 x 16 KB each) and P
-// buffers (2 x 16 KB) of an attention unit.  Region X passes from one unit to the next
-// through a counter of units whose MMAs have completed.
+// Copies: on B200 every async copy costs its issuing thread about 0.2 us whatever its
+// size, so the loop copies large contiguous runs: weights are stored once, at
+// pi0x_create, as m-tiles of swizzled 128 x 64 K-blocks (one 16 KB bulk copy per
+// K-block); the activation operands (norm outputs, attention output, GeGLU product,
+// MLP input) are written by their producers as tiled K-blocks (tiled_off), one bulk
+// copy per K-block, issued by four lanes at once.  The attention's prefix K/V (a call
+// input) is prefetched into L2, a slice per CTA, when the QKV stage of its layer begins.
 //
-// Every wait is bounded (LoopArgs::wait_ns) and gives up early once the error word is
-// set; on the way out each role waits for the copies it issued, the MMA warp for its
-// MMAs, and TMEM is freed.
+// Shared memory: region X (128 KB) holds either the activation ring of a GEMM unit
+// or the K/V rings (3 x 16 KB each) and P buffers (2 x 16 KB) of an attention unit,
+// handed from unit to unit through a counter of units whose MMAs have completed; then
+// the weight ring (5 x 16 KB).
+//
+// Every wait is bounded (LoopArgs::wait_ns) and gives up early once the error word
+// is set; on the way out each role waits for the copies it issued, the MMA warp for
+// its MMAs, and TMEM is freed.
 #include <math.h>
-
-#include <cooperative_groups.h>
 
 #include "common.cuh"
 #include "kernels.cuh"
 
 namespace pi0x {
 
+#ifdef PI0X_LOOP_TIMELINE
+// Profiling build: globaltimer stamps per (stage, CTA, slot) into a device buffer.
+__device__ unsigned long long *g_loop_tl = nullptr;
+#define LOOP_STAMP(gs, slot)                                                                           \
+  do {                                                                                                 \
+    if (g_loop_tl) g_loop_tl[((size_t)(gs) * gridDim.x + blockIdx.x) * 16 + (slot)] = globaltimer_ns(); \
+  } while (0)
+#else
+#define LOOP_STAMP(gs, slot) \
+  do {                       \
+  } while (0)
+#endif
+
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int kWSlots = 15;
-constexpr uint32_t kWSlotBytes = 8192;
-constexpr int kASlots = 4;
-constexpr uint32_t kASlotBytes = 16384;
+constexpr uint32_t kXBytes = 128 * 1024;
+constexpr int kWSlots = 5;
+constexpr uint32_t kWSlotBytes = 16384;           // one K-block of a 128-row weight m-tile
 constexpr int kKB = kLoopKeyBlock;            // 32 keys per attention block
+constexpr int kKVBufs = 3;
 constexpr uint32_t kKVTile = kKB * 512;       // 32 keys x 256 dims bf16 = 16 KB
 constexpr uint32_t kKVSub = kKB * 128;        // one 64-dim sub-tile = 4 KB
 constexpr uint32_t kAtomBytes = 8 * 128;      // 8 keys x 64 dims: one 8-row box
 constexpr uint32_t kPTile = 128 * 128;        // 128 rows x 128 B (32 keys used)
 
-constexpr uint32_t kOffW = 0;
-constexpr uint32_t kOffX = kOffW + kWSlots * kWSlotBytes;
+constexpr uint32_t kOffX = 0;
 constexpr uint32_t kOffA = kOffX;
 constexpr uint32_t kOffK = kOffX;
-constexpr uint32_t kOffV = kOffK + 2 * kKVTile;
-constexpr uint32_t kOffP = kOffV + 2 * kKVTile;
-constexpr uint32_t kXBytes = 6 * kKVTile;  // 96 KB
-static_assert(kASlots * kASlotBytes <= kXBytes, "activation ring fits region X");
+constexpr uint32_t kOffV = kOffK + kKVBufs * kKVTile;
+constexpr uint32_t kOffP = kOffV + kKVBufs * kKVTile;
 static_assert(kOffP + 2 * kPTile == kOffX + kXBytes, "attention buffers fill region X");
-constexpr uint32_t kOffBar = kOffX + kXBytes;
+constexpr uint32_t kOffW = kOffX + kXBytes;
+constexpr uint32_t kOffBar = kOffW + kWSlots * kWSlotBytes;
+constexpr int kMaxASlots = 24;
 
 struct Bars {
   uint64_t w_full[kWSlots], w_empty[kWSlots];
-  uint64_t a_full[kASlots], a_empty[kASlots];
-  uint64_t acc_full, acc_empty;
-  uint64_t k_full[2], k_empty[2], v_full[2], pv_done[2];
+  uint64_t a_full[kMaxASlots], a_empty[kMaxASlots];
+  uint64_t acc_full;
+  uint64_t k_full[kKVBufs], k_empty[kKVBufs], v_full[kKVBufs], pv_done[kKVBufs];
   uint64_t s_full[2], s_empty[2], p_full[2];
   uint64_t q_full, mma_fin;
   uint32_t tmem_slot;
   uint32_t x_done;    // units that used region X and whose MMAs have completed (monotonic)
-  int last;           // split-K: this CTA reduces the chunk
-  float red[8];       // EULER row reduction
+  uint32_t tmem_done; // units whose accumulator reads (GEMM) / O readout (attention) are done
+  uint32_t ready;     // stages whose predecessor has completed (monotonic, set by the poller)
+  int last;           // epilogue broadcast: the m-tile's partials are all stored
+  float red[8];
   uint32_t w_fills[kWSlots];  // drain bookkeeping
-  uint32_t a_fills[kASlots];
-  uint32_t k_fills[2], v_fills[2];
+  uint32_t a_fills[kMaxASlots];
+  uint32_t k_fills[kKVBufs], v_fills[kKVBufs];
 };
-constexpr uint32_t kSmemTotal = kOffBar + ((sizeof(Bars) + 127) / 128) * 128 + 1024 + 4 * 1024 /* EULER row */;
+constexpr uint32_t kBarBytes = ((sizeof(Bars) + 127) / 128) * 128;
+constexpr uint32_t kOffRow = kOffBar + kBarBytes;   // XOUT: the normalised row (1024 fp32)
+constexpr uint32_t kSmemTotal = kOffRow + 4096 + 1024 /* alignment slack */;
 static_assert(kSmemTotal <= 232448, "shared memory per CTA");
 
-// TMEM columns: S buffers 0 and 32, Q 64..191 (bf16 pairs), O 192..447, GEMM 448..511
+// TMEM columns: S 0..127 (two buffers x two dim-halves of 32 columns), Q 128..255
+// (bf16 pairs), O 256..511.  A GEMM unit's accumulator (128 weight rows x box_rows
+// tokens) uses 256..383: units run one at a time per CTA and each starts after the
+// previous one's TMEM reads.
 constexpr uint32_t kTmemS = 0;
-constexpr uint32_t kTmemQ = 64;
-constexpr uint32_t kTmemO = 192;
-constexpr uint32_t kTmemAcc = 448;
+constexpr uint32_t kTmemQ = 128;
+constexpr uint32_t kTmemO = 256;
+constexpr uint32_t kTmemAcc = 256;
 constexpr uint32_t kTmemCols = 512;
 
 constexpr unsigned kFull = 0xffffffffu;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleSlack = 8.0f;
 
+__device__ __forceinline__ int ld_relaxed(const int *p) {
+  int v;
+  asm volatile("ld.relaxed.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
 __device__ __forceinline__ int ld_acquire(const int *p) {
   int v;
   asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
   return v;
+}
+__device__ __forceinline__ void red_release_add(int *p, int v) {
+  asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 __device__ __forceinline__ void fence_proxy_async_global() { asm volatile("fence.proxy.async.global;" ::: "memory"); }
 __device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
@@ -132,21 +174,6 @@ __device__ __forceinline__ bool lwait(uint64_t *bar, uint32_t parity, const Loop
     }
   }
 }
-// Wait until *p >= target (acquire), with the same limits.
-__device__ __forceinline__ bool lpoll(const int *p, int target, const LoopArgs &a) {
-  if (ld_acquire(p) >= target) return true;
-  const unsigned long long t0 = globaltimer_ns();
-  while (true) {
-    for (int i = 0; i < 16; ++i)
-      if (ld_acquire(p) >= target) return true;
-    if (err_set(a)) return false;
-    if (globaltimer_ns() - t0 > a.wait_ns) {
-      atomicOr(a.err, kErrTimeoutFlag);
-      return false;
-    }
-  }
-}
-
 // Drain wait at exit: bounded by time only (it must wait for copies in flight even
 // after the error word was set).
 __device__ __forceinline__ void dwait(uint64_t *bar, uint32_t parity, const LoopArgs &a) {
@@ -154,32 +181,44 @@ __device__ __forceinline__ void dwait(uint64_t *bar, uint32_t parity, const Loop
   while (!mbar_try_wait(bar, parity))
     if (globaltimer_ns() - t0 > a.wait_ns) return;
 }
-// Region X hand-off: the epilogue counts units whose MMAs completed; a loader waits
-// until every earlier unit that used region X is counted (a monotonic counter, so a
-// loader that looks late never misreads a phase).
-__device__ __forceinline__ void x_release(Bars &bs) {
-  __threadfence_block();
-  atomicAdd(&bs.x_done, 1u);
-}
-__device__ __forceinline__ bool x_acquire(Bars &bs, uint32_t need, const LoopArgs &a, unsigned bit) {
-  const volatile uint32_t *c = &bs.x_done;
+// Wait until *c >= need for a shared-memory counter written by another role
+// (monotonic, so a late reader never misreads it); bounded like lwait.
+__device__ __forceinline__ bool smem_wait(const uint32_t *cnt, uint32_t need, const LoopArgs &a, unsigned bit) {
+  const volatile uint32_t *c = cnt;
   if (*c >= need) {
     __threadfence_block();
     return true;
   }
+  // back off between polls: a tight loop of shared-memory loads competes for the SM's
+  // shared-memory / shuffle pipe with the warps doing the work being waited for
   const unsigned long long t0 = globaltimer_ns();
   while (true) {
-    for (int i = 0; i < 64; ++i)
+    for (int i = 0; i < 16; ++i) {
       if (*c >= need) {
         __threadfence_block();
         return true;
       }
+      __nanosleep(64);
+    }
     if (err_set(a)) return false;
     if (globaltimer_ns() - t0 > a.wait_ns) {
       atomicOr(a.err, bit);
       return false;
     }
   }
+}
+__device__ __forceinline__ void smem_publish(uint32_t *cnt, uint32_t v) {
+  __threadfence_block();
+  *(volatile uint32_t *)cnt = v;
+}
+// Stage gate: the poller opened stage gs (its predecessor completed, acquired at gpu scope).
+__device__ __forceinline__ bool gate(Bars &bs, int gs, const LoopArgs &a) {
+  return smem_wait(&bs.ready, (uint32_t)gs + 1u, a, kErrTimeoutFlag);
+}
+// Region X hand-off.
+__device__ __forceinline__ void x_release(Bars &bs) {
+  __threadfence_block();
+  atomicAdd(&bs.x_done, 1u);
 }
 
 __device__ __forceinline__ void tmem_ld_x16(uint32_t taddr, float (&v)[16]) {
@@ -195,6 +234,15 @@ __device__ __forceinline__ void tmem_ld_x16(uint32_t taddr, float (&v)[16]) {
   for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// Store of 8 bf16 at offset `off` of every replica of a tiled activation buffer.
+__device__ __forceinline__ void store_reps(bf16 *buf, size_t off, size_t rep_stride, uint4 v) {
+#pragma unroll
+  for (int r = 0; r < kLoopReps; ++r) *reinterpret_cast<uint4 *>(buf + r * rep_stride + off) = v;
+}
+__device__ __forceinline__ void prefetch_l2(const void *p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
 __device__ __forceinline__ uint4 pack8(const float *v) {
   uint32_t p[4];
 #pragma unroll
@@ -207,15 +255,12 @@ __device__ __forceinline__ uint4 pack8(const float *v) {
 
 // ---- program geometry ------------------------------------------------------------
 struct StageInfo {
-  int kind, layer, step, gs;  // gs: index of the stage in the call
+  int kind, layer, step;
 };
-__device__ __forceinline__ int stage_count(const LoopArgs &a) { return loop_stages_per_step(a.L, a.attn_splits); }
+__device__ __forceinline__ int total_stages(const LoopArgs &a) { return loop_total_stages(a.N, a.L, a.attn_splits); }
 __device__ __forceinline__ StageInfo stage_at(const LoopArgs &a, int gs) {
   StageInfo si;
-  const int spp = stage_count(a);
-  si.gs = gs;
-  si.step = gs / spp;
-  loop_stage(gs % spp, a.L, a.attn_splits, si.kind, si.layer);
+  loop_stage(gs, a.L, a.attn_splits, si.kind, si.layer, si.step);
   return si;
 }
 __device__ __forceinline__ int q_tiles(const LoopArgs &a, int step0) {
@@ -230,84 +275,106 @@ __device__ __forceinline__ int combine_ctas(const LoopArgs &a, int step0) {
   const int c = (combine_items(a, step0) + 3) / 4;
   return c < a.grid ? c : a.grid;
 }
-__device__ __forceinline__ int action_ctas(const LoopArgs &a) { return a.grid < 128 ? a.grid : 128; }
-__device__ __forceinline__ int euler_units(const LoopArgs &a) { return a.B * a.H * ((a.A + 15) / 16); }
-__device__ __forceinline__ int euler_ctas(const LoopArgs &a) {
-  const int u = euler_units(a);
+// TIN: 128 units of 8 output columns (all rows); XOUT: units of (action row, 16 outputs).
+__device__ __forceinline__ int tin_ctas(const LoopArgs &a) { return a.grid < kWidth / 8 ? a.grid : kWidth / 8; }
+__device__ __forceinline__ int xout_units(const LoopArgs &a) { return a.B * a.H * ((a.A + 15) / 16); }
+__device__ __forceinline__ int xout_ctas(const LoopArgs &a) {
+  const int u = xout_units(a);
   return u < a.grid ? u : a.grid;
 }
 // Arrivals that complete stage `si`.
 __device__ __forceinline__ int stage_expect(const LoopArgs &a, const StageInfo &si) {
   const int step0 = si.step == 0;
   switch (si.kind) {
-    case LK_ACTION_IN: return action_ctas(a);
+    case LK_TIN: return tin_ctas(a);
+    case LK_XOUT: return xout_ctas(a);
     case LK_ATTN: return attn_units(a, step0);
     case LK_COMBINE: return combine_ctas(a, step0);
-    case LK_EULER: return euler_ctas(a);
-    default: return loop_gemm_plan(si.kind, a.grid).nchunks;
+    default: {
+      const LoopGemm p = loop_gemm_plan(si.kind, a.grid);
+      return p.mtiles * p.ksplit;
+    }
   }
 }
-// Wait (one thread) until the stage before `gs` has completed.
-__device__ __forceinline__ bool wait_prev(const LoopArgs &a, int gs) {
-  if (gs == 0) return true;
-  const StageInfo p = stage_at(a, gs - 1);
-  return lpoll(a.done + (gs - 1), stage_expect(a, p), a);
-}
-// Release of a stage's work item (one thread, after the item's stores are ordered
-// before it by epi_bar()).
-__device__ __forceinline__ void release(const LoopArgs &a, int gs) {
-  __threadfence();
-  atomicAdd(a.done + gs, 1);
-}
+// Release of a stage's work item (one thread, after epi_bar() ordered the item's
+// stores before it).
+__device__ __forceinline__ void release(const LoopArgs &a, int gs) { red_release_add(a.done + gs, 1); }
 
+// GEMM unit u: m-tile m (weight rows 128 m ..), K split s, K-blocks [kb0, kb1).
 struct GUnit {
-  int n0, w, kb0, kb1, chunk, split;
+  int m, s, kb0, kb1;
 };
 __device__ __forceinline__ GUnit gemm_unit(const LoopGemm &p, int u) {
   GUnit g;
-  g.chunk = u / p.splits;
-  g.split = u % p.splits;
-  const int G = p.N / 16;
-  const int g0 = (int)((long)g.chunk * G / p.nchunks), g1 = (int)((long)(g.chunk + 1) * G / p.nchunks);
-  g.n0 = g0 * 16;
-  g.w = (g1 - g0) * 16;
-  const int nk = p.K / 64, kps = (nk + p.splits - 1) / p.splits;
-  g.kb0 = g.split * kps;
-  g.kb1 = min(nk, g.kb0 + kps);
+  g.m = u / p.ksplit;
+  g.s = u % p.ksplit;
+  const int nk = p.K / 64;
+  g.kb0 = (int)((long)g.s * nk / p.ksplit);
+  g.kb1 = (int)((long)(g.s + 1) * nk / p.ksplit);
   return g;
 }
-__device__ __forceinline__ const CUtensorMap *weight_map(const LoopArgs &a, int kind, int layer) {
+// Tokens [t0, t1) of the stored range [r_lo, r_hi) that split s of an m-tile adds up
+// (an even count per split, so the paired epilogues take two tokens at a time).
+__device__ __forceinline__ void red_slice(int r_lo, int r_hi, int ksplit, int s, int &t0, int &t1) {
+  const int per = (((r_hi - r_lo) + ksplit - 1) / ksplit + 1) & ~1;
+  t0 = min(r_hi, r_lo + s * per);
+  t1 = min(r_hi, t0 + per);
+}
+// Bounded wait until a global counter reaches `need` (then acquired at gpu scope).
+__device__ bool gwait(const int *cnt, int need, const LoopArgs &a, unsigned bit) {
+  if (ld_acquire(cnt) >= need) return true;
+  const unsigned long long t0 = globaltimer_ns();
+  while (true) {
+    bool hit = false;
+    for (int i = 0; i < 32 && !hit; ++i) hit = ld_relaxed(cnt) >= need;
+    if (hit) break;
+    if (err_set(a)) return false;
+    if (globaltimer_ns() - t0 > a.wait_ns) {
+      atomicOr(a.err, bit);
+      return false;
+    }
+  }
+  (void)ld_acquire(cnt);
+  return true;
+}
+__device__ __forceinline__ const bf16 *weight_tiles(const LoopArgs &a, int kind, int layer) {
   switch (kind) {
-    case LK_TIN: return a.m_tin;
-    case LK_TOUT: return a.m_tout;
-    case LK_QKV: return a.m_qkv[layer];
-    case LK_O: return a.m_o[layer];
-    case LK_GU: return a.m_gu[layer];
-    default: return a.m_down[layer];
+    case LK_TOUT: return a.w_tout;
+    case LK_QKV: return a.w_qkv[layer];
+    case LK_O: return a.w_o[layer];
+    case LK_GU: return a.w_gu[layer];
+    default: return a.w_down[layer];
   }
 }
-__device__ __forceinline__ const CUtensorMap *act_map(const LoopArgs &a, int kind) {
+// Activation operand of a GEMM stage (tiled K-blocks of box_rows rows).
+__device__ __forceinline__ const bf16 *act_tiles(const LoopArgs &a, int kind) {
+  const size_t rep = (size_t)(blockIdx.x % kLoopReps) * a.rep_rows;
   switch (kind) {
-    case LK_TIN: return a.m_aemb;
-    case LK_TOUT: return a.m_uemb;
-    case LK_QKV: case LK_GU: return a.m_xn;
-    case LK_O: return a.m_att;
-    default: return a.m_act;
+    case LK_TOUT: return a.uemb + rep * kWidth;
+    case LK_QKV: case LK_GU: return a.xn + rep * kWidth;
+    case LK_O: return a.att + rep * kQDim;
+    default: return a.act + rep * kMlp;
   }
 }
-// Activation rows of a GEMM stage: A rows [a_row0, a_row0 + M), output rows out_row0 + r.
-__device__ __forceinline__ void gemm_rows(const LoopArgs &a, int kind, int step0, int &a_row0, int &M, int &out_row0) {
-  const int BH = a.B * a.H;
-  if (kind == LK_TIN || kind == LK_TOUT) {
-    a_row0 = 0;
-    M = BH;
-    out_row0 = kind == LK_TOUT ? a.B : 0;
+// Rows of a GEMM stage: the MMA runs over every row of the activation tile; tile rows
+// [r_lo, r_hi) are stored, tile row r as output row r + out_off.
+__device__ __forceinline__ void gemm_rows(const LoopArgs &a, int kind, int step0, int &r_lo, int &r_hi, int &out_off) {
+  if (kind == LK_TOUT) {
+    r_lo = 0;
+    r_hi = a.B * a.H;
+    out_off = a.B;
     return;
   }
-  a_row0 = step0 ? 0 : a.B;
-  M = a.R - a_row0;
-  out_row0 = a_row0;
+  r_lo = step0 ? 0 : a.B;
+  r_hi = a.R;
+  out_off = 0;
 }
+__device__ __forceinline__ uint32_t a_slot_bytes(const LoopArgs &a) { return (uint32_t)a.box_rows * 128u; }
+__device__ __forceinline__ int a_slots(const LoopArgs &a) {
+  const int n = (int)(kXBytes / a_slot_bytes(a));
+  return n < kMaxASlots ? n : kMaxASlots;
+}
+
 
 // ---- attention key slots (32-key blocks) -------------------------------------------
 // Source of key slot kk of sample b: 2*row of the prefix tensor (B*P rows), 2*row+1 of
@@ -338,12 +405,12 @@ __device__ __forceinline__ void load_kv_tile(int blk, uint32_t tile, uint64_t *f
   const int code = slot_code(kb + lane, nbp, nv, contig, b, a, vi);
   const int c0 = __shfl_sync(kFull, code, 0);
   if (__all_sync(kFull, c0 >= 0 && code == c0 + 2 * lane)) {
-    if (lane == 0) {
-      mbar_expect_tx(full, kKVTile);
+    if (lane == 0) mbar_expect_tx(full, kKVTile);
+    __syncwarp();
+    if (lane < 4) {  // one 32-row box per 64-dim sub-tile, four issuing lanes
       const CUtensorMap *m = (c0 & 1) ? smap32 : pmap32;
       const int y = (c0 & 1) ? sfx_row0 + (c0 >> 1) : (c0 >> 1);
-#pragma unroll
-      for (int sub = 0; sub < 4; ++sub) tma_load_2d(tile + sub * kKVSub, m, sub * 64, y, full);
+      tma_load_2d(tile + lane * kKVSub, m, lane * 64, y, full);
     }
     __syncwarp();
     cp_async_mbar_arrive(full);
@@ -400,39 +467,81 @@ __device__ __forceinline__ AUnit attn_unit(const LoopArgs &a, int u, int step0) 
   return t;
 }
 
-// ---- role: weight producer (warp 0, one lane) ---------------------------------------
-__device__ void role_weights(const LoopArgs &a, uint8_t *smem, Bars &bs) {
-  const int total = a.N * stage_count(a);
+// ---- poller (warp 3, lane 0): open stage gs once stage gs - 1 has completed ----------
+__device__ bool poll_stage(const LoopArgs &a, Bars &bs, int gs) {
+  if (gs > 0) {
+    const int *cnt = a.done + (gs - 1);
+    const int target = stage_expect(a, stage_at(a, gs - 1));
+    if (ld_relaxed(cnt) < target) {
+      const unsigned long long t0 = globaltimer_ns();
+      while (true) {
+        bool hit = false;
+        for (int i = 0; i < 32 && !hit; ++i) hit = ld_relaxed(cnt) >= target;
+        if (hit) break;
+        if (err_set(a)) return false;
+        if (globaltimer_ns() - t0 > a.wait_ns) {
+          atomicOr(a.err, kErrTimeoutFlag);
+          return false;
+        }
+      }
+    }
+    (void)ld_acquire(cnt);  // acquire the predecessor's results at gpu scope
+  }
+  if (gs == a.debug_stall_stage) {  // test hook: a counter that nothing raises
+    const unsigned long long t0 = globaltimer_ns();
+    while (ld_relaxed(a.done + gs) < (1 << 30)) {
+      if (err_set(a)) return false;
+      if (globaltimer_ns() - t0 > a.wait_ns) {
+        atomicOr(a.err, kErrTimeoutFlag);
+        return false;
+      }
+    }
+  }
+  smem_publish(&bs.ready, (uint32_t)gs + 1u);
+  return true;
+}
+
+// ---- role: weight producer (warp 0, lanes 0 and 1) ----------------------------------
+// One 16 KB bulk copy per K-block of the unit's m-tile (the K-blocks of a unit are one
+// contiguous run of the tiled weight); the two lanes take alternate K-blocks so two
+// copies are in issue at once.
+__device__ void role_weights(const LoopArgs &a, uint8_t *smem, Bars &bs, int me) {
+  const int total = total_stages(a);
   uint32_t wi = 0;
   bool ok = true;
-  // the weight maps live in device memory: acquire them once
-  tma_map_acquire(a.m_tin);
-  tma_map_acquire(a.m_tout);
-  for (int l = 0; l < a.L; ++l) {
-    tma_map_acquire(a.m_qkv[l]);
-    tma_map_acquire(a.m_o[l]);
-    tma_map_acquire(a.m_gu[l]);
-    tma_map_acquire(a.m_down[l]);
-  }
   for (int gs = 0; gs < total && ok; ++gs) {
     const StageInfo si = stage_at(a, gs);
     if (!loop_is_gemm(si.kind)) continue;
     const LoopGemm p = loop_gemm_plan(si.kind, a.grid);
-    const CUtensorMap *map = weight_map(a, si.kind, si.layer);
-    const int U = p.nchunks * p.splits;
+    const bf16 *wt = weight_tiles(a, si.kind, si.layer);
+    const int U = p.mtiles * p.ksplit;
+    // the same unit's weights one layer later (the next step's first layer after the
+    // last): they go to L2 now, so their copies a layer from now are L2 hits
+    const bf16 *wnext = nullptr;
+    if (si.kind != LK_TOUT) {
+      if (si.layer + 1 < a.L)
+        wnext = weight_tiles(a, si.kind, si.layer + 1);
+      else if (si.step + 1 < a.N)
+        wnext = weight_tiles(a, si.kind, 0);
+    }
     for (int u = blockIdx.x; u < U && ok; u += gridDim.x) {
       const GUnit g = gemm_unit(p, u);
+      const bf16 *src = wt + (size_t)g.m * 128 * p.K;
+      if (wnext && me == 0)
+        prefetch_l2(wnext + (size_t)g.m * 128 * p.K + (size_t)g.kb0 * 128 * 64, (uint32_t)(g.kb1 - g.kb0) * kWSlotBytes);
       for (int kb = g.kb0; kb < g.kb1; ++kb, ++wi) {
+        if ((int)(wi & 1u) != me) continue;  // the other issuing lane's fill
         const int slot = wi % kWSlots;
         const uint32_t n = wi / kWSlots;
         if (n > 0 && !lwait(&bs.w_empty[slot], (n - 1) & 1u, a, kErrTimeoutProducer)) {
           ok = false;
           break;
         }
-        mbar_arrive_expect_tx(&bs.w_full[slot], (uint32_t)g.w * 128u);
-        for (int r = 0; r < g.w; r += 16)
-          tma_load_2d(smem + kOffW + slot * kWSlotBytes + r * 128, map, kb * 64, g.n0 + r, &bs.w_full[slot]);
+        mbar_arrive_expect_tx(&bs.w_full[slot], kWSlotBytes);
+        bulk_load(smem_u32(smem + kOffW + slot * kWSlotBytes), src + (size_t)kb * 128 * 64, kWSlotBytes,
+                  &bs.w_full[slot]);
         bs.w_fills[slot] = n + 1;
+        if (kb + 1 >= g.kb1) LOOP_STAMP(gs, 5);
       }
     }
   }
@@ -440,9 +549,11 @@ __device__ void role_weights(const LoopArgs &a, uint8_t *smem, Bars &bs) {
 
 // ---- role: MMA issuer (warp 1, whole warp; one elected lane issues) ------------------
 __device__ void role_mma(const LoopArgs &a, uint8_t *smem, Bars &bs, uint32_t tmem) {
-  const int total = a.N * stage_count(a);
+  const int total = total_stages(a);
   const uint32_t sbase = smem_u32(smem);
-  uint32_t wi = 0, ai = 0, acc_n = 0, kj = 0, vj = 0, sj = 0, pj = 0, qn = 0;
+  const int nas = a_slots(a);
+  const uint32_t asb = a_slot_bytes(a);
+  uint32_t wi = 0, ai = 0, acc_n = 0, kj = 0, vj = 0, sj = 0, pj = 0, qn = 0, units_before = 0;
   bool ok = true;
   const uint64_t kdesc0 = smem_desc_k_sw128(sbase + kOffK, 0);
   const uint64_t pdesc0 = smem_desc_k_sw128(sbase + kOffP, 0);
@@ -453,40 +564,48 @@ __device__ void role_mma(const LoopArgs &a, uint8_t *smem, Bars &bs, uint32_t tm
     const StageInfo si = stage_at(a, gs);
     if (loop_is_gemm(si.kind)) {
       const LoopGemm p = loop_gemm_plan(si.kind, a.grid);
-      const int U = p.nchunks * p.splits;
+      const int U = p.mtiles * p.ksplit;
+      // D[128 weight rows, box_rows tokens] += W[128, 16] X[box_rows, 16]^T: A is the
+      // weight K-block, B the activation K-block, both K-major with the 128-byte swizzle
+      const uint32_t idesc = idesc_bf16_f32(128, a.box_rows);
       for (int u = blockIdx.x; u < U && ok; u += gridDim.x) {
         const GUnit g = gemm_unit(p, u);
-        if (acc_n > 0 && !__all_sync(kFull, lwait(&bs.acc_empty, (acc_n - 1) & 1u, a, kErrTimeoutMma))) {
+        // the accumulator may be written once every earlier unit's TMEM reads are done
+        bool good = true;
+        if ((threadIdx.x & 31) == 0) good = smem_wait(&bs.tmem_done, units_before, a, kErrTimeoutMma);
+        if (!__all_sync(kFull, __shfl_sync(kFull, (int)good, 0) != 0)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint32_t idesc = idesc_bf16_f32(128, g.w);
-        for (int kb = g.kb0; kb < g.kb1; ++kb, ++wi, ++ai) {
-          const int ws = wi % kWSlots, as = ai % kASlots;
+        for (int kb = g.kb0; kb < g.kb1 && ok; ++kb, ++wi, ++ai) {
+          const int ws = wi % kWSlots, as = ai % nas;
           if (!__all_sync(kFull, lwait(&bs.w_full[ws], (wi / kWSlots) & 1u, a, kErrTimeoutMma)) ||
-              !__all_sync(kFull, lwait(&bs.a_full[as], (ai / kASlots) & 1u, a, kErrTimeoutMma))) {
+              !__all_sync(kFull, lwait(&bs.a_full[as], (ai / nas) & 1u, a, kErrTimeoutMma))) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t ab = sbase + kOffA + as * kASlotBytes, wb = sbase + kOffW + ws * kWSlotBytes;
+          const uint32_t wb = sbase + kOffW + ws * kWSlotBytes, ab = sbase + kOffA + as * asb;
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            tc_mma_bf16_w(tmem + kTmemAcc, smem_desc_k_sw128(ab, kk * 32), smem_desc_k_sw128(wb, kk * 32), idesc,
+            tc_mma_bf16_w(tmem + kTmemAcc, smem_desc_k_sw128(wb, kk * 32), smem_desc_k_sw128(ab, kk * 32), idesc,
                           (kb > g.kb0 || kk > 0) ? 1u : 0u);
-          tc_commit_w(&bs.w_empty[ws]);
           tc_commit_w(&bs.a_empty[as]);
+          tc_commit_w(&bs.w_empty[ws]);
         }
         if (!ok) break;
+        if ((threadIdx.x & 31) == 0) LOOP_STAMP(gs, 6);
         tc_commit_w(&bs.acc_full);
         ++acc_n;
+        ++units_before;
       }
     } else if (si.kind == LK_ATTN) {
       const int step0 = si.step == 0;
       const int U = attn_units(a, step0);
       for (int u = blockIdx.x; u < U && ok; u += gridDim.x) {
         const AUnit t = attn_unit(a, u, step0);
+        ++units_before;
         if (t.nb == 0) continue;
         if (!__all_sync(kFull, lwait(&bs.q_full, qn & 1u, a, kErrTimeoutMma))) {
           ok = false;
@@ -495,19 +614,22 @@ __device__ void role_mma(const LoopArgs &a, uint8_t *smem, Bars &bs, uint32_t tm
         ++qn;
         tc_fence_after();
         auto issue_s = [&]() -> bool {  // S[sj & 1] = Q K(kj)^T
-          const int kbuf = kj % 2, sb = sj & 1;
-          if (!__all_sync(kFull, lwait(&bs.k_full[kbuf], (kj / 2) & 1u, a, kErrTimeoutMma))) return false;
+          const int kbuf = kj % kKVBufs, sb = sj & 1;
+          if (!__all_sync(kFull, lwait(&bs.k_full[kbuf], (kj / kKVBufs) & 1u, a, kErrTimeoutMma))) return false;
           if (sj >= 2 && !__all_sync(kFull, lwait(&bs.s_empty[sb], ((sj >> 1) - 1) & 1u, a, kErrTimeoutMma)))
             return false;
           fence_proxy_async_smem();
           tc_fence_after();
           const uint64_t kd = kdesc0 + (uint64_t)((kbuf * kKVTile) >> 4);
+          // two independent chains: head dims 0..127 into S columns sb*64 + 0..31,
+          // dims 128..255 into sb*64 + 32..63 (the softmax adds them)
 #pragma unroll
           for (int s = 0; s < 4; ++s)
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
-              tc_mma_bf16_ts_w(tmem + kTmemS + (uint32_t)(sb * kKB), tmem + kTmemQ + (uint32_t)(32 * s + 8 * kk),
-                               kd + (uint64_t)((s * kKVSub + kk * 32) >> 4), idesc_s, (s | kk) != 0);
+              tc_mma_bf16_ts_w(tmem + kTmemS + (uint32_t)(sb * 2 * kKB + (s >> 1) * kKB),
+                               tmem + kTmemQ + (uint32_t)(32 * s + 8 * kk),
+                               kd + (uint64_t)((s * kKVSub + kk * 32) >> 4), idesc_s, ((s & 1) | kk) != 0);
           tc_commit_w(&bs.s_full[sb]);
           tc_commit_w(&bs.k_empty[kbuf]);
           ++kj;
@@ -515,9 +637,9 @@ __device__ void role_mma(const LoopArgs &a, uint8_t *smem, Bars &bs, uint32_t tm
           return true;
         };
         auto issue_pv = [&](int j) -> bool {  // O += P(pj) V(vj)
-          const int vbuf = vj % 2, pb = pj % 2;
+          const int vbuf = vj % kKVBufs, pb = pj % 2;
           if (!__all_sync(kFull, lwait(&bs.p_full[pb], (pj / 2) & 1u, a, kErrTimeoutMma))) return false;
-          if (!__all_sync(kFull, lwait(&bs.v_full[vbuf], (vj / 2) & 1u, a, kErrTimeoutMma))) return false;
+          if (!__all_sync(kFull, lwait(&bs.v_full[vbuf], (vj / kKVBufs) & 1u, a, kErrTimeoutMma))) return false;
           fence_proxy_async_smem();
           tc_fence_after();
           const uint64_t pd = pdesc0 + (uint64_t)((pb * kPTile) >> 4);
@@ -548,21 +670,16 @@ __device__ void role_mma(const LoopArgs &a, uint8_t *smem, Bars &bs, uint32_t tm
 // ---- role: activation loader of GEMM units, K loader of attention units (warp 2) ------
 // and V loader of attention units (warp 3, is_v).
 __device__ void role_loader(const LoopArgs &a, uint8_t *smem, Bars &bs, bool is_v, int lane) {
-  const int total = a.N * stage_count(a);
+  const int total = total_stages(a);
   const uint32_t sbase = smem_u32(smem);
+  const int nas = a_slots(a);
+  const uint32_t asb = a_slot_bytes(a);
   uint32_t ai = 0, kj = 0, x_units = 0;
   bool ok = true;
-  if (lane == 0 && !is_v) {
-    tma_map_acquire(a.m_xn);
-    tma_map_acquire(a.m_att);
-    tma_map_acquire(a.m_act);
-    tma_map_acquire(a.m_aemb);
-    tma_map_acquire(a.m_uemb);
-  }
   // region X: wait until every earlier unit that used it has finished its MMAs
   auto take_x = [&]() -> bool {
     bool good = true;
-    if (lane == 0) good = x_acquire(bs, x_units, a, kErrTimeoutProducer);
+    if (lane == 0) good = smem_wait(&bs.x_done, x_units, a, kErrTimeoutProducer);
     ++x_units;
     good = __shfl_sync(kFull, (int)good, 0) != 0;
     __syncwarp();
@@ -571,40 +688,62 @@ __device__ void role_loader(const LoopArgs &a, uint8_t *smem, Bars &bs, bool is_
   for (int gs = 0; gs < total && ok; ++gs) {
     const StageInfo si = stage_at(a, gs);
     const int step0 = si.step == 0;
+    if (is_v) {  // the stage's gate first (this warp's own V loads of stage gs come after)
+      if (lane == 0) ok = poll_stage(a, bs, gs);
+      ok = __shfl_sync(kFull, (int)ok, 0) != 0;
+      if (!ok) break;
+    }
     if (loop_is_gemm(si.kind)) {
       const LoopGemm p = loop_gemm_plan(si.kind, a.grid);
-      const int U = p.nchunks * p.splits;
+      const int U = p.mtiles * p.ksplit;
       if (blockIdx.x >= U) continue;
-      int a_row0, M, out_row0;
-      gemm_rows(a, si.kind, step0, a_row0, M, out_row0);
-      (void)M;
-      (void)out_row0;
-      const CUtensorMap *amap = act_map(a, si.kind);
-      bool waited = false;
+      const bf16 *abase = act_tiles(a, si.kind);
+      const size_t kb_elems = (size_t)a.box_rows * 64;  // one K-block tile
+      if (si.kind == LK_QKV && !is_v && lane < 2 && a.P > 0) {
+        // this CTA's slice of the layer's prefix K (lane 0) / V (lane 1) into L2
+        const size_t bytes = (size_t)a.B * a.P * kHeadDim * 2;
+        const size_t slice = ((bytes + gridDim.x - 1) / gridDim.x + 15) & ~size_t(15);
+        const size_t off = (size_t)blockIdx.x * slice;
+        if (off < bytes) {
+          const uint8_t *base = reinterpret_cast<const uint8_t *>(lane ? a.cp->prefix_v[si.layer] : a.cp->prefix_k[si.layer]);
+          prefetch_l2(base + off, (uint32_t)(bytes - off < slice ? bytes - off : slice));
+        }
+      }
+      bool opened = false;
       for (int u = blockIdx.x; u < U && ok; u += gridDim.x) {
         ok = take_x();
         if (!ok) break;
         if (is_v) continue;
-        if (lane == 0) {
-          if (!waited) {
-            ok = wait_prev(a, gs) && !(si.gs == a.debug_stall_stage && !lpoll(a.done + gs, 1 << 30, a));
-            fence_proxy_async_global();
-            waited = true;
-          }
-          const GUnit g = gemm_unit(p, u);
-          for (int kb = g.kb0; kb < g.kb1 && ok; ++kb, ++ai) {
-            const int slot = ai % kASlots;
-            const uint32_t n = ai / kASlots;
-            if (n > 0 && !lwait(&bs.a_empty[slot], (n - 1) & 1u, a, kErrTimeoutProducer)) {
-              ok = false;
-              break;
-            }
-            mbar_arrive_expect_tx(&bs.a_full[slot], (uint32_t)a.box_rows * 128u);
-            tma_load_2d(smem + kOffA + slot * kASlotBytes, amap, kb * 64, a_row0, &bs.a_full[slot]);
-            bs.a_fills[slot] = n + 1;
-          }
+        if (!opened) {
+          ok = gate(bs, gs, a);
+          fence_proxy_async_global();  // the tiles were written through the generic proxy
+          if (lane == 0) LOOP_STAMP(gs, 4);
+          opened = true;
         }
-        ok = __all_sync(kFull, __shfl_sync(kFull, (int)ok, 0) != 0);
+        ok = __all_sync(kFull, ok);
+        if (!ok) break;
+        const GUnit g = gemm_unit(p, u);
+        const int nk = g.kb1 - g.kb0;
+        // lanes 0..3 copy one K-block tile each per round
+        for (int i0 = 0; i0 < nk && ok; i0 += 4) {
+          const int i = i0 + lane;
+          bool good = true;
+          if (lane < 4 && i < nk) {
+            const uint32_t f = ai + (uint32_t)i;
+            const int slot = f % nas;
+            const uint32_t n = f / nas;
+            if (n > 0) good = lwait(&bs.a_empty[slot], (n - 1) & 1u, a, kErrTimeoutProducer);
+            if (good) {
+              mbar_arrive_expect_tx(&bs.a_full[slot], asb);
+              bulk_load(smem_u32(smem + kOffA + slot * asb), abase + (size_t)(g.kb0 + i) * kb_elems, asb,
+                        &bs.a_full[slot]);
+              bs.a_fills[slot] = n + 1;
+            }
+          }
+          ok = __all_sync(kFull, good);
+        }
+        if (lane == 0) LOOP_STAMP(gs, 3);
+        ai += (uint32_t)nk;
       }
     } else if (si.kind == LK_ATTN) {
       const int U = attn_units(a, step0);
@@ -641,15 +780,15 @@ __device__ void role_loader(const LoopArgs &a, uint8_t *smem, Bars &bs, bool is_
           const int blk = t.blk0 + j;
           if (!sfx_ready && blk >= t.nbp) {  // suffix keys come from this step's QKV stage
             if (lane == 0) {
-              ok = wait_prev(a, gs);
+              ok = gate(bs, gs, a);
               fence_proxy_async_global();
             }
             ok = __all_sync(kFull, __shfl_sync(kFull, (int)ok, 0) != 0);
             if (!ok) break;
             sfx_ready = true;
           }
-          const int buf = kj % 2;
-          const uint32_t n = kj / 2;
+          const int buf = kj % kKVBufs;
+          const uint32_t n = kj / kKVBufs;
           if (n > 0) ok = __all_sync(kFull, lwait(&empty[buf], (n - 1) & 1u, a, kErrTimeoutProducer));
           if (!ok) break;
           load_kv_tile(blk, ring + buf * kKVTile, &full[buf], pmap, smap, pmap32, smap32, sfx_row0, pref, suf, t.nbp,
@@ -663,126 +802,314 @@ __device__ void role_loader(const LoopArgs &a, uint8_t *smem, Bars &bs, bool is_
   cp_async_wait<0>();
 }
 
-// ---- GEMM epilogues (one output row per thread, 16 columns) ------------------------------
-__device__ __forceinline__ float row_rstd64(const float *ss, int ld, int orow) {
+// ---- GEMM epilogues ---------------------------------------------------------------
+// rstd of output row `orow` from the fused-norm producer's per-m-tile sums of h^2.
+__device__ __forceinline__ float row_rstd(const float *ss, int ld, int orow) {
   float t = 0.f;
-#pragma unroll 8
+#pragma unroll
   for (int g = 0; g < kLoopNormSlots; ++g) t += ss[(size_t)g * ld + orow];
   return 1.0f / sqrtf(t / (float)kWidth + kRmsEps);
 }
+__device__ __forceinline__ const float *producer_gain(const LoopArgs &a, int kind, int layer) {
+  if (kind == LK_TOUT) return a.in_norm[0];
+  if (kind == LK_O) return a.post_norm[layer];
+  if (kind == LK_DOWN) return layer + 1 < a.L ? a.in_norm[layer + 1] : nullptr;
+  return nullptr;
+}
+__device__ __forceinline__ uint2 pack4(float a0, float a1, float a2, float a3) {
+  const __nv_bfloat162 p0 = __floats2bfloat162_rn(a0, a1), p1 = __floats2bfloat162_rn(a2, a3);
+  return make_uint2(*reinterpret_cast<const uint32_t *>(&p0), *reinterpret_cast<const uint32_t *>(&p1));
+}
+__device__ __forceinline__ void store_reps4(bf16 *buf, size_t off, size_t rep_stride, uint2 v) {
+#pragma unroll
+  for (int r = 0; r < kLoopReps; ++r) *reinterpret_cast<uint2 *>(buf + r * rep_stride + off) = v;
+}
+// RoPE position of output row `orow`: the state token sits at n_b, action j at n_b + 1 + j.
+__device__ __forceinline__ int rope_pos(const LoopArgs &a, int orow) {
+  if (orow < a.B) return a.nvalid[orow];
+  const int b = (orow - a.B) / a.H, j = (orow - a.B) % a.H;
+  return a.nvalid[b] + 1 + j;
+}
+__device__ __forceinline__ void add4(float4 &d, const float4 &x) {
+  d.x += x.x;
+  d.y += x.y;
+  d.z += x.z;
+  d.w += x.w;
+}
 
-struct EpiCtx {
-  int kind, layer, step, orow, b, j;
-  float rs;
-  int pos;
-};
-
-// Residual / bias producers with the fused RMSNorm outputs.
-__device__ __forceinline__ void epi_store16(const LoopArgs &a, const EpiCtx &c, int n, float (&v)[16]) {
-  const int orow = c.orow;
-  if (c.kind == LK_TIN) {
-    const float *vec = a.tvec + (size_t)c.step * kWidth + n;
-    float t[16];
+// Reduce + epilogue of tokens [t0, t1) of m-tile g.m (warps 4-7).  `stage` receives
+// the m-tile's partial tiles for the slice, split-major (split s, slice token j, 128
+// rows as 32 quads of 4 rows), from cp.async copies every thread has issued; every
+// output adds its splits in a fixed order, so the result does not depend on timing.
+// One warp per SM sub-partition runs this, so the items of a thread are unrolled with
+// independent registers (no shuffles or divergent branches) to overlap their latencies,
+// and their global operands load while the copies are in flight.
+//
+// Residual kinds (TOUT: bias; O, DOWN: residual), item (token, quad q = lane), a warp
+// per token: update h and, with a following norm, store bf16 h*(1+g) and the token's
+// sum of h^2 over the m-tile (norm slot m).  Paired kinds, item (token, pair quad):
+// rows 16i+e and 16i+8+e of the m-tile hold rotation pair (d, d+128) of one head for
+// QKV (the stored weight interleaves them) and gate / up of one hidden feature for GU,
+// so pair quad pq (i = pq >> 1, e = 4 (pq & 1) ..) reads quads 4i + (pq & 1) and that
+// + 2, scales both by the token's rstd, then rotates and stores q / k / v (QKV) or
+// stores GeGLU(g, u) (GU).  rstd_s / pos_s hold the slice's per-token rstd and RoPE
+// position (paired kinds).
+constexpr int kRedItems = 4;
+__device__ void reduce_unit(const LoopArgs &a, const StageInfo &si, const LoopGemm &p, const GUnit &g, int t0,
+                            int t1, int out_off, int et, const float4 *stage, const float *rstd_s, const int *pos_s,
+                            int gs) {
+  (void)gs;  // timeline stamps only
+  // the call's pointers and sizes in registers: read through `a` after every store
+  // (which may alias it, as far as the compiler can tell) they would be reloaded
+  const int kind = si.kind, layer = si.layer;
+  const int lane = et & 31, ks = p.ksplit, T = t1 - t0;
+  const int rb = a.box_rows, ss_ld = a.ss_ld, R = a.R;
+  const size_t rep_w = (size_t)a.rep_rows * kWidth, rep_m = (size_t)a.rep_rows * kMlp;
+  float *const hbuf = a.h;
+  bf16 *const xn = a.xn, *const act = a.act, *const qb = a.q, *const kbuf = a.ks, *const vbuf = a.vs;
+  const float *const tout_b = a.tout_b, *const rope = a.rope_tab;
+  const float4 zero = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (kind == LK_QKV || kind == LK_GU) {
+    const int items = T * 16, hd = g.m >> 1;
+    const bool rot = kind == LK_QKV && hd < kHeads + 1;
+    float4 c01[kRedItems], c23[kRedItems];
+    auto load_ops = [&](int it0) {
 #pragma unroll
-    for (int i = 0; i < 16; ++i) t[i] = silu_f(v[i] + vec[i]);
-    uint4 *dst = reinterpret_cast<uint4 *>(a.uemb + (size_t)orow * kWidth + n);
-    dst[0] = pack8(t);
-    dst[1] = pack8(t + 8);
-  } else if (c.kind == LK_TOUT || c.kind == LK_O || c.kind == LK_DOWN) {
-    float *hp = a.h + (size_t)orow * kWidth + n;
-    float4 *h4 = reinterpret_cast<float4 *>(hp);
-    if (c.kind == LK_TOUT) {
-      const float4 *b4 = reinterpret_cast<const float4 *>(a.tout_b + n);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float4 bb = b4[i];
-        v[4 * i] += bb.x; v[4 * i + 1] += bb.y; v[4 * i + 2] += bb.z; v[4 * i + 3] += bb.w;
-      }
-    } else {
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float4 hh = h4[i];
-        v[4 * i] += hh.x; v[4 * i + 1] += hh.y; v[4 * i + 2] += hh.z; v[4 * i + 3] += hh.w;
-      }
-    }
-#pragma unroll
-    for (int i = 0; i < 4; ++i) h4[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
-    const float *gain = c.kind == LK_TOUT ? a.in_norm[0]
-                        : c.kind == LK_O  ? a.post_norm[c.layer]
-                        : (c.layer + 1 < a.L ? a.in_norm[c.layer + 1] : nullptr);
-    if (gain) {  // fused RMSNorm producer: bf16(h * (1 + g)) and the group's sum of h^2
-      float *ss = c.kind == LK_O ? a.ss_m : a.ss_a;
-      float t[16], ssq = 0.f;
-      const float4 *g4 = reinterpret_cast<const float4 *>(gain + n);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float4 gg = g4[i];
-        ssq = fmaf(v[4 * i], v[4 * i], ssq);
-        ssq = fmaf(v[4 * i + 1], v[4 * i + 1], ssq);
-        ssq = fmaf(v[4 * i + 2], v[4 * i + 2], ssq);
-        ssq = fmaf(v[4 * i + 3], v[4 * i + 3], ssq);
-        t[4 * i] = v[4 * i] * (1.0f + gg.x);
-        t[4 * i + 1] = v[4 * i + 1] * (1.0f + gg.y);
-        t[4 * i + 2] = v[4 * i + 2] * (1.0f + gg.z);
-        t[4 * i + 3] = v[4 * i + 3] * (1.0f + gg.w);
-      }
-      uint4 *xd = reinterpret_cast<uint4 *>(a.xn + (size_t)orow * kWidth + n);
-      xd[0] = pack8(t);
-      xd[1] = pack8(t + 8);
-      ss[(size_t)(n >> 4) * a.ss_ld + orow] = ssq;
-    }
-  } else if (c.kind == LK_QKV) {
-    // group gc = 8 rotation pairs (ib .. ib+7, +128) of head hd (8 = k, 9 = v)
-    const int gc = n >> 4, hd = gc >> 4, ib = (gc & 15) * 8;
-    float lo[8], hi[8];
-#pragma unroll
-    for (int w = 0; w < 8; ++w) {
-      lo[w] = v[w] * c.rs;
-      hi[w] = v[8 + w] * c.rs;
-    }
-    if (hd < kHeads + 1) {
-      const float4 *tab = reinterpret_cast<const float4 *>(a.rope_tab + ((size_t)c.pos * (kHeadDim / 2) + ib) * 2);
-#pragma unroll
-      for (int w2 = 0; w2 < 4; ++w2) {
-        const float4 t = tab[w2];
-#pragma unroll
-        for (int h2 = 0; h2 < 2; ++h2) {
-          const int w = 2 * w2 + h2;
-          const float cs = h2 ? t.z : t.x, sn = h2 ? t.w : t.y;
-          const float x0 = lo[w], x1 = hi[w];
-          lo[w] = x0 * cs - x1 * sn;
-          hi[w] = x1 * cs + x0 * sn;
+      for (int i = 0; i < kRedItems; ++i) {
+        const int it = it0 + 128 * i;
+        c01[i] = c23[i] = zero;
+        if (rot && it < items) {
+          const int pq = it & 15, d0 = ((g.m & 1) * 8 + (pq >> 1)) * 8 + (pq & 1) * 4;
+          const float4 *tab = reinterpret_cast<const float4 *>(rope + ((size_t)pos_s[it >> 4] * (kHeadDim / 2) + d0) * 2);
+          c01[i] = tab[0];
+          c23[i] = tab[1];
         }
       }
-    }
-    bf16 *dst;
-    if (hd < kHeads)
-      dst = a.q + (size_t)orow * kQDim + hd * kHeadDim + ib;
-    else
-      dst = (hd == kHeads ? a.ks : a.vs) + ((size_t)c.layer * a.R + orow) * kHeadDim + ib;
-    *reinterpret_cast<uint4 *>(dst) = pack8(lo);
-    *reinterpret_cast<uint4 *>(dst + kHeadDim / 2) = pack8(hi);
-  } else {  // LK_GU: 8 gate then the matching 8 up features
-    float t[8];
+    };
+    load_ops(et);
+    cp_async_wait<0>();
+    epi_bar();  // every thread's staging copies have landed
+    for (int it0 = et; it0 < items; it0 += 128 * kRedItems) {
+      if (it0 != et) load_ops(it0);
+      float4 lo4[kRedItems], hi4[kRedItems];
 #pragma unroll
-    for (int w = 0; w < 8; ++w) t[w] = gelu_tanh_f(v[w] * c.rs) * (v[8 + w] * c.rs);
-    *reinterpret_cast<uint4 *>(a.act + (size_t)orow * kMlp + (n >> 4) * 8) = pack8(t);
+      for (int i = 0; i < kRedItems; ++i) {
+        const int it = it0 + 128 * i;
+        lo4[i] = hi4[i] = zero;
+        if (it >= items) continue;
+        const int j = it >> 4, pq = it & 15, ql = (pq >> 1) * 4 + (pq & 1);
+        const float4 *st = stage + (size_t)j * 32;
+        for (int sp = 0; sp < ks; ++sp) {
+          add4(lo4[i], st[(size_t)sp * T * 32 + ql]);
+          add4(hi4[i], st[(size_t)sp * T * 32 + ql + 2]);
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < kRedItems; ++i) {
+        const int it = it0 + 128 * i;
+        if (it >= items) continue;
+        const int j = it >> 4, pq = it & 15, orow = t0 + j + out_off;
+        const int gq = pq >> 1, e0 = (pq & 1) * 4;
+        const float rs = rstd_s[j];
+        float lo[4] = {lo4[i].x * rs, lo4[i].y * rs, lo4[i].z * rs, lo4[i].w * rs};
+        float hi[4] = {hi4[i].x * rs, hi4[i].y * rs, hi4[i].z * rs, hi4[i].w * rs};
+        if (kind == LK_GU) {
+          float t[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) t[q] = gelu_tanh_fast(lo[q]) * hi[q];
+          store_reps4(act, tiled_off(orow, g.m * 64 + gq * 8 + e0, rb), rep_m, pack4(t[0], t[1], t[2], t[3]));
+          continue;
+        }
+        if (rot) {
+          const float cs[4] = {c01[i].x, c01[i].z, c23[i].x, c23[i].z}, sn[4] = {c01[i].y, c01[i].w, c23[i].y, c23[i].w};
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const float x0 = lo[q], x1 = hi[q];
+            lo[q] = x0 * cs[q] - x1 * sn[q];
+            hi[q] = x1 * cs[q] + x0 * sn[q];
+          }
+        }
+        const int d0 = ((g.m & 1) * 8 + gq) * 8 + e0;
+        bf16 *dst = hd < kHeads ? qb + (size_t)orow * kQDim + hd * kHeadDim + d0
+                                : (hd == kHeads ? kbuf : vbuf) + ((size_t)layer * R + orow) * kHeadDim + d0;
+        *reinterpret_cast<uint2 *>(dst) = pack4(lo[0], lo[1], lo[2], lo[3]);
+        *reinterpret_cast<uint2 *>(dst + kHeadDim / 2) = pack4(hi[0], hi[1], hi[2], hi[3]);
+      }
+    }
+    return;
+  }
+  const int items = T * 32;
+  const float *gain = producer_gain(a, kind, layer);
+  float *ss = kind == LK_O ? a.ss_m : a.ss_a;
+  const int n = g.m * 128 + 4 * lane;  // the item's 4 features
+  float4 ex[kRedItems], gx[kRedItems];
+  auto load_ops = [&](int it0) {
+#pragma unroll
+    for (int i = 0; i < kRedItems; ++i) {
+      const int it = it0 + 128 * i;
+      ex[i] = gx[i] = zero;
+      if (it >= items) continue;
+      const int orow = t0 + (it >> 5) + out_off;
+      ex[i] = kind == LK_TOUT ? *reinterpret_cast<const float4 *>(tout_b + n)
+                              : *reinterpret_cast<const float4 *>(hbuf + (size_t)orow * kWidth + n);
+      if (gain) gx[i] = *reinterpret_cast<const float4 *>(gain + n);
+    }
+  };
+  load_ops(et);
+  cp_async_wait<0>();
+  epi_bar();  // every thread's staging copies have landed
+  for (int it0 = et; it0 < items; it0 += 128 * kRedItems) {
+    if (it0 != et) load_ops(it0);
+    float4 v4[kRedItems];
+#pragma unroll
+    for (int i = 0; i < kRedItems; ++i) {
+      const int it = it0 + 128 * i;
+      v4[i] = zero;
+      if (it >= items) continue;
+      // splits 0, 2, 4 .. and 1, 3, 5 .. in two chains, then their sum (a fixed order)
+      const float4 *st = stage + (size_t)(it >> 5) * 32 + lane;
+      float4 odd = zero;
+      int sp = 0;
+      for (; sp + 1 < ks; sp += 2) {
+        add4(v4[i], st[(size_t)sp * T * 32]);
+        add4(odd, st[(size_t)(sp + 1) * T * 32]);
+      }
+      if (sp < ks) add4(v4[i], st[(size_t)sp * T * 32]);
+      add4(v4[i], odd);
+    }
+#pragma unroll
+    for (int i = 0; i < kRedItems; ++i) {
+      const int it = it0 + 128 * i;
+      if (it >= items) continue;  // warp-uniform: items is a multiple of 32
+      const int orow = t0 + (it >> 5) + out_off;
+      float4 v = v4[i];
+      add4(v, ex[i]);
+      *reinterpret_cast<float4 *>(hbuf + (size_t)orow * kWidth + n) = v;
+      if (gain) {
+        const float4 gg = gx[i];
+        store_reps4(xn, tiled_off(orow, n, rb), rep_w,
+                    pack4(v.x * (1.0f + gg.x), v.y * (1.0f + gg.y), v.z * (1.0f + gg.z), v.w * (1.0f + gg.w)));
+        const float sq = warp_sum(fmaf(v.x, v.x, fmaf(v.y, v.y, fmaf(v.z, v.z, v.w * v.w))));
+        if (lane == 0) ss[(size_t)g.m * ss_ld + orow] = sq;
+      }
+    }
   }
 }
 
-// ---- role: epilogues, softmax and small stages (warps 4-7) -----------------------------
+// TIN unit c (warps 4-7): columns [8c, 8c + 8) of the step's action-time MLP input
+// for every action row, u = silu(w_xa x + tvec[k]); thread et takes row et (x_1 at
+// step 0, else the integrated x).
+__device__ __forceinline__ void tin_unit(const LoopArgs &a, int cidx, int k, int et) {
+  const int A = a.A, BH = a.B * a.H, n0 = cidx * 8;
+  const float *xsrc = k == 0 ? a.cp->x1 : a.xw;
+  const float *tv = a.tvec + (size_t)k * kWidth + n0;
+  for (int r = et; r < BH; r += 128) {
+    float u[8];
+#pragma unroll
+    for (int o = 0; o < 8; ++o) u[o] = tv[o];
+    const float4 *xr = reinterpret_cast<const float4 *>(xsrc + (size_t)r * A);
+#pragma unroll 4
+    for (int j4 = 0; j4 < A / 4; ++j4) {
+      const float4 xv = xr[j4];
+#pragma unroll
+      for (int o = 0; o < 8; ++o) {
+        const float4 wv = reinterpret_cast<const float4 *>(a.w_xa + (size_t)(n0 + o) * A)[j4];
+        u[o] = fmaf(wv.x, xv.x, u[o]);
+        u[o] = fmaf(wv.y, xv.y, u[o]);
+        u[o] = fmaf(wv.z, xv.z, u[o]);
+        u[o] = fmaf(wv.w, xv.w, u[o]);
+      }
+    }
+#pragma unroll
+    for (int o = 0; o < 8; ++o) u[o] = silu_f(u[o]);
+    store_reps(a.uemb, tiled_off(r, n0, a.box_rows), (size_t)a.rep_rows * kWidth, pack8(u));
+  }
+}
+
+// XOUT unit (warps 4-7): action row i, outputs [16 ch, 16 ch + 16): final RMSNorm of
+// the row, v = action_out_proj (fp32), velocity (x-prediction: v - x_1), x <- x +
+// dt v (x_0 on the last step).  Warp w takes outputs 16 ch + w + 4 o.
+__device__ __forceinline__ void xout_unit(const LoopArgs &a, Bars &bs, float *yrow, int i, int ch, int k, int et) {
+  const int warp = et >> 5, lane = et & 31;
+  const int A = a.A;
+  float xo[4], x1o[4], bo[4];
+#pragma unroll
+  for (int o = 0; o < 4; ++o) {
+    const int aa = ch * 16 + warp + 4 * o;
+    xo[o] = x1o[o] = bo[o] = 0.f;
+    if (aa < A) {
+      xo[o] = a.xw[(size_t)i * A + aa];
+      bo[o] = a.aout_b[aa];
+      if (a.x_pred) x1o[o] = a.cp->x1[(size_t)i * A + aa];
+    }
+  }
+  const float4 *src = reinterpret_cast<const float4 *>(a.h + (size_t)(a.B + i) * kWidth) + et * 2;
+  const float4 *g4 = reinterpret_cast<const float4 *>(a.fnorm) + et * 2;
+  const float4 x0 = src[0], x1 = src[1], g0 = g4[0], g1 = g4[1];
+  float ss = x0.x * x0.x + x0.y * x0.y + x0.z * x0.z + x0.w * x0.w + x1.x * x1.x + x1.y * x1.y + x1.z * x1.z +
+             x1.w * x1.w;
+  ss = warp_sum(ss);
+  if (lane == 0) bs.red[warp] = ss;
+  epi_bar();
+  const float tot = (bs.red[0] + bs.red[1]) + (bs.red[2] + bs.red[3]);
+  const float inv = 1.0f / sqrtf(tot / (float)kWidth + kRmsEps);
+  float4 *y4 = reinterpret_cast<float4 *>(yrow) + et * 2;
+  y4[0] = make_float4((x0.x * inv) * (1.0f + g0.x), (x0.y * inv) * (1.0f + g0.y), (x0.z * inv) * (1.0f + g0.z),
+                      (x0.w * inv) * (1.0f + g0.w));
+  y4[1] = make_float4((x1.x * inv) * (1.0f + g1.x), (x1.y * inv) * (1.0f + g1.y), (x1.z * inv) * (1.0f + g1.z),
+                      (x1.w * inv) * (1.0f + g1.w));
+  epi_bar();
+  float dt;
+  if (a.linspace)
+    dt = (float)((double)(k + 1) / (double)a.N) - (float)((double)k / (double)a.N);
+  else
+    dt = (float)(-1.0 / (double)a.N);
+  const float4 *yr = reinterpret_cast<const float4 *>(yrow);
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
+  for (int c4 = lane; c4 < kWidth / 4; c4 += 32) {
+    const float4 yv = yr[c4];
+#pragma unroll
+    for (int o = 0; o < 4; ++o) {
+      const int aa = ch * 16 + warp + 4 * o;
+      if (aa < A) {
+        const float4 wv = reinterpret_cast<const float4 *>(a.aout_w + (size_t)aa * kWidth)[c4];
+        acc[o] = fmaf(wv.x, yv.x, acc[o]);
+        acc[o] = fmaf(wv.y, yv.y, acc[o]);
+        acc[o] = fmaf(wv.z, yv.z, acc[o]);
+        acc[o] = fmaf(wv.w, yv.w, acc[o]);
+      }
+    }
+  }
+#pragma unroll
+  for (int o = 0; o < 4; ++o) acc[o] = warp_sum(acc[o]);
+  if (lane == 0) {
+#pragma unroll
+    for (int o = 0; o < 4; ++o) {
+      const int aa = ch * 16 + warp + 4 * o;
+      if (aa < A) {
+        float v = acc[o] + bo[o];
+        if (a.x_pred) v -= x1o[o];  // output is the clean action: velocity = x_hat - noise
+        const float xn = __fadd_rn(xo[o], __fmul_rn(dt, v));
+        a.xw[(size_t)i * A + aa] = xn;
+        if (k == a.N - 1) a.cp->x0[(size_t)i * A + aa] = xn;
+      }
+    }
+  }
+  epi_bar();  // yrow and red are reused by the next unit
+}
+
+// ---- role: epilogues, softmax and row stages (warps 4-7) -------------------------------
 __device__ void role_epi(const LoopArgs &a, uint8_t *smem, Bars &bs, uint32_t tmem, int et) {
-  const int total = a.N * stage_count(a);
+  const int total = total_stages(a);
   const int warp = et >> 5, lane = et & 31;
   const uint32_t t_lane = (uint32_t)(warp * 32) << 16;
-  uint32_t acc_n = 0, sj = 0, pj = 0, pvj = 0;
+  uint32_t acc_n = 0, sj = 0, pj = 0, pvj = 0, tmem_units = 0;
   bool ok = true;
-  float *yrow = reinterpret_cast<float *>(smem + kOffBar + ((sizeof(Bars) + 127) / 128) * 128);
-  auto poll_prev = [&](int gs) -> bool {
-    bool good = true;
-    if (lane == 0) good = wait_prev(a, gs) && !(gs == a.debug_stall_stage && !lpoll(a.done + gs, 1 << 30, a));
-    good = __shfl_sync(kFull, (int)good, 0) != 0;
-    __syncwarp();
+  float *yrow = reinterpret_cast<float *>(smem + kOffRow);
+  auto open = [&](int gs) -> bool {
+    const bool good = gate(bs, gs, a);
+    LOOP_STAMP(gs, 0);
     return good;
   };
   for (int gs = 0; gs < total && ok; ++gs) {
@@ -790,106 +1117,87 @@ __device__ void role_epi(const LoopArgs &a, uint8_t *smem, Bars &bs, uint32_t tm
     const int step0 = si.step == 0;
     if (loop_is_gemm(si.kind)) {
       const LoopGemm p = loop_gemm_plan(si.kind, a.grid);
-      const int U = p.nchunks * p.splits;
+      const int U = p.mtiles * p.ksplit;
       if (blockIdx.x >= U) continue;
-      ok = poll_prev(gs);
+      ok = open(gs);
       if (!ok) break;
-      int a_row0, M, out_row0;
-      gemm_rows(a, si.kind, step0, a_row0, M, out_row0);
-      const int r = et;
-      const bool valid = r < M;
-      EpiCtx c;
-      c.kind = si.kind;
-      c.layer = si.layer;
-      c.step = si.step;
-      c.orow = out_row0 + r;
-      c.rs = 1.f;
-      c.pos = 0;
-      if (valid && (si.kind == LK_QKV || si.kind == LK_GU))
-        c.rs = row_rstd64(si.kind == LK_QKV ? a.ss_a : a.ss_m, a.ss_ld, c.orow);
-      if (valid && si.kind == LK_QKV) {
-        int b, j;
-        if (c.orow < a.B) {
-          b = c.orow;
-          j = 0;
-        } else {
-          b = (c.orow - a.B) / a.H;
-          j = 1 + (c.orow - a.B) % a.H;
-        }
-        c.pos = a.nvalid[b] + j;
-      }
+      int r_lo, r_hi, out_off;
+      gemm_rows(a, si.kind, step0, r_lo, r_hi, out_off);
+      const int NT = a.box_rows;
+      // U <= grid (at most 64 m-tiles, at least 128 CTAs): every unit of an m-tile
+      // runs on its own CTA, so waiting for the m-tile's partials cannot wait on itself
       for (int u = blockIdx.x; u < U && ok; u += gridDim.x) {
         const GUnit g = gemm_unit(p, u);
         ok = __all_sync(kFull, lwait(&bs.acc_full, acc_n & 1u, a, kErrTimeoutEpilogue));
         if (!ok) break;
         ++acc_n;
         tc_fence_after();
-        if (et == 0) x_release(bs);  // the unit's MMAs have completed
-        if (p.splits == 1) {
-          for (int gi = 0; gi < g.w; gi += 16) {
-            float v[16];
-            tmem_ld_x16(tmem + t_lane + kTmemAcc + (uint32_t)gi, v);
-            if (valid) epi_store16(a, c, g.n0 + gi, v);
-          }
-          tc_fence_before();
-          fence_proxy_async_global();
-          epi_bar();
-          if (et == 0) {
-            mbar_arrive(&bs.acc_empty);
-            release(a, gs);
-          }
-        } else {
-          float *mine = a.gpart + ((size_t)(g.chunk * p.splits + g.split) * 128 + r) * 64;
-          for (int gi = 0; gi < g.w; gi += 16) {
-            float v[16];
-            tmem_ld_x16(tmem + t_lane + kTmemAcc + (uint32_t)gi, v);
-            if (valid) {
-              float4 *d4 = reinterpret_cast<float4 *>(mine + gi);
+        LOOP_STAMP(gs, 1);
+        // partial tile, token-major: row et of the m-tile for the stored tokens
+        float *mine = a.gpart + (size_t)u * 128 * NT;
+        for (int c0 = r_lo & ~15; c0 < r_hi; c0 += 16) {
+          float v[16];
+          tmem_ld_x16(tmem + t_lane + kTmemAcc + (uint32_t)c0, v);
 #pragma unroll
-              for (int i = 0; i < 4; ++i) d4[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+          for (int i = 0; i < 16; ++i) __stcg(mine + (size_t)(c0 + i) * 128 + et, v[i]);
+        }
+        tc_fence_before();
+        epi_bar();
+        LOOP_STAMP(gs, 8);
+        ++tmem_units;
+        int *cnt = a.mt_cnt + (size_t)gs * kLoopMaxMtiles + g.m;
+        if (et == 0) {
+          smem_publish(&bs.tmem_done, tmem_units);
+          red_release_add(cnt, 1);
+        }
+        int t0, t1;
+        red_slice(r_lo, r_hi, p.ksplit, g.s, t0, t1);
+        if (t0 < t1) {
+          // per-token rstd / RoPE position of the slice while the other splits finish
+          float *rstd_s = yrow;
+          int *pos_s = reinterpret_cast<int *>(yrow + kLoopMaxRows);
+          if (si.kind == LK_QKV || si.kind == LK_GU) {
+            const float *ssn = si.kind == LK_QKV ? a.ss_a : a.ss_m;
+            for (int j = et; j < t1 - t0; j += 128) {
+              const int orow = t0 + j + out_off;
+              rstd_s[j] = row_rstd(ssn, a.ss_ld, orow);
+              pos_s[j] = si.kind == LK_QKV ? rope_pos(a, orow) : 0;
             }
           }
-          tc_fence_before();
-          __threadfence();
+          // once every split's partial is stored, every thread copies 16-byte chunks of
+          // the slice of each split into region X (free: this unit's MMAs have
+          // completed, and region X is handed on only after the reduce)
+          if (et == 0) bs.last = gwait(cnt, p.ksplit, a, kErrTimeoutEpilogue) ? 1 : 0;
           epi_bar();
-          if (et == 0) {
-            mbar_arrive(&bs.acc_empty);
-            const int prev = atomicAdd(a.counters + g.chunk, 1);
-            bs.last = prev == p.splits - 1;
-          }
-          epi_bar();
-          if (bs.last) {
-            __threadfence();
-            if (valid) {
-              const float *base = a.gpart + ((size_t)g.chunk * p.splits * 128 + r) * 64;
-              for (int gi = 0; gi < g.w; gi += 16) {
-                float v[16];
-#pragma unroll
-                for (int i = 0; i < 16; ++i) v[i] = 0.f;
-                for (int s = 0; s < p.splits; ++s) {
-                  const float4 *p4 = reinterpret_cast<const float4 *>(base + (size_t)s * 128 * 64 + gi);
-#pragma unroll
-                  for (int i = 0; i < 4; ++i) {
-                    const float4 t = __ldcg(p4 + i);
-                    v[4 * i] += t.x; v[4 * i + 1] += t.y; v[4 * i + 2] += t.z; v[4 * i + 3] += t.w;
-                  }
-                }
-                epi_store16(a, c, g.n0 + gi, v);
-              }
+          ok = bs.last != 0;
+          if (!ok) break;
+          {
+            const int per_split = (t1 - t0) * 32, chunks = p.ksplit * per_split;
+            const float4 *src0 = reinterpret_cast<const float4 *>(a.gpart + (size_t)g.m * p.ksplit * NT * 128) + t0 * 32;
+            const uint32_t dst0 = smem_u32(smem + kOffX);
+            for (int c = et; c < chunks; c += 128) {
+              const int sp = c / per_split;
+              cp_async16(dst0 + (uint32_t)c * 16u, src0 + (size_t)sp * NT * 32 + (c - sp * per_split), true);
             }
-            fence_proxy_async_global();
-            epi_bar();
-            if (et == 0) {
-              a.counters[g.chunk] = 0;  // ready for the next split-K stage
-              release(a, gs);
-            }
+            cp_async_commit();
           }
+          LOOP_STAMP(gs, 7);
+          reduce_unit(a, si, p, g, t0, t1, out_off, et, reinterpret_cast<const float4 *>(smem + kOffX), rstd_s, pos_s, gs);
+          LOOP_STAMP(gs, 10);
+          fence_proxy_async_global();  // outputs are read by bulk copies in the next stage
+        }
+        epi_bar();
+        LOOP_STAMP(gs, 11);
+        if (et == 0) {
+          x_release(bs);  // region X: the unit's MMAs and its reduce are done
+          LOOP_STAMP(gs, 2);
+          release(a, gs);
         }
       }
     } else if (si.kind == LK_ATTN) {
       const int U = attn_units(a, step0);
       if (blockIdx.x >= U) continue;
-      ok = poll_prev(gs);  // q of this step's QKV stage
+      ok = open(gs);  // q of this step's QKV stage
       if (!ok) break;
       const int Tq = step0 ? a.H + 1 : a.H;
       const int nrows = kHeads * Tq;
@@ -909,31 +1217,45 @@ __device__ void role_epi(const LoopArgs &a, uint8_t *smem, Bars &bs, uint32_t tm
         const int sfx_state = sfx_base + a.H;
         float m_used = -INFINITY, l = 0.f;
         if (t.nb > 0) {
-          // Q row -> TMEM lane et, columns kTmemQ.. (two bf16 per 32-bit column)
+          // Q row -> TMEM lane et, columns kTmemQ.. (two bf16 per 32-bit column); two
+          // batches of 16 independent 16-byte loads
           const uint4 *src = reinterpret_cast<const uint4 *>(a.q + (size_t)tok * kQDim + head * kHeadDim);
 #pragma unroll 1
-          for (int cc = 0; cc < 4; ++cc) {
-            float v[32];
+          for (int hb = 0; hb < 2; ++hb) {
+            uint4 qq[16];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              const uint4 uu = row_ok ? src[cc * 8 + e] : make_uint4(0, 0, 0, 0);
-              v[4 * e] = __uint_as_float(uu.x);
-              v[4 * e + 1] = __uint_as_float(uu.y);
-              v[4 * e + 2] = __uint_as_float(uu.z);
-              v[4 * e + 3] = __uint_as_float(uu.w);
+            for (int e = 0; e < 16; ++e) qq[e] = row_ok ? src[hb * 16 + e] : make_uint4(0, 0, 0, 0);
+#pragma unroll
+            for (int cc = 0; cc < 2; ++cc) {
+              float v[32];
+#pragma unroll
+              for (int e = 0; e < 8; ++e) {
+                v[4 * e] = __uint_as_float(qq[cc * 8 + e].x);
+                v[4 * e + 1] = __uint_as_float(qq[cc * 8 + e].y);
+                v[4 * e + 2] = __uint_as_float(qq[cc * 8 + e].z);
+                v[4 * e + 3] = __uint_as_float(qq[cc * 8 + e].w);
+              }
+              tmem_st_32x32b_x32(tmem + t_lane + kTmemQ + 32 * (hb * 2 + cc), v);
             }
-            tmem_st_32x32b_x32(tmem + t_lane + kTmemQ + 32 * cc, v);
           }
           tc_fence_before();
           mbar_arrive(&bs.q_full);
+          LOOP_STAMP(gs, 1);
           const uint32_t pv0 = pvj;  // global index of this unit's first P.V
           for (int j = 0; j < t.nb && ok; ++j, ++sj, ++pj) {
             const int sb = sj & 1, pb = pj & 1;
             ok = __all_sync(kFull, lwait(&bs.s_full[sb], (sj >> 1) & 1u, a, kErrTimeoutEpilogue));
             if (!ok) break;
             tc_fence_after();
+            if (j == 0) LOOP_STAMP(gs, 3);
             float sv[32];
-            tmem_ld_32x32b_x32(tmem + t_lane + kTmemS + sb * kKB, sv);
+            {
+              float s2[32];
+              tmem_ld_32x32b_x32(tmem + t_lane + kTmemS + sb * 2 * kKB, sv);
+              tmem_ld_32x32b_x32(tmem + t_lane + kTmemS + sb * 2 * kKB + kKB, s2);
+#pragma unroll
+              for (int i = 0; i < 32; ++i) sv[i] += s2[i];
+            }
             tc_fence_before();
             mbar_arrive(&bs.s_empty[sb]);
             const int kbase = (t.blk0 + j) * kKB;
@@ -962,7 +1284,7 @@ __device__ void role_epi(const LoopArgs &a, uint8_t *smem, Bars &bs, uint32_t tm
               l *= alpha;
               if (j >= 1) {  // O holds P.V of this unit's blocks < j: wait for the last of them
                 const uint32_t g = pj - 1;
-                ok = __all_sync(kFull, lwait(&bs.pv_done[g % 2], (g / 2) & 1u, a, kErrTimeoutEpilogue));
+                ok = __all_sync(kFull, lwait(&bs.pv_done[g % kKVBufs], (g / kKVBufs) & 1u, a, kErrTimeoutEpilogue));
                 if (!ok) break;
                 tc_fence_after();
                 for (int c0 = 0; c0 < kHeadDim; c0 += 32) {
@@ -978,7 +1300,7 @@ __device__ void role_epi(const LoopArgs &a, uint8_t *smem, Bars &bs, uint32_t tm
             }
             if (pj >= 2) {  // P buffer pb was last read by P.V number pj - 2 (this unit's or the last one's)
               const uint32_t g = pj - 2;
-              ok = __all_sync(kFull, lwait(&bs.pv_done[g % 2], (g / 2) & 1u, a, kErrTimeoutEpilogue));
+              ok = __all_sync(kFull, lwait(&bs.pv_done[g % kKVBufs], (g / kKVBufs) & 1u, a, kErrTimeoutEpilogue));
               if (!ok) break;
             }
             {
@@ -1005,16 +1327,16 @@ __device__ void role_epi(const LoopArgs &a, uint8_t *smem, Bars &bs, uint32_t tm
           }
           if (ok) {
             const uint32_t g = pv0 + t.nb - 1;
-            ok = __all_sync(kFull, lwait(&bs.pv_done[g % 2], (g / 2) & 1u, a, kErrTimeoutEpilogue));
+            ok = __all_sync(kFull, lwait(&bs.pv_done[g % kKVBufs], (g / kKVBufs) & 1u, a, kErrTimeoutEpilogue));
           }
           pvj = pv0 + t.nb;
           tc_fence_after();
         }
         if (et == 0) x_release(bs);  // every MMA of the unit has completed
         if (!ok) break;
+        LOOP_STAMP(gs, 7);
         const float inv_l = l > 0.f ? 1.0f / l : 0.f;
         if (a.attn_splits == 1) {
-          bf16 *dst = a.att + (size_t)tok * kQDim + head * kHeadDim;
           for (int c0 = 0; c0 < kHeadDim; c0 += 32) {
             float v[32];
             if (t.nb > 0) {
@@ -1027,9 +1349,10 @@ __device__ void role_epi(const LoopArgs &a, uint8_t *smem, Bars &bs, uint32_t tm
               float w32[32];
 #pragma unroll
               for (int e = 0; e < 32; ++e) w32[e] = v[e] * inv_l;
-              uint4 *d4 = reinterpret_cast<uint4 *>(dst + c0);
 #pragma unroll
-              for (int e = 0; e < 4; ++e) d4[e] = pack8(w32 + 8 * e);
+              for (int e = 0; e < 4; ++e)
+                store_reps(a.att, tiled_off(tok, head * kHeadDim + c0 + 8 * e, a.box_rows),
+                           (size_t)a.rep_rows * kQDim, pack8(w32 + 8 * e));
             }
           }
         } else {
@@ -1057,12 +1380,17 @@ __device__ void role_epi(const LoopArgs &a, uint8_t *smem, Bars &bs, uint32_t tm
         tc_fence_before();
         fence_proxy_async_global();
         epi_bar();
-        if (et == 0) release(a, gs);
+        ++tmem_units;
+        if (et == 0) {
+          smem_publish(&bs.tmem_done, tmem_units);  // O has been read out
+          LOOP_STAMP(gs, 2);
+          release(a, gs);
+        }
       }
     } else if (si.kind == LK_COMBINE) {
       const int nc = combine_ctas(a, step0);
       if (blockIdx.x >= nc) continue;
-      ok = poll_prev(gs);
+      ok = open(gs);
       if (!ok) break;
       const int Tq = step0 ? a.H + 1 : a.H;
       const int nrows = kHeads * Tq, qps = q_tiles(a, step0), items = a.B * nrows;
@@ -1072,21 +1400,22 @@ __device__ void role_epi(const LoopArgs &a, uint8_t *smem, Bars &bs, uint32_t tm
         if (it >= items) continue;
         const int b = it / nrows, qi = it % nrows, ti = qi / 128, qr = qi % 128;
         const size_t prow0 = ((size_t)(b * qps + ti) * S) * 128 + qr;
-        float M = -INFINITY;
-        for (int s = 0; s < S; ++s) {
-          const size_t pr = prow0 + (size_t)s * 128;
-          if (__ldcg(a.part_ml + 2 * pr + 1) > 0.f) M = fmaxf(M, __ldcg(a.part_ml + 2 * pr));
+        // lane s < S holds split s's (m, l); the block's max and weights by shuffles
+        float ms = -INFINITY, lsv = 0.f;
+        if (lane < S) {
+          ms = __ldcg(a.part_ml + 2 * (prow0 + (size_t)lane * 128));
+          lsv = __ldcg(a.part_ml + 2 * (prow0 + (size_t)lane * 128) + 1);
         }
-        float den = 0.f, acc[8];
+        const float M = warp_max(lsv > 0.f ? ms : -INFINITY);
+        const float wl = lsv > 0.f ? lsv * ex2_approx(ms - M) : 0.f;
+        const float den = warp_sum(wl);
+        float acc[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) acc[e] = 0.f;
         for (int s = 0; s < S; ++s) {
-          const size_t pr = prow0 + (size_t)s * 128;
-          const float ms = __ldcg(a.part_ml + 2 * pr), ls = __ldcg(a.part_ml + 2 * pr + 1);
-          if (!(ls > 0.f)) continue;
-          const float wgt = ls * ex2_approx(ms - M);
-          den += wgt;
-          const float4 *src = reinterpret_cast<const float4 *>(a.part_o + pr * kHeadDim + lane * 8);
+          const float wgt = __shfl_sync(kFull, wl, s);
+          if (wgt == 0.f) continue;
+          const float4 *src = reinterpret_cast<const float4 *>(a.part_o + (prow0 + (size_t)s * 128) * kHeadDim + lane * 8);
           const float4 x0 = __ldcg(src), x1 = __ldcg(src + 1);
           acc[0] = fmaf(wgt, x0.x, acc[0]); acc[1] = fmaf(wgt, x0.y, acc[1]);
           acc[2] = fmaf(wgt, x0.z, acc[2]); acc[3] = fmaf(wgt, x0.w, acc[3]);
@@ -1098,97 +1427,39 @@ __device__ void role_epi(const LoopArgs &a, uint8_t *smem, Bars &bs, uint32_t tm
         const float inv = den > 0.f ? 1.0f / den : 0.f;
 #pragma unroll
         for (int e = 0; e < 8; ++e) acc[e] *= inv;
-        *reinterpret_cast<uint4 *>(a.att + (size_t)tok * kQDim + hd * kHeadDim + lane * 8) = pack8(acc);
+        store_reps(a.att, tiled_off(tok, hd * kHeadDim + lane * 8, a.box_rows), (size_t)a.rep_rows * kQDim,
+                   pack8(acc));
       }
       fence_proxy_async_global();
       epi_bar();
-      if (et == 0) release(a, gs);
-    } else if (si.kind == LK_ACTION_IN) {
-      const int nc = action_ctas(a);
+      if (et == 0) {
+        LOOP_STAMP(gs, 2);
+        release(a, gs);
+      }
+    } else if (si.kind == LK_TIN) {
+      const int nc = tin_ctas(a);
       if (blockIdx.x >= nc) continue;
-      ok = poll_prev(gs);
+      ok = open(gs);
       if (!ok) break;
-      const int BH = a.B * a.H;
-      for (int cidx = blockIdx.x; cidx < kWidth / 8; cidx += nc) {
-        const int n0 = cidx * 8;
-        for (int r = et; r < BH; r += 128) {
-          float acc[8];
-#pragma unroll
-          for (int o = 0; o < 8; ++o) acc[o] = 0.f;
-          const float *x = a.xw + (size_t)r * a.A;
-          for (int i = 0; i < a.A; ++i) {
-            const float xi = x[i];
-#pragma unroll
-            for (int o = 0; o < 8; ++o) acc[o] = fmaf(__bfloat162float(a.ain_w[(size_t)(n0 + o) * a.A + i]), xi, acc[o]);
-          }
-#pragma unroll
-          for (int o = 0; o < 8; ++o) acc[o] += a.ain_b[n0 + o];
-          *reinterpret_cast<uint4 *>(a.aemb + (size_t)r * kWidth + n0) = pack8(acc);
-        }
-      }
-      fence_proxy_async_global();
+      for (int cidx = blockIdx.x; cidx < kWidth / 8; cidx += nc) tin_unit(a, cidx, si.step, et);
+      fence_proxy_async_global();  // u is read by TMA in the next stage
       epi_bar();
-      if (et == 0) release(a, gs);
-    } else if (si.kind == LK_EULER) {
-      const int nc = euler_ctas(a);
+      if (et == 0) {
+        LOOP_STAMP(gs, 2);
+        release(a, gs);
+      }
+    } else {  // LK_XOUT
+      const int nc = xout_ctas(a);
       if (blockIdx.x >= nc) continue;
-      ok = poll_prev(gs);
+      ok = open(gs);
       if (!ok) break;
-      const int nch = (a.A + 15) / 16, units = euler_units(a);
-      const int k = si.step;
-      float dt;
-      if (a.linspace) {
-        dt = (float)((double)(k + 1) / (double)a.N) - (float)((double)k / (double)a.N);
-      } else {
-        dt = (float)(-1.0 / (double)a.N);
-      }
-      const int last = k == a.N - 1;
-      for (int u = blockIdx.x; u < units; u += nc) {
-        const int i = u / nch, ch = u % nch;
-        const float4 *src = reinterpret_cast<const float4 *>(a.h + (size_t)(a.B + i) * kWidth) + et * 2;
-        const float4 x0 = src[0], x1 = src[1];
-        float ss = x0.x * x0.x + x0.y * x0.y + x0.z * x0.z + x0.w * x0.w + x1.x * x1.x + x1.y * x1.y +
-                   x1.z * x1.z + x1.w * x1.w;
-        ss = warp_sum(ss);
-        if (lane == 0) bs.red[warp] = ss;
-        epi_bar();
-        const float tot = (bs.red[0] + bs.red[1]) + (bs.red[2] + bs.red[3]);
-        const float inv = 1.0f / sqrtf(tot / (float)kWidth + kRmsEps);
-        const float4 *g4 = reinterpret_cast<const float4 *>(a.fnorm) + et * 2;
-        const float4 g0 = g4[0], g1 = g4[1];
-        float4 *y4 = reinterpret_cast<float4 *>(yrow) + et * 2;
-        y4[0] = make_float4((x0.x * inv) * (1.0f + g0.x), (x0.y * inv) * (1.0f + g0.y), (x0.z * inv) * (1.0f + g0.z),
-                            (x0.w * inv) * (1.0f + g0.w));
-        y4[1] = make_float4((x1.x * inv) * (1.0f + g1.x), (x1.y * inv) * (1.0f + g1.y), (x1.z * inv) * (1.0f + g1.z),
-                            (x1.w * inv) * (1.0f + g1.w));
-        epi_bar();
-        for (int o = warp; o < 16; o += 4) {
-          const int aa = ch * 16 + o;
-          if (aa >= a.A) break;
-          const float4 *wr = reinterpret_cast<const float4 *>(a.aout_w + (size_t)aa * kWidth);
-          const float4 *yr = reinterpret_cast<const float4 *>(yrow);
-          float acc = 0.f;
-          for (int c4 = lane; c4 < kWidth / 4; c4 += 32) {
-            const float4 wv = wr[c4], yv = yr[c4];
-            acc = fmaf(wv.x, yv.x, acc);
-            acc = fmaf(wv.y, yv.y, acc);
-            acc = fmaf(wv.z, yv.z, acc);
-            acc = fmaf(wv.w, yv.w, acc);
-          }
-          acc = warp_sum(acc);
-          if (lane == 0) {
-            const size_t xi = (size_t)i * a.A + aa;
-            float v = acc + a.aout_b[aa];
-            if (a.x_pred) v -= a.cp->x1[xi];
-            const float xn = __fadd_rn(a.xw[xi], __fmul_rn(dt, v));
-            a.xw[xi] = xn;
-            if (last) a.cp->x0[xi] = xn;
-          }
-        }
-        epi_bar();  // yrow and red are reused by the next unit
-      }
+      const int nch = (a.A + 15) / 16;
+      for (int u = blockIdx.x; u < xout_units(a); u += nc) xout_unit(a, bs, yrow, u / nch, u % nch, si.step, et);
       epi_bar();
-      if (et == 0) release(a, gs);
+      if (et == 0) {
+        LOOP_STAMP(gs, 2);
+        release(a, gs);
+      }
     }
   }
 }
@@ -1204,26 +1475,29 @@ __global__ void __launch_bounds__(kThreads, 1) k_loop(const __grid_constant__ Lo
       mbar_init(&bs.w_empty[i], 1);
       bs.w_fills[i] = 0;
     }
-    for (int i = 0; i < kASlots; ++i) {
+    for (int i = 0; i < kMaxASlots; ++i) {
       mbar_init(&bs.a_full[i], 1);
       mbar_init(&bs.a_empty[i], 1);
       bs.a_fills[i] = 0;
     }
     mbar_init(&bs.acc_full, 1);
-    mbar_init(&bs.acc_empty, 1);
-    bs.x_done = 0;
-    for (int i = 0; i < 2; ++i) {
+    bs.tmem_done = 0;
+    for (int i = 0; i < kKVBufs; ++i) {
       mbar_init(&bs.k_full[i], 32);  // one cp.async-completion arrival per loader lane (+ TMA bytes)
       mbar_init(&bs.k_empty[i], 1);
       mbar_init(&bs.v_full[i], 32);
       mbar_init(&bs.pv_done[i], 1);
+      bs.k_fills[i] = bs.v_fills[i] = 0;
+    }
+    for (int i = 0; i < 2; ++i) {
       mbar_init(&bs.s_full[i], 1);
       mbar_init(&bs.s_empty[i], 128);
       mbar_init(&bs.p_full[i], 128);
-      bs.k_fills[i] = bs.v_fills[i] = 0;
     }
     mbar_init(&bs.q_full, 128);
     mbar_init(&bs.mma_fin, 1);
+    bs.x_done = 0;
+    bs.ready = 0;
     bs.last = 0;
     fence_mbar_init();
   }
@@ -1237,7 +1511,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_loop(const __grid_constant__ Lo
   const uint32_t tmem = bs.tmem_slot;
   if (!err_set(a)) {
     if (warp == 0) {
-      if (lane == 0) role_weights(a, smem, bs);
+      if (lane < 2) role_weights(a, smem, bs, lane);
       __syncwarp();
     } else if (warp == 1) {
       role_mma(a, smem, bs, tmem);
@@ -1254,13 +1528,13 @@ __global__ void __launch_bounds__(kThreads, 1) k_loop(const __grid_constant__ Lo
       for (int i = 0; i < kWSlots; ++i)
         if (bs.w_fills[i]) dwait(&bs.w_full[i], (bs.w_fills[i] - 1) & 1u, a);
     if (warp == 2) {
-      for (int i = 0; i < kASlots; ++i)
+      for (int i = 0; i < kMaxASlots; ++i)
         if (bs.a_fills[i]) dwait(&bs.a_full[i], (bs.a_fills[i] - 1) & 1u, a);
-      for (int i = 0; i < 2; ++i)
+      for (int i = 0; i < kKVBufs; ++i)
         if (bs.k_fills[i]) dwait(&bs.k_full[i], (bs.k_fills[i] - 1) & 1u, a);
     }
     if (warp == 3)
-      for (int i = 0; i < 2; ++i)
+      for (int i = 0; i < kKVBufs; ++i)
         if (bs.v_fills[i]) dwait(&bs.v_full[i], (bs.v_fills[i] - 1) & 1u, a);
   }
   tc_fence_before();
@@ -1273,12 +1547,17 @@ __global__ void __launch_bounds__(kThreads, 1) k_loop(const __grid_constant__ Lo
 
 }  // namespace
 
+// Split-KV plan: each 128-row query tile's key blocks are cut into `splits` ranges of
+// `bps` blocks, one unit each, as many as the grid holds but at least
+// kAttnMinBlocks blocks per unit (below that, writing and merging the fp32 partials
+// costs more than the keys it saves).  One split means no COMBINE stage.
+constexpr int kAttnMinBlocks = 4;
 void loop_attn_plan(int B, int H, int P, int grid, int &splits, int &bps) {
   const int qps = (kHeads * (H + 1) + 127) / 128;
   const int nblk = (P + kKB - 1) / kKB + (H + kKB) / kKB;
   const int qt = B * qps;
   int s = grid / (qt > 0 ? qt : 1);
-  const int max_s = (nblk + 1) / 2;  // at least two key blocks per split
+  const int max_s = (nblk + kAttnMinBlocks - 1) / kAttnMinBlocks;
   if (s > max_s) s = max_s;
   if (s < 1) s = 1;
   bps = (nblk + s - 1) / s;
@@ -1287,23 +1566,46 @@ void loop_attn_plan(int B, int H, int P, int grid, int &splits, int &bps) {
 
 size_t loop_smem_bytes() { return kSmemTotal; }
 
-int loop_max_grid(int dev) {
+int loop_max_grid(int dev, const char **why) {
   int sms = 0, coop = 0, per_sm = 0;
+  *why = nullptr;
   if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
       cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev) != cudaSuccess || !coop) {
     cudaGetLastError();
+    *why = "the device does not support cooperative launches";
     return 0;
   }
-  if (cudaFuncSetAttribute(k_loop, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemTotal) != cudaSuccess ||
-      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_loop, kThreads, kSmemTotal) != cudaSuccess ||
+  if (cudaFuncSetAttribute(k_loop, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemTotal) != cudaSuccess) {
+    cudaGetLastError();
+    *why = "the loop kernel's shared memory cannot be configured";
+    return 0;
+  }
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_loop, kThreads, kSmemTotal) != cudaSuccess ||
       per_sm < 1) {
     cudaGetLastError();
+    *why = "one loop CTA does not fit an SM (registers or shared memory)";
     return 0;
   }
   return sms;
 }
 
+// The GEMM reduce stages a unit's slice of every split in region X: the largest
+// slice (an even token count) times the splits must fit, and every m-tile's units must
+// fit the grid (each unit waits for the others of its m-tile).
+static bool loop_plan_fits(const LoopArgs &a) {
+  const int kinds[5] = {LK_TOUT, LK_QKV, LK_O, LK_GU, LK_DOWN};
+  for (int k : kinds) {
+    const LoopGemm p = loop_gemm_plan(k, a.grid);
+    if (p.mtiles > kLoopMaxMtiles || p.mtiles * p.ksplit > a.grid) return false;
+    const int rows = a.R;  // the widest stored range
+    const int per = ((rows + p.ksplit - 1) / p.ksplit + 1) & ~1;
+    if ((size_t)per * p.ksplit * 512 > kXBytes) return false;
+  }
+  return a.box_rows % 16 == 0 && a.box_rows >= 16 && a.box_rows <= kLoopMaxRows;
+}
+
 cudaError_t launch_loop(const LoopArgs &a, cudaStream_t s) {
+  if (!loop_plan_fits(a)) return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(k_loop, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemTotal);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
@@ -1318,5 +1620,10 @@ cudaError_t launch_loop(const LoopArgs &a, cudaStream_t s) {
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, k_loop, a);
 }
+
+#ifdef PI0X_LOOP_TIMELINE
+// Profiling build only: device buffer of (stages x CTAs x 8) globaltimer stamps.
+extern "C" int pi0x_loop_timeline_set(void *p) { return (int)cudaMemcpyToSymbol(g_loop_tl, &p, sizeof(p)); }
+#endif
 
 }  // namespace pi0x

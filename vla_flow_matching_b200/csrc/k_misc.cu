@@ -92,7 +92,7 @@ void launch_time_vec(const TW *w_time, const float *bias, int num_steps, int lin
 template <typename TW>
 __global__ void __launch_bounds__(256) k_state_embed(const CallPtrs *cp, const TW *w, const float *bias, int S,
                                                       float *h, const float *gain, bf16 *xn, float *ss,
-                                                      int ss_ld, int nslots) {
+                                                      int ss_ld, int nslots, int tiled_rb, int rep_rows) {
   pdl_wait();
   pdl_trigger();
   __shared__ float sv[64];
@@ -108,7 +108,12 @@ __global__ void __launch_bounds__(256) k_state_embed(const CallPtrs *cp, const T
     h[(size_t)b * kWidth + n] = hv;
     if (gain) {
       ssq = fmaf(hv, hv, ssq);
-      xn[(size_t)b * kWidth + n] = __float2bfloat16_rn(hv * (1.0f + gain[n]));
+      const bf16 x = __float2bfloat16_rn(hv * (1.0f + gain[n]));
+      if (tiled_rb > 0) {  // the persistent loop's tiled layout, every replica
+        for (int r = 0; r < kLoopReps; ++r) xn[(size_t)r * rep_rows * kWidth + tiled_off(b, n, tiled_rb)] = x;
+      } else {
+        xn[(size_t)b * kWidth + n] = x;
+      }
     }
   }
   if (gain) {
@@ -126,8 +131,28 @@ __global__ void __launch_bounds__(256) k_state_embed(const CallPtrs *cp, const T
 
 template <typename TW>
 void launch_state_embed(const CallPtrs *cp, const TW *w, const float *b, int B, int S, float *h, cudaStream_t s,
-                        const float *gain, bf16 *xn, float *ss, int ss_ld, int nslots) {
-  launch_pdl(k_state_embed<TW>, B, 256, 0, s, cp, w, b, S, h, gain, xn, ss, ss_ld, nslots);
+                        const float *gain, bf16 *xn, float *ss, int ss_ld, int nslots, int tiled_rb,
+                        int rep_rows) {
+  launch_pdl(k_state_embed<TW>, B, 256, 0, s, cp, w, b, S, h, gain, xn, ss, ss_ld, nslots, tiled_rb, rep_rows);
+}
+
+// Copy of a bf16 (N, K) weight in the persistent loop's layout: m-tile m (rows
+// 128m .. 128m + 127) is stored at 128 m K as K-blocks of 128 rows x 64 columns, each
+// row 128 bytes with the 128-byte swizzle (tiled_off with rb = 128), so the K-blocks
+// of one unit are one contiguous run and each is the MMA's M-side operand as stored.
+__global__ void k_tile_weight(const bf16 *src, int K, bf16 *dst) {
+  const int m = blockIdx.x, kb = blockIdx.y;
+  bf16 *tile = dst + (size_t)m * 128 * K;
+  for (int t = threadIdx.x; t < 128 * 8; t += blockDim.x) {
+    const int r = t >> 3, c8 = t & 7;
+    const uint4 v = *reinterpret_cast<const uint4 *>(src + (size_t)(m * 128 + r) * K + kb * 64 + c8 * 8);
+    *reinterpret_cast<uint4 *>(tile + tiled_off(r, kb * 64 + c8 * 8, 128)) = v;
+  }
+}
+cudaError_t launch_tile_weight(const bf16 *src, int N, int K, bf16 *dst, cudaStream_t s) {
+  if (N % 128 != 0 || K % 64 != 0) return cudaErrorInvalidValue;
+  k_tile_weight<<<dim3(N / 128, K / 64), 256, 0, s>>>(src, K, dst);
+  return cudaGetLastError();
 }
 
 // Action tokens: out[i] = action_in_proj(x[i]) for every (sample, horizon) row.
@@ -405,9 +430,9 @@ void launch_delay_ns(unsigned long long ns, cudaStream_t s) { k_delay<<<1, 1, 0,
 template void launch_time_vec<float>(const float *, const float *, int, int, float *, cudaStream_t);
 template void launch_time_vec<bf16>(const bf16 *, const float *, int, int, float *, cudaStream_t);
 template void launch_state_embed<float>(const CallPtrs *, const float *, const float *, int, int, float *,
-                                        cudaStream_t, const float *, bf16 *, float *, int, int);
+                                        cudaStream_t, const float *, bf16 *, float *, int, int, int, int);
 template void launch_state_embed<bf16>(const CallPtrs *, const bf16 *, const float *, int, int, float *,
-                                       cudaStream_t, const float *, bf16 *, float *, int, int);
+                                       cudaStream_t, const float *, bf16 *, float *, int, int, int, int);
 template void launch_action_in<float, float>(const float *, const float *, const float *, int, int, float *,
                                              cudaStream_t);
 template void launch_action_in<bf16, bf16>(const float *, const bf16 *, const float *, int, int, bf16 *,

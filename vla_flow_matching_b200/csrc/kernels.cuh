@@ -32,6 +32,7 @@ struct CallPtrs {
   // 32-row boxes of the same tensors (the persistent small-batch loop's 32-key blocks)
   CUtensorMap kv_map32[2][kMaxDepth];
   CUtensorMap sfx_map32[2];
+
   const bf16 *prefix_k[kMaxDepth];
   const bf16 *prefix_v[kMaxDepth];
   const uint8_t *mask;
@@ -133,7 +134,9 @@ void launch_time_vec(const TW *w_time, const float *bias, int num_steps, int lin
 template <typename TW>
 void launch_state_embed(const CallPtrs *cp, const TW *w, const float *b, int B, int S, float *h, cudaStream_t s,
                         const float *gain = nullptr, bf16 *xn = nullptr, float *ss = nullptr, int ss_ld = 0,
-                        int nslots = kNormSlots);
+                        int nslots = kNormSlots, int tiled_rb = 0, int rep_rows = 0);
+// Weight copy in the persistent loop's m-tile layout (see k_tile_weight in k_misc.cu).
+cudaError_t launch_tile_weight(const bf16 *src, int N, int K, bf16 *dst, cudaStream_t s);
 template <typename TW, typename T>
 void launch_action_in(const float *x, const TW *w, const float *b, int rows, int A, T *out, cudaStream_t s);
 template <typename T>
@@ -186,7 +189,6 @@ void launch_gemm_simt(const float *A, int lda, const float *Bw, int ldb, int M, 
 // Weight operand of a tcgen05 GEMM: tensor maps with 64-row and wide boxes.
 struct TcWeight {
   CUtensorMap tm64, tm_wide;
-  CUtensorMap tm16;  // 64 x 16 boxes (the persistent small-batch loop)
   int N = 0, K = 0, bn_wide = 128;
   const CUtensorMap &map(int bn) const { return bn == 64 ? tm64 : tm_wide; }
 };
@@ -198,42 +200,48 @@ void launch_gemm_tc(int epi, const CUtensorMap &tmA, const CUtensorMap &tmB, con
 
 // ---- persistent small-batch loop (k_loop.cu) -----------------------------------
 // One cooperative launch runs every Euler step of a call when every step's rows fit
-// one 128-row MMA tile (B * (H + 1) <= 128): one CTA per SM, the steps' stages in
+// one 128-row MMA tile (B * (H + 1) <= 128): one CTA per SM, the call's stages in
 // program order, each stage waiting on the done-counter of the one before it.
 //
-// Stages of one Euler step (index i within the step):
-//   0 ACTION_IN, 1 TIN (action-time MLP in + SiLU), 2 TOUT (MLP out -> h, layer-0 norm
-//   inputs), then per layer QKV, ATTN, [COMBINE when attention is split], O, GU, DOWN,
-//   and last EULER (final norm, out-projection, x += dt v).
+// Program of one Euler step: TIN (action-time MLP input of the step), TOUT (MLP
+// output -> residual stream, layer-0 norm inputs), per layer QKV, ATTN, [COMBINE
+// when attention is split over key ranges], O, GU, DOWN, and last XOUT (final norm,
+// out-projection, x += dt v).
 enum LoopKind : int {
-  LK_ACTION_IN = 0, LK_TIN = 1, LK_TOUT = 2, LK_QKV = 3, LK_ATTN = 4, LK_COMBINE = 5,
-  LK_O = 6, LK_GU = 7, LK_DOWN = 8, LK_EULER = 9
+  LK_TIN = 0, LK_TOUT = 1, LK_QKV = 2, LK_ATTN = 3, LK_COMBINE = 4, LK_O = 5, LK_GU = 6, LK_DOWN = 7, LK_XOUT = 8
 };
 constexpr int kLoopMaxRows = 128;
-constexpr int kLoopNormSlots = 64;   // fused-norm partial sums: one slot per 16-column group
+constexpr int kLoopNormSlots = 8;    // fused-norm partial sums: one slot per 128-feature m-tile
 constexpr int kLoopKeyBlock = 32;    // attention key block of the loop kernel
-constexpr int kLoopMinGrid = 128;    // GEMM units stay <= 64 columns wide
+constexpr int kLoopMinGrid = 128;    // enough CTAs to split every GEMM's K over most SMs
+constexpr int kLoopReps = 1;         // replicas of each tiled activation operand
+constexpr int kLoopMaxMtiles = 64;   // m-tiles of the widest GEMM (gate/up: 8192 / 128)
 
 __host__ __device__ inline int loop_layer_stages(int attn_splits) { return attn_splits > 1 ? 6 : 5; }
 __host__ __device__ inline int loop_stages_per_step(int L, int attn_splits) {
-  return 3 + L * loop_layer_stages(attn_splits) + 1;
+  return 2 + L * loop_layer_stages(attn_splits) + 1;
 }
-// Kind and layer of stage i of a step.
-__host__ __device__ inline void loop_stage(int i, int L, int attn_splits, int &kind, int &layer) {
+__host__ __device__ inline int loop_total_stages(int N, int L, int attn_splits) {
+  return N * loop_stages_per_step(L, attn_splits);
+}
+// Kind, layer and Euler step of stage gs of the call.
+__host__ __device__ inline void loop_stage(int gs, int L, int attn_splits, int &kind, int &layer, int &step) {
+  const int spp = loop_stages_per_step(L, attn_splits);
+  step = gs / spp;
+  const int i = gs % spp;
   layer = 0;
-  if (i < 3) {
-    kind = i;
+  if (i < 2) {
+    kind = i == 0 ? LK_TIN : LK_TOUT;
     return;
   }
-  const int ls = loop_layer_stages(attn_splits);
-  const int j = i - 3;
-  if (j >= L * ls) {
-    kind = LK_EULER;
+  if (i == spp - 1) {
+    kind = LK_XOUT;
     layer = L - 1;
     return;
   }
-  layer = j / ls;
-  int sub = j % ls;
+  const int ls = loop_layer_stages(attn_splits);
+  layer = (i - 2) / ls;
+  int sub = (i - 2) % ls;
   if (ls == 5 && sub >= 2) ++sub;  // no COMBINE stage
   switch (sub) {
     case 0: kind = LK_QKV; break;
@@ -245,26 +253,33 @@ __host__ __device__ inline void loop_stage(int i, int L, int attn_splits, int &k
   }
 }
 
-// GEMM stage plan: N columns in 16-column groups, split over `nchunks` contiguous
-// chunks (<= 64 columns each) and `splits` equal K ranges; unit u = chunk * splits + split.
+// GEMM stage plan.  The weight is the MMA's M operand: 128 of its rows (output
+// features) form an m-tile, and the call's rows (tokens, a multiple of 16 <= 128) are
+// the N operand.  Each m-tile's K range is split over `ksplit` CTAs (as many as the
+// grid allows, at most one per 64-wide K-block), unit u = m * ksplit + s.  The units
+// of an m-tile then add their fp32 partial tiles in split order, each unit a slice of
+// the tokens.
 struct LoopGemm {
-  int N, K, splits, nchunks;
+  int N, K, mtiles, ksplit;
 };
 __host__ __device__ inline LoopGemm loop_gemm_plan(int kind, int grid) {
   LoopGemm p{1024, 1024, 1, 1};
   switch (kind) {
     case LK_QKV: p.N = kQkvDim; break;
-    case LK_O: p.K = kQDim; p.splits = 2; break;
+    case LK_O: p.K = kQDim; break;
     case LK_GU: p.N = 2 * kMlp; break;
-    case LK_DOWN: p.K = kMlp; p.splits = 4; break;
+    case LK_DOWN: p.K = kMlp; break;
     default: break;
   }
-  const int G = p.N / 16, per = grid / p.splits;
-  p.nchunks = G < per ? G : per;
+  p.mtiles = p.N / 128;
+  const int nk = p.K / 64;
+  int s = grid / p.mtiles;
+  if (s > nk) s = nk;
+  p.ksplit = s < 1 ? 1 : s;
   return p;
 }
 __host__ __device__ inline bool loop_is_gemm(int kind) {
-  return kind == LK_TIN || kind == LK_TOUT || kind == LK_QKV || kind == LK_O || kind == LK_GU || kind == LK_DOWN;
+  return kind == LK_TOUT || kind == LK_QKV || kind == LK_O || kind == LK_GU || kind == LK_DOWN;
 }
 
 struct LoopArgs {
@@ -272,31 +287,35 @@ struct LoopArgs {
   int linspace, x_pred, causal;
   int grid;
   int attn_splits, attn_bps;   // split-KV: splits per query tile, 32-key blocks per split
-  int box_rows;                // activation TMA box rows (64 or 128)
+  int box_rows;                // rows of an activation K-block tile: the call's rows rounded up to 16,
+                               // the N of every GEMM MMA
+  int rep_rows;                // replica r of a tiled activation with K columns starts at r * rep_rows * K
   int ss_ld;
   int debug_stall_stage;       // >= 0: that stage waits on a counter nothing raises (tests)
   unsigned long long wait_ns;  // time limit of every wait
   float *h, *ss_a, *ss_m, *gpart, *tvec, *xw, *part_o, *part_ml;
-  bf16 *xn, *q, *ks, *vs, *att, *act, *aemb, *uemb;
+  bf16 *xn, *q, *ks, *vs, *att, *act, *uemb;
   int *counters, *done;
+  int *mt_cnt;                 // per (stage, m-tile): units whose partial tile is stored
   const int *nvalid, *vidx;
   const float *rope_tab;
   const CallPtrs *cp;
   unsigned *err;
-  const bf16 *ain_w;
-  const float *ain_b, *tout_b, *aout_w, *aout_b, *fnorm;
+  // action-time MLP input with action_in folded in: u = silu(w_xa x + tvec[k]), w_xa =
+  // W_in[:, :W] W_action_in (fp32, W x A); tvec[k] carries W_in[:, :W] b_action_in
+  const float *w_xa;
+  const float *tout_b, *aout_w, *aout_b, *fnorm;
   const float *in_norm[kMaxDepth], *post_norm[kMaxDepth];
-  // tensor maps in device memory: weights (64 x 16 boxes) and activations
-  const CUtensorMap *m_tin, *m_tout;
-  const CUtensorMap *m_qkv[kMaxDepth], *m_o[kMaxDepth], *m_gu[kMaxDepth], *m_down[kMaxDepth];
-  const CUtensorMap *m_xn, *m_att, *m_act, *m_aemb, *m_uemb;
+  // weights as 128-row m-tiles of 64-wide swizzled K-blocks (k_tile_weight)
+  const bf16 *w_tout;
+  const bf16 *w_qkv[kMaxDepth], *w_o[kMaxDepth], *w_gu[kMaxDepth], *w_down[kMaxDepth];
 };
 
 // Split-KV plan of the loop attention (splits per query tile, key blocks per split).
 void loop_attn_plan(int B, int H, int P, int grid, int &splits, int &bps);
 size_t loop_smem_bytes();
-// CTAs of the loop kernel on `dev` (one per SM), or 0 if it cannot run there.
-int loop_max_grid(int dev);
+// CTAs of the loop kernel on `dev` (one per SM), or 0 with the reason in *why.
+int loop_max_grid(int dev, const char **why);
 // Enqueue the loop kernel (cooperative launch) on `s`.
 cudaError_t launch_loop(const LoopArgs &a, cudaStream_t s);
 

@@ -5,6 +5,7 @@
 #include <stdint.h>
 #include <string.h>
 
+#include <algorithm>
 #include <cmath>
 #include <new>
 #include <string>
@@ -111,11 +112,10 @@ struct Workspace {
   int *counters; // split-K per-tile arrival counters
   float *ss_a, *ss_m;  // fused RMSNorm partial sums of squares, kNormSlots x ss_ld (bf16 mode)
   int ss_ld = 0;
-  // persistent small-batch loop (bf16 mode): 64-slot norm sums, stage done-counters,
-  // activation tensor maps in device memory ([i][0] = 64-row, [i][1] = 128-row boxes)
+  // persistent small-batch loop (bf16 mode): 64-slot norm sums, stage done-counters
   float *ss64_a = nullptr, *ss64_m = nullptr;
   int *done = nullptr;
-  CUtensorMap *d_amaps = nullptr;
+  int *mt_cnt = nullptr;  // persistent loop: per (stage, m-tile) partial-tile counters
   float *rope_tab;     // (cos, sin) per position and pair (bf16 mode)
   void *xn, *q, *ks, *vs, *att, *act, *a_emb, *u_emb;
   // host-input staging (device side), allocated lazily
@@ -139,12 +139,16 @@ struct pi0x_handle {
   // weights (device)
   void *state_w, *ain_w, *tin_a, *tin_t, *tout_w;
   float *state_b, *ain_b, *tin_b, *tout_b, *aout_w, *aout_b, *fnorm, *inv_freq;
+  // persistent loop (bf16 mode): action_in folded into the action-time MLP input,
+  // w_xa = W_in[:, :W] W_action_in (W x A) and tin_b_loop = b_in + W_in[:, :W] b_action_in
+  float *w_xa = nullptr, *tin_b_loop = nullptr;
   LayerW layer[kMaxDepth];
   // weight-side tensor maps + tile widths (bf16 mode)
   TcWeight g_tin, g_tout, g_qkv[kMaxDepth], g_o[kMaxDepth], g_gu[kMaxDepth], g_down[kMaxDepth];
-  // 16-row-box weight maps in device memory for the persistent loop: tin, tout, then
-  // per layer qkv, o, gu, down
-  CUtensorMap *d_wmaps = nullptr;
+  // the persistent loop's copy of the GEMM weights in its unit order (k_tile_weight):
+  // tout, then per layer qkv, o, gu, down
+  void *wtile = nullptr;
+  pi0x::bf16 *wt_tout = nullptr, *wt_qkv[kMaxDepth], *wt_o[kMaxDepth], *wt_gu[kMaxDepth], *wt_down[kMaxDepth];
   int loop_grid = 0;          // CTAs of the persistent loop (0: the loop cannot launch here)
   bool loop_direct = false;   // the cooperative launch could not be captured: launch it directly
   bool loop_off = false;      // pi0x_debug_set_loop(h, 0): small batches take the multi-kernel path
@@ -243,7 +247,8 @@ size_t weight_bytes(const pi0x_config &c, size_t es) {
   const size_t W = kWidth;
   size_t act = W * c.state_dim + W * c.action_dim + 2 * W * W + W * W +
                (size_t)c.depth * ((size_t)kQkvDim * W + W * kQDim + 2 * (size_t)kMlp * W + W * kMlp);
-  size_t f32 = 4 * W + (size_t)c.action_dim * W + c.action_dim + W + 128 + (size_t)c.depth * 2 * W;
+  size_t f32 = 4 * W + (size_t)c.action_dim * W + c.action_dim + W + 128 + (size_t)c.depth * 2 * W +
+               (size_t)c.action_dim * W + W;  // + the loop's folded action-time MLP input
   return act * es + f32 * 4 + 64 * 1024 * (size_t)(16 + 6 * c.depth);
 }
 
@@ -253,8 +258,7 @@ int build_weight_maps(pi0x_handle *h) {
     g.N = N;
     g.K = K;
     g.bn_wide = plan_gemm_tc(1 << 20, N, K).bn;
-    return make_map(&g.tm64, w, N, K, K, 64) && make_map(&g.tm_wide, w, N, K, K, g.bn_wide) &&
-           make_map(&g.tm16, w, N, K, K, 16);
+    return make_map(&g.tm64, w, N, K, K, 64) && make_map(&g.tm_wide, w, N, K, K, g.bn_wide);
   };
   bool ok = mk(h->g_tin, h->tin_a, kWidth, kWidth) && mk(h->g_tout, h->tout_w, kWidth, kWidth);
   for (int l = 0; l < L && ok; ++l) {
@@ -265,17 +269,30 @@ int build_weight_maps(pi0x_handle *h) {
     g_last_error = "cuTensorMapEncodeTiled failed for a weight operand";
     return PI0X_ECUDA;
   }
-  std::vector<CUtensorMap> maps;
-  maps.push_back(h->g_tin.tm16);
-  maps.push_back(h->g_tout.tm16);
+  return PI0X_OK;
+}
+
+// The persistent loop's copy of every GEMM weight, as 128-row m-tiles of swizzled K-blocks.
+int build_loop_weights(pi0x_handle *h) {
+  const int L = h->cfg.depth;
+  const size_t W = kWidth;
+  const size_t per_layer = (size_t)kQkvDim * W + W * kQDim + 2 * (size_t)kMlp * W + W * kMlp;
+  CK(cudaMalloc(&h->wtile, 2 * (W * W + (size_t)L * per_layer)));
+  bf16 *p = (bf16 *)h->wtile;
+  auto tile = [&](const void *src, int kind, bf16 *&dst) -> cudaError_t {
+    const LoopGemm g = loop_gemm_plan(kind, h->loop_grid);
+    dst = p;
+    p += (size_t)g.N * g.K;
+    return launch_tile_weight((const bf16 *)src, g.N, g.K, dst, 0);
+  };
+  CK(tile(h->tout_w, LK_TOUT, h->wt_tout));
   for (int l = 0; l < L; ++l) {
-    maps.push_back(h->g_qkv[l].tm16);
-    maps.push_back(h->g_o[l].tm16);
-    maps.push_back(h->g_gu[l].tm16);
-    maps.push_back(h->g_down[l].tm16);
+    CK(tile(h->layer[l].qkv, LK_QKV, h->wt_qkv[l]));
+    CK(tile(h->layer[l].o, LK_O, h->wt_o[l]));
+    CK(tile(h->layer[l].gu, LK_GU, h->wt_gu[l]));
+    CK(tile(h->layer[l].down, LK_DOWN, h->wt_down[l]));
   }
-  CK(cudaMalloc(&h->d_wmaps, maps.size() * sizeof(CUtensorMap)));
-  CK(cudaMemcpy(h->d_wmaps, maps.data(), maps.size() * sizeof(CUtensorMap), cudaMemcpyHostToDevice));
+  CK(cudaStreamSynchronize(0));
   return PI0X_OK;
 }
 
@@ -312,7 +329,10 @@ int ensure_workspace(pi0x_handle *h, int B, int P, int N) {
   const size_t raw_floats = h->bf16 ? 0 : Rp * 2 * kMlp;
   add(4 * raw_floats);
   // bf16 split-K GEMMs: split-K is used only while tiles x splits <= 148 (plan_gemm_tc)
-  const size_t gpart_floats = h->bf16 ? (size_t)148 * 128 * 64 : 0;
+  // split-K partial tiles: the multi-kernel GEMMs' and the loop's (one 128 x box_rows
+  // tile per unit, at most one unit per CTA and stage)
+  const size_t gpart_floats =
+      h->bf16 ? std::max((size_t)148 * 128 * 64, (size_t)std::max(h->loop_grid, 148) * 128 * kLoopMaxRows) : 0;
   add(4 * gpart_floats);
   add(4 * 1024);
   const size_t ss_floats = h->bf16 ? (size_t)kNormSlots * Rp : 0;
@@ -321,24 +341,26 @@ int ensure_workspace(pi0x_handle *h, int B, int P, int N) {
   // positions 0 .. P + H (n_b <= P), 128 (cos, sin) pairs each
   const size_t rope_floats = h->bf16 ? (size_t)(nP + H + 1) * (kHeadDim / 2) * 2 : 0;
   add(4 * rope_floats);
-  add(es * Rp * kWidth);
+  // xn, att, act and u hold kLoopReps replicas for the persistent loop (bf16 mode)
+  const size_t reps = h->bf16 ? kLoopReps : 1;
+  add(reps * es * Rp * kWidth);
   add(es * Rp * kQDim);
   add(es * (size_t)L * Rp * kHeadDim);
   add(es * (size_t)L * Rp * kHeadDim);
-  add(es * Rp * kQDim);
-  add(es * Rp * kMlp);
+  add(reps * es * Rp * kQDim);
+  add(reps * es * Rp * kMlp);
   add(es * Rp * kWidth);
-  add(es * Rp * kWidth);
+  add(reps * es * Rp * kWidth);
   // split-KV partials: splits*mtiles*B stays below 96 + 148 CTAs (attn_tc_splits)
   const size_t part_floats = h->bf16 ? (size_t)256 * 128 * (kHeadDim + 2) : 0;
   add(4 * part_floats);
   // persistent loop: 64-slot norm sums (two sets), one done-counter per stage, maps
   const size_t ss64_floats = h->bf16 ? (size_t)kLoopNormSlots * Rp : 0;
-  const size_t done_ints = h->bf16 ? (size_t)nN * loop_stages_per_step(L, 2) : 0;
+  const size_t done_ints = h->bf16 ? (size_t)loop_total_stages(nN, L, 2) : 0;
   add(4 * ss64_floats);
   add(4 * ss64_floats);
   add(4 * done_ints);
-  add(h->bf16 ? 10 * sizeof(CUtensorMap) : 0);
+  add(4 * done_ints * kLoopMaxMtiles);
   void *base = nullptr;
   CK(cudaMalloc(&base, bytes));
   ws.arena.base = static_cast<uint8_t *>(base);
@@ -355,19 +377,19 @@ int ensure_workspace(pi0x_handle *h, int B, int P, int N) {
   ws.ss_m = (float *)ws.arena.take(4 * ss_floats);
   ws.ss_ld = (int)Rp;
   ws.rope_tab = (float *)ws.arena.take(4 * rope_floats);
-  ws.xn = ws.arena.take(es * Rp * kWidth);
+  ws.xn = ws.arena.take(reps * es * Rp * kWidth);
   ws.q = ws.arena.take(es * Rp * kQDim);
   ws.ks = ws.arena.take(es * (size_t)L * Rp * kHeadDim);
   ws.vs = ws.arena.take(es * (size_t)L * Rp * kHeadDim);
-  ws.att = ws.arena.take(es * Rp * kQDim);
-  ws.act = ws.arena.take(es * Rp * kMlp);
+  ws.att = ws.arena.take(reps * es * Rp * kQDim);
+  ws.act = ws.arena.take(reps * es * Rp * kMlp);
   ws.a_emb = ws.arena.take(es * Rp * kWidth);
-  ws.u_emb = ws.arena.take(es * Rp * kWidth);
+  ws.u_emb = ws.arena.take(reps * es * Rp * kWidth);
   ws.part = (float *)ws.arena.take(4 * part_floats);
   ws.ss64_a = (float *)ws.arena.take(4 * ss64_floats);
   ws.ss64_m = (float *)ws.arena.take(4 * ss64_floats);
   ws.done = (int *)ws.arena.take(4 * done_ints);
-  ws.d_amaps = h->bf16 ? (CUtensorMap *)ws.arena.take(10 * sizeof(CUtensorMap)) : nullptr;
+  ws.mt_cnt = (int *)ws.arena.take(4 * done_ints * kLoopMaxMtiles);
   CK(cudaMemset(base, 0, bytes));
   ws.B = nB;
   ws.P = nP;
@@ -383,13 +405,7 @@ int ensure_workspace(pi0x_handle *h, int B, int P, int N) {
       g_last_error = "cuTensorMapEncodeTiled failed for an activation operand";
       return PI0X_ECUDA;
     }
-    const ActMap *am[5] = {&ws.m_xn, &ws.m_att, &ws.m_act, &ws.m_aemb, &ws.m_uemb};
-    CUtensorMap dm[10];
-    for (int i = 0; i < 5; ++i) {
-      dm[2 * i] = am[i]->m64;
-      dm[2 * i + 1] = am[i]->m128;
-    }
-    CK(cudaMemcpy(ws.d_amaps, dm, sizeof(dm), cudaMemcpyHostToDevice));
+
   }
   return PI0X_OK;
 }
@@ -621,7 +637,8 @@ int enqueue_loop(pi0x_handle *h, int B, int P, int N, cudaStream_t s) {
 
 // ---- the Euler loop of a small batch: one persistent kernel ------------------------
 bool use_loop(const pi0x_handle *h, int B) {
-  return h->bf16 && !h->loop_off && h->loop_grid >= kLoopMinGrid && (long)B * (h->cfg.horizon + 1) <= kLoopMaxRows;
+  return h->bf16 && !h->loop_off && h->loop_grid >= kLoopMinGrid && (long)B * (h->cfg.horizon + 1) <= kLoopMaxRows &&
+         h->cfg.action_dim <= 32 && h->cfg.action_dim % 4 == 0;
 }
 
 int enqueue_persistent(pi0x_handle *h, int B, int P, int N, cudaStream_t s, int stall_stage,
@@ -639,17 +656,18 @@ int enqueue_persistent(pi0x_handle *h, int B, int P, int N, cudaStream_t s, int 
     g_last_error = "persistent loop: too many attention units for the partial buffer";
     return PI0X_EUNSUPPORTED;
   }
-  const int spp = loop_stages_per_step(L, splits);
   CK(cudaMemsetAsync(ws.counters, 0, 4 * 1024, s));
-  CK(cudaMemsetAsync(ws.done, 0, 4 * (size_t)N * spp, s));
+  CK(cudaMemsetAsync(ws.done, 0, 4 * (size_t)loop_total_stages(N, L, splits), s));
+  CK(cudaMemsetAsync(ws.mt_cnt, 0, 4 * (size_t)loop_total_stages(N, L, splits) * kLoopMaxMtiles, s));
   RUN(PI0X_K_PREP, launch_prep_mask(h->d_ptrs, B, P, ws.nvalid, ws.vidx, s));
-  RUN(PI0X_K_PREP, launch_time_vec<bf16>((const bf16 *)h->tin_t, h->tin_b, N,
+  RUN(PI0X_K_PREP, launch_time_vec<bf16>((const bf16 *)h->tin_t, h->tin_b_loop, N,
                                          h->time_grid == PI0X_TIME_LINSPACE ? 1 : 0, ws.tvec, s));
   RUN(PI0X_K_PREP, launch_copy_x1(h->d_ptrs, B * H * c.action_dim, ws.xw, s));
   RUN(PI0X_K_PREP, launch_rope_table(h->inv_freq, P + H + 1, ws.rope_tab, s));
+  const int rb = (R + 15) / 16 * 16;  // rows of an activation K-block tile: the GEMMs' MMA N
   RUN(PI0X_K_EMBED, launch_state_embed<bf16>(h->d_ptrs, (const bf16 *)h->state_w, h->state_b, B, c.state_dim,
                                              ws.h, s, h->layer[0].in_norm, (bf16 *)ws.xn, ws.ss64_a, ws.ss_ld,
-                                             kLoopNormSlots));
+                                             kLoopNormSlots, rb, (int)round_up((size_t)ws.R, 128)));
   LoopArgs a;
   memset(&a, 0, sizeof(a));
   a.B = B;
@@ -666,7 +684,8 @@ int enqueue_persistent(pi0x_handle *h, int B, int P, int N, cudaStream_t s, int 
   a.grid = h->loop_grid;
   a.attn_splits = splits;
   a.attn_bps = bps;
-  a.box_rows = R <= 64 ? 64 : 128;
+  a.box_rows = rb;
+  a.rep_rows = (int)round_up((size_t)ws.R, 128);
   a.ss_ld = ws.ss_ld;
   a.debug_stall_stage = stall_stage;
   a.wait_ns = wait_ns;
@@ -684,17 +703,16 @@ int enqueue_persistent(pi0x_handle *h, int B, int P, int N, cudaStream_t s, int 
   a.vs = (bf16 *)ws.vs;
   a.att = (bf16 *)ws.att;
   a.act = (bf16 *)ws.act;
-  a.aemb = (bf16 *)ws.a_emb;
   a.uemb = (bf16 *)ws.u_emb;
   a.counters = ws.counters;
   a.done = ws.done;
+  a.mt_cnt = ws.mt_cnt;
   a.nvalid = ws.nvalid;
   a.vidx = ws.vidx;
   a.rope_tab = ws.rope_tab;
   a.cp = h->d_ptrs;
   a.err = h->d_err;
-  a.ain_w = (const bf16 *)h->ain_w;
-  a.ain_b = h->ain_b;
+  a.w_xa = h->w_xa;
   a.tout_b = h->tout_b;
   a.aout_w = h->aout_w;
   a.aout_b = h->aout_b;
@@ -702,19 +720,12 @@ int enqueue_persistent(pi0x_handle *h, int B, int P, int N, cudaStream_t s, int 
   for (int l = 0; l < L; ++l) {
     a.in_norm[l] = h->layer[l].in_norm;
     a.post_norm[l] = h->layer[l].post_norm;
-    a.m_qkv[l] = h->d_wmaps + 2 + 4 * l;
-    a.m_o[l] = h->d_wmaps + 3 + 4 * l;
-    a.m_gu[l] = h->d_wmaps + 4 + 4 * l;
-    a.m_down[l] = h->d_wmaps + 5 + 4 * l;
+    a.w_qkv[l] = h->wt_qkv[l];
+    a.w_o[l] = h->wt_o[l];
+    a.w_gu[l] = h->wt_gu[l];
+    a.w_down[l] = h->wt_down[l];
   }
-  a.m_tin = h->d_wmaps;
-  a.m_tout = h->d_wmaps + 1;
-  const int box = a.box_rows == 128 ? 1 : 0;
-  a.m_xn = ws.d_amaps + 0 + box;
-  a.m_att = ws.d_amaps + 2 + box;
-  a.m_act = ws.d_amaps + 4 + box;
-  a.m_aemb = ws.d_amaps + 6 + box;
-  a.m_uemb = ws.d_amaps + 8 + box;
+  a.w_tout = h->wt_tout;
   RUN(PI0X_K_LOOP, CK(launch_loop(a, s)));
   CK(cudaGetLastError());
   return PI0X_OK;
@@ -941,7 +952,9 @@ int pi0x_create(const pi0x_config *cfg, const pi0x_weights *w, pi0x_handle **out
   FETCH(w->state_proj_w, W * c.state_dim, v);  UP(v, true, h->state_w);
   FETCH(w->state_proj_b, W, v);                UP(v, false, h->state_b);
   FETCH(w->action_in_w, W * c.action_dim, v);  UP(v, true, h->ain_w);
+  std::vector<float> ain_w_host = v;
   FETCH(w->action_in_b, W, v);                 UP(v, false, h->ain_b);
+  std::vector<float> ain_b_host = v;
   FETCH(w->time_in_w, W * 2 * W, v);
   v2.resize(W * W);
   v3.resize(W * W);
@@ -953,6 +966,29 @@ int pi0x_create(const pi0x_config *cfg, const pi0x_weights *w, pi0x_handle **out
   UP(v2, true, h->tin_a);
   UP(v3, true, h->tin_t);
   FETCH(w->time_in_b, W, v);                   UP(v, false, h->tin_b);
+  if (h->bf16) {
+    // persistent loop: w_xa = W_in[:, :W] W_action_in and b_in + W_in[:, :W] b_action_in,
+    // formed in float64 from the bf16 operands the other kernels use, rounded once
+    const int A = c.action_dim;
+    auto rb = [](float f) { return bf16_bits_to_f32(f32_to_bf16_bits(f)); };
+    std::vector<float> wxa((size_t)W * A), tb(W);
+    std::vector<double> ain_r(ain_w_host.size()), acc(A);
+    for (size_t i = 0; i < ain_w_host.size(); ++i) ain_r[i] = (double)rb(ain_w_host[i]);
+    for (size_t n = 0; n < W; ++n) {
+      double bacc = (double)v[n];
+      for (int j = 0; j < A; ++j) acc[j] = 0.0;
+      for (size_t i = 0; i < W; ++i) {
+        const double wi = (double)rb(v2[n * W + i]);
+        bacc += wi * (double)ain_b_host[i];
+        const double *ar = &ain_r[i * A];
+        for (int j = 0; j < A; ++j) acc[j] += wi * ar[j];
+      }
+      for (int j = 0; j < A; ++j) wxa[n * A + j] = (float)acc[j];
+      tb[n] = (float)bacc;
+    }
+    UP(wxa, false, h->w_xa);
+    UP(tb, false, h->tin_b_loop);
+  }
   FETCH(w->time_out_w, W * W, v);              UP(v, true, h->tout_w);
   FETCH(w->time_out_b, W, v);                  UP(v, false, h->tout_b);
   FETCH(w->action_out_w, W * c.action_dim, v); UP(v, false, h->aout_w);
@@ -994,7 +1030,15 @@ int pi0x_create(const pi0x_config *cfg, const pi0x_weights *w, pi0x_handle **out
     st = build_weight_maps(h);
     if (st) return fail(st);
   }
-  if (h->bf16) h->loop_grid = loop_max_grid(dev);
+  if (h->bf16) {
+    const char *why = nullptr;
+    h->loop_grid = loop_max_grid(dev, &why);
+    if (why) g_last_error = std::string("persistent small-batch loop unavailable (multi-kernel path used): ") + why;
+    if (h->loop_grid >= kLoopMinGrid) {
+      st = build_loop_weights(h);
+      if (st) return fail(st);
+    }
+  }
   e = cudaMalloc(&h->d_ptrs, sizeof(CallPtrs));
   if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&h->cap, cudaStreamNonBlocking);
   if (e == cudaSuccess) e = cudaMalloc(&h->d_err, sizeof(unsigned));
@@ -1069,6 +1113,7 @@ int pi0x_sample(pi0x_handle *h, const void *const *prefix_k, const void *const *
     g_last_error = "pi0x_sample: cuTensorMapEncodeTiled failed for the prefix K/V (pointers must be 16-byte aligned)";
     return PI0X_EINVAL;
   }
+
   CK(cudaMemcpyAsync(h->d_ptrs, &cp, sizeof(cp), cudaMemcpyHostToDevice, s));
   if (h->prof_on) {
     // Profiled call: direct launches with an event pair around each kernel.  A
@@ -1203,7 +1248,7 @@ void pi0x_destroy(pi0x_handle *h) {
   free_workspace(h->ws);
   if (h->ws.stage.base) cudaFree(h->ws.stage.base);
   if (h->warena.base) cudaFree(h->warena.base);
-  if (h->d_wmaps) cudaFree(h->d_wmaps);
+  if (h->wtile) cudaFree(h->wtile);
   if (h->d_ptrs) cudaFree(h->d_ptrs);
   if (h->d_err) cudaFree(h->d_err);
   delete h;
