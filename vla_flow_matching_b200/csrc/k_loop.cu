@@ -268,8 +268,9 @@ __device__ __forceinline__ int q_tiles(const LoopArgs &a, int step0) {
   return (kHeads * Tq + 127) / 128;
 }
 __device__ __forceinline__ int attn_units(const LoopArgs &a, int step0) { return a.B * q_tiles(a, step0) * a.attn_splits; }
+// COMBINE warp items: (query tile, 32-row group, 8-dim group).
 __device__ __forceinline__ int combine_items(const LoopArgs &a, int step0) {
-  return a.B * kHeads * (step0 ? a.H + 1 : a.H);
+  return a.B * q_tiles(a, step0) * 4 * (kHeadDim / 8);
 }
 __device__ __forceinline__ int combine_ctas(const LoopArgs &a, int step0) {
   const int c = (combine_items(a, step0) + 3) / 4;
@@ -321,21 +322,20 @@ __device__ __forceinline__ void red_slice(int r_lo, int r_hi, int ksplit, int s,
   t1 = min(r_hi, t0 + per);
 }
 // Bounded wait until a global counter reaches `need` (then acquired at gpu scope).
+// Every poll is an acquire load: the load that sees the count is the acquire, with no
+// further L2 round trip after it.
 __device__ bool gwait(const int *cnt, int need, const LoopArgs &a, unsigned bit) {
   if (ld_acquire(cnt) >= need) return true;
   const unsigned long long t0 = globaltimer_ns();
   while (true) {
-    bool hit = false;
-    for (int i = 0; i < 32 && !hit; ++i) hit = ld_relaxed(cnt) >= need;
-    if (hit) break;
+    for (int i = 0; i < 32; ++i)
+      if (ld_acquire(cnt) >= need) return true;
     if (err_set(a)) return false;
     if (globaltimer_ns() - t0 > a.wait_ns) {
       atomicOr(a.err, bit);
       return false;
     }
   }
-  (void)ld_acquire(cnt);
-  return true;
 }
 __device__ __forceinline__ const bf16 *weight_tiles(const LoopArgs &a, int kind, int layer) {
   switch (kind) {
@@ -470,22 +470,8 @@ __device__ __forceinline__ AUnit attn_unit(const LoopArgs &a, int u, int step0) 
 // ---- poller (warp 3, lane 0): open stage gs once stage gs - 1 has completed ----------
 __device__ bool poll_stage(const LoopArgs &a, Bars &bs, int gs) {
   if (gs > 0) {
-    const int *cnt = a.done + (gs - 1);
-    const int target = stage_expect(a, stage_at(a, gs - 1));
-    if (ld_relaxed(cnt) < target) {
-      const unsigned long long t0 = globaltimer_ns();
-      while (true) {
-        bool hit = false;
-        for (int i = 0; i < 32 && !hit; ++i) hit = ld_relaxed(cnt) >= target;
-        if (hit) break;
-        if (err_set(a)) return false;
-        if (globaltimer_ns() - t0 > a.wait_ns) {
-          atomicOr(a.err, kErrTimeoutFlag);
-          return false;
-        }
-      }
-    }
-    (void)ld_acquire(cnt);  // acquire the predecessor's results at gpu scope
+    // acquire the predecessor's results at gpu scope (the load that sees the count)
+    if (!gwait(a.done + (gs - 1), stage_expect(a, stage_at(a, gs - 1)), a, kErrTimeoutFlag)) return false;
   }
   if (gs == a.debug_stall_stage) {  // test hook: a counter that nothing raises
     const unsigned long long t0 = globaltimer_ns();
@@ -1172,13 +1158,11 @@ __device__ void role_epi(const LoopArgs &a, uint8_t *smem, Bars &bs, uint32_t tm
           ok = bs.last != 0;
           if (!ok) break;
           {
-            const int per_split = (t1 - t0) * 32, chunks = p.ksplit * per_split;
-            const float4 *src0 = reinterpret_cast<const float4 *>(a.gpart + (size_t)g.m * p.ksplit * NT * 128) + t0 * 32;
-            const uint32_t dst0 = smem_u32(smem + kOffX);
-            for (int c = et; c < chunks; c += 128) {
-              const int sp = c / per_split;
-              cp_async16(dst0 + (uint32_t)c * 16u, src0 + (size_t)sp * NT * 32 + (c - sp * per_split), true);
-            }
+            const int per_split = (t1 - t0) * 32;  // 16-byte chunks of one split's slice
+            const float4 *src = reinterpret_cast<const float4 *>(a.gpart + (size_t)g.m * p.ksplit * NT * 128) + t0 * 32;
+            uint32_t dst = smem_u32(smem + kOffX);
+            for (int sp = 0; sp < p.ksplit; ++sp, src += (size_t)NT * 32, dst += (uint32_t)per_split * 16u)
+              for (int c = et; c < per_split; c += 128) cp_async16(dst + (uint32_t)c * 16u, src + c, true);
             cp_async_commit();
           }
           LOOP_STAMP(gs, 7);
@@ -1203,12 +1187,21 @@ __device__ void role_epi(const LoopArgs &a, uint8_t *smem, Bars &bs, uint32_t tm
       const int nrows = kHeads * Tq;
       const float scale_l2 = 0.0625f * kLog2e;
       for (int u = blockIdx.x; u < U && ok; u += gridDim.x) {
-        const AUnit t = attn_unit(a, u, step0);
-        const int qi = t.ti * 128 + et;
+        // the unit's query tile from u alone: its Q loads go out before the key range,
+        // which waits on the sample's valid prefix length
+        const int qps = q_tiles(a, step0), qt = u / a.attn_splits, qb = qt / qps;
+        const int qi = (qt % qps) * 128 + et;
         const bool row_ok = qi < nrows;
         const int jq = qi / kHeads, head = qi % kHeads;
         int tok = 0;
-        if (row_ok) tok = step0 ? (jq == 0 ? t.b : a.B + t.b * a.H + jq - 1) : a.B + t.b * a.H + jq;
+        if (row_ok) tok = step0 ? (jq == 0 ? qb : a.B + qb * a.H + jq - 1) : a.B + qb * a.H + jq;
+        uint4 qq[32];
+        {
+          const uint4 *src = reinterpret_cast<const uint4 *>(a.q + (size_t)tok * kQDim + head * kHeadDim);
+#pragma unroll
+          for (int e = 0; e < 32; ++e) qq[e] = row_ok ? src[e] : make_uint4(0, 0, 0, 0);
+        }
+        const AUnit t = attn_unit(a, u, step0);
         const bool state_q = step0 && jq == 0;
         const int ja = step0 ? jq - 1 : jq;
         const int sfx_base = t.nbp * kKB;
@@ -1217,16 +1210,10 @@ __device__ void role_epi(const LoopArgs &a, uint8_t *smem, Bars &bs, uint32_t tm
         const int sfx_state = sfx_base + a.H;
         float m_used = -INFINITY, l = 0.f;
         if (t.nb > 0) {
-          // Q row -> TMEM lane et, columns kTmemQ.. (two bf16 per 32-bit column); two
-          // batches of 16 independent 16-byte loads
-          const uint4 *src = reinterpret_cast<const uint4 *>(a.q + (size_t)tok * kQDim + head * kHeadDim);
-#pragma unroll 1
-          for (int hb = 0; hb < 2; ++hb) {
-            uint4 qq[16];
+          // Q row -> TMEM lane et, columns kTmemQ.. (two bf16 per 32-bit column)
+          {
 #pragma unroll
-            for (int e = 0; e < 16; ++e) qq[e] = row_ok ? src[hb * 16 + e] : make_uint4(0, 0, 0, 0);
-#pragma unroll
-            for (int cc = 0; cc < 2; ++cc) {
+            for (int cc = 0; cc < 4; ++cc) {
               float v[32];
 #pragma unroll
               for (int e = 0; e < 8; ++e) {
@@ -1235,7 +1222,7 @@ __device__ void role_epi(const LoopArgs &a, uint8_t *smem, Bars &bs, uint32_t tm
                 v[4 * e + 2] = __uint_as_float(qq[cc * 8 + e].z);
                 v[4 * e + 3] = __uint_as_float(qq[cc * 8 + e].w);
               }
-              tmem_st_32x32b_x32(tmem + t_lane + kTmemQ + 32 * (hb * 2 + cc), v);
+              tmem_st_32x32b_x32(tmem + t_lane + kTmemQ + 32 * cc, v);
             }
           }
           tc_fence_before();
@@ -1356,7 +1343,9 @@ __device__ void role_epi(const LoopArgs &a, uint8_t *smem, Bars &bs, uint32_t tm
             }
           }
         } else {
-          const size_t prow = (size_t)u * 128 + et;  // u = (b * qps + ti) * splits + split
+          // partial O of unit u = (b * qps + ti) * splits + split as [u][4-dim chunk][row]:
+          // the 32 rows of a warp store 512 contiguous bytes per chunk
+          float4 *pbase = reinterpret_cast<float4 *>(a.part_o) + (size_t)u * (kHeadDim / 4) * 128 + et;
           for (int c0 = 0; c0 < kHeadDim; c0 += 32) {
             float v[32];
             if (t.nb > 0) {
@@ -1366,13 +1355,14 @@ __device__ void role_epi(const LoopArgs &a, uint8_t *smem, Bars &bs, uint32_t tm
               for (int e = 0; e < 32; ++e) v[e] = 0.f;
             }
             if (row_ok) {
-              float4 *d4 = reinterpret_cast<float4 *>(a.part_o + prow * kHeadDim + c0);
 #pragma unroll
               for (int e = 0; e < 8; ++e)
-                d4[e] = make_float4(v[4 * e] * inv_l, v[4 * e + 1] * inv_l, v[4 * e + 2] * inv_l, v[4 * e + 3] * inv_l);
+                __stcg(pbase + (size_t)(c0 / 4 + e) * 128,
+                       make_float4(v[4 * e] * inv_l, v[4 * e + 1] * inv_l, v[4 * e + 2] * inv_l, v[4 * e + 3] * inv_l));
             }
           }
           if (row_ok) {
+            const size_t prow = (size_t)u * 128 + et;
             a.part_ml[2 * prow] = m_used;
             a.part_ml[2 * prow + 1] = l;
           }
@@ -1393,42 +1383,60 @@ __device__ void role_epi(const LoopArgs &a, uint8_t *smem, Bars &bs, uint32_t tm
       ok = open(gs);
       if (!ok) break;
       const int Tq = step0 ? a.H + 1 : a.H;
-      const int nrows = kHeads * Tq, qps = q_tiles(a, step0), items = a.B * nrows;
-      const int S = a.attn_splits;
-      for (int base = blockIdx.x * 4; base < items; base += nc * 4) {
-        const int it = base + warp;
-        if (it >= items) continue;
-        const int b = it / nrows, qi = it % nrows, ti = qi / 128, qr = qi % 128;
-        const size_t prow0 = ((size_t)(b * qps + ti) * S) * 128 + qr;
-        // lane s < S holds split s's (m, l); the block's max and weights by shuffles
-        float ms = -INFINITY, lsv = 0.f;
-        if (lane < S) {
-          ms = __ldcg(a.part_ml + 2 * (prow0 + (size_t)lane * 128));
-          lsv = __ldcg(a.part_ml + 2 * (prow0 + (size_t)lane * 128) + 1);
-        }
-        const float M = warp_max(lsv > 0.f ? ms : -INFINITY);
-        const float wl = lsv > 0.f ? lsv * ex2_approx(ms - M) : 0.f;
-        const float den = warp_sum(wl);
-        float acc[8];
+      const int nrows = kHeads * Tq, qps = q_tiles(a, step0), S = a.attn_splits;
+      // warp item (query tile qt, 32-row group, 8 dims): lane = row, so every load of a
+      // split's (m, l) and 4-dim chunk is 32 consecutive rows.  All (m, l) load at once,
+      // then all chunks (at most kLoopMaxSplits splits).
+      for (int it = blockIdx.x * 4 + warp; it < combine_items(a, step0); it += nc * 4) {
+        const int qt = it / 128, rg = (it / 32) & 3, dg = it & 31;
+        const int b = qt / qps, qi = (qt % qps) * 128 + rg * 32 + lane;
+        if (qi >= nrows) continue;
+        const size_t prow0 = (size_t)qt * S * 128 + rg * 32 + lane;  // split s at + s * 128
+        float ms[kLoopMaxSplits], ls[kLoopMaxSplits];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) acc[e] = 0.f;
-        for (int s = 0; s < S; ++s) {
-          const float wgt = __shfl_sync(kFull, wl, s);
-          if (wgt == 0.f) continue;
-          const float4 *src = reinterpret_cast<const float4 *>(a.part_o + (prow0 + (size_t)s * 128) * kHeadDim + lane * 8);
-          const float4 x0 = __ldcg(src), x1 = __ldcg(src + 1);
-          acc[0] = fmaf(wgt, x0.x, acc[0]); acc[1] = fmaf(wgt, x0.y, acc[1]);
-          acc[2] = fmaf(wgt, x0.z, acc[2]); acc[3] = fmaf(wgt, x0.w, acc[3]);
-          acc[4] = fmaf(wgt, x1.x, acc[4]); acc[5] = fmaf(wgt, x1.y, acc[5]);
-          acc[6] = fmaf(wgt, x1.z, acc[6]); acc[7] = fmaf(wgt, x1.w, acc[7]);
+        for (int sp = 0; sp < kLoopMaxSplits; ++sp) {
+          ms[sp] = ls[sp] = 0.f;
+          if (sp < S) {
+            const float2 ml = __ldcg(reinterpret_cast<const float2 *>(a.part_ml) + prow0 + (size_t)sp * 128);
+            ms[sp] = ml.x;
+            ls[sp] = ml.y;
+          }
+        }
+        // unit (qt, sp) holds chunk k of its row r at part_o float4 (unit * 64 + k) * 128 + r
+        const float4 *src = reinterpret_cast<const float4 *>(a.part_o) + ((size_t)qt * S * (kHeadDim / 4) + dg * 2) * 128 +
+                            rg * 32 + lane;
+        float4 x[kLoopMaxSplits][2];
+#pragma unroll
+        for (int sp = 0; sp < kLoopMaxSplits; ++sp)
+#pragma unroll
+          for (int e = 0; e < 2; ++e)
+            x[sp][e] = sp < S ? __ldcg(src + ((size_t)sp * (kHeadDim / 4) + e) * 128)  // (every unit stores its rows)
+                              : make_float4(0.f, 0.f, 0.f, 0.f);
+        float M = -INFINITY;
+#pragma unroll
+        for (int sp = 0; sp < kLoopMaxSplits; ++sp)
+          if (sp < S && ls[sp] > 0.f) M = fmaxf(M, ms[sp]);
+        float den = 0.f;
+        float o[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int sp = 0; sp < kLoopMaxSplits; ++sp) {
+          if (!(sp < S && ls[sp] > 0.f)) continue;
+          const float wgt = ls[sp] * ex2_approx(ms[sp] - M);
+          den += wgt;
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            o[4 * e] = fmaf(wgt, x[sp][e].x, o[4 * e]);
+            o[4 * e + 1] = fmaf(wgt, x[sp][e].y, o[4 * e + 1]);
+            o[4 * e + 2] = fmaf(wgt, x[sp][e].z, o[4 * e + 2]);
+            o[4 * e + 3] = fmaf(wgt, x[sp][e].w, o[4 * e + 3]);
+          }
         }
         const int j = qi / kHeads, hd = qi % kHeads;
         const int tok = step0 ? (j == 0 ? b : a.B + b * a.H + j - 1) : a.B + b * a.H + j;
         const float inv = den > 0.f ? 1.0f / den : 0.f;
 #pragma unroll
-        for (int e = 0; e < 8; ++e) acc[e] *= inv;
-        store_reps(a.att, tiled_off(tok, hd * kHeadDim + lane * 8, a.box_rows), (size_t)a.rep_rows * kQDim,
-                   pack8(acc));
+        for (int e = 0; e < 8; ++e) o[e] *= inv;
+        store_reps(a.att, tiled_off(tok, hd * kHeadDim + dg * 8, a.box_rows), (size_t)a.rep_rows * kQDim, pack8(o));
       }
       fence_proxy_async_global();
       epi_bar();
@@ -1559,6 +1567,7 @@ void loop_attn_plan(int B, int H, int P, int grid, int &splits, int &bps) {
   int s = grid / (qt > 0 ? qt : 1);
   const int max_s = (nblk + kAttnMinBlocks - 1) / kAttnMinBlocks;
   if (s > max_s) s = max_s;
+  if (s > kLoopMaxSplits) s = kLoopMaxSplits;
   if (s < 1) s = 1;
   bps = (nblk + s - 1) / s;
   splits = (nblk + bps - 1) / bps;
