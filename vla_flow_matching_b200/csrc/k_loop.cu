@@ -30,11 +30,12 @@
 //             weight K-blocks of every stage, in program order, into a 5-slot ring of
 //             16 KB.  Weights are inputs, so it runs ahead of the activations across
 //             stage boundaries, bounded only by the ring.
-//   warp 1    tcgen05.mma issuer (GEMM units; S = Q K^T and O += P V of attention).
+//   warp 1    tcgen05.mma issuer of attention units (S = Q K^T, O += P V).
 //   warp 2    activation loader of GEMM units; K loader of attention units.
 //   warp 3    poller of the stage done-counters (lane 0), V loader of attention units.
-//   warps 4-7 epilogues (TMEM lane quarter = warp % 4), the softmax of attention
-//             units and the row-wise stages (TIN, COMBINE, XOUT).
+//   warps 4-7 the MMAs of GEMM units (warp w: every fourth K-block, into its own
+//             accumulator chain), their epilogues (TMEM lane quarter = warp % 4), the
+//             softmax of attention units and the row-wise stages (TIN, COMBINE, XOUT).
 //
 // GEMM units: the weight is the MMA's M side.  128 weight rows (output features) form
 // an m-tile and the call's rows, rounded up to 16 tokens, are N, so one tcgen05.mma
@@ -114,6 +115,8 @@ struct Bars {
   uint64_t k_full[kKVBufs], k_empty[kKVBufs], v_full[kKVBufs], pv_done[kKVBufs];
   uint64_t s_full[2], s_empty[2], p_full[2];
   uint64_t q_full, mma_fin;
+  uint64_t epi_fin;   // the epilogue warps' GEMM MMAs have completed (exit)
+  uint64_t red_full;  // GEMM reduce: the m-tile's partial slices have landed in region X
   uint32_t tmem_slot;
   uint32_t x_done;    // units that used region X and whose MMAs have completed (monotonic)
   uint32_t tmem_done; // units whose accumulator reads (GEMM) / O readout (attention) are done
@@ -123,6 +126,8 @@ struct Bars {
   uint32_t w_fills[kWSlots];  // drain bookkeeping
   uint32_t a_fills[kMaxASlots];
   uint32_t k_fills[kKVBufs], v_fills[kKVBufs];
+  uint32_t red_fills;
+  uint32_t epi_err;  // an epilogue warp's wait gave up (read by all four after a barrier)
 };
 constexpr uint32_t kBarBytes = ((sizeof(Bars) + 127) / 128) * 128;
 constexpr uint32_t kOffRow = kOffBar + kBarBytes;   // XOUT: the normalised row (1024 fp32)
@@ -539,7 +544,7 @@ __device__ void role_mma(const LoopArgs &a, uint8_t *smem, Bars &bs, uint32_t tm
   const uint32_t sbase = smem_u32(smem);
   const int nas = a_slots(a);
   const uint32_t asb = a_slot_bytes(a);
-  uint32_t wi = 0, ai = 0, acc_n = 0, kj = 0, vj = 0, sj = 0, pj = 0, qn = 0, units_before = 0;
+  uint32_t kj = 0, vj = 0, sj = 0, pj = 0, qn = 0;
   bool ok = true;
   const uint64_t kdesc0 = smem_desc_k_sw128(sbase + kOffK, 0);
   const uint64_t pdesc0 = smem_desc_k_sw128(sbase + kOffP, 0);
@@ -548,50 +553,11 @@ __device__ void role_mma(const LoopArgs &a, uint8_t *smem, Bars &bs, uint32_t tm
   constexpr uint32_t idesc_o = idesc_bf16_f32(128, kHeadDim) | (1u << 16);  // B (V) MN-major
   for (int gs = 0; gs < total && ok; ++gs) {
     const StageInfo si = stage_at(a, gs);
-    if (loop_is_gemm(si.kind)) {
-      const LoopGemm p = loop_gemm_plan(si.kind, a.grid);
-      const int U = p.mtiles * p.ksplit;
-      // D[128 weight rows, box_rows tokens] += W[128, 16] X[box_rows, 16]^T: A is the
-      // weight K-block, B the activation K-block, both K-major with the 128-byte swizzle
-      const uint32_t idesc = idesc_bf16_f32(128, a.box_rows);
-      for (int u = blockIdx.x; u < U && ok; u += gridDim.x) {
-        const GUnit g = gemm_unit(p, u);
-        // the accumulator may be written once every earlier unit's TMEM reads are done
-        bool good = true;
-        if ((threadIdx.x & 31) == 0) good = smem_wait(&bs.tmem_done, units_before, a, kErrTimeoutMma);
-        if (!__all_sync(kFull, __shfl_sync(kFull, (int)good, 0) != 0)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        for (int kb = g.kb0; kb < g.kb1 && ok; ++kb, ++wi, ++ai) {
-          const int ws = wi % kWSlots, as = ai % nas;
-          if (!__all_sync(kFull, lwait(&bs.w_full[ws], (wi / kWSlots) & 1u, a, kErrTimeoutMma)) ||
-              !__all_sync(kFull, lwait(&bs.a_full[as], (ai / nas) & 1u, a, kErrTimeoutMma))) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t wb = sbase + kOffW + ws * kWSlotBytes, ab = sbase + kOffA + as * asb;
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            tc_mma_bf16_w(tmem + kTmemAcc, smem_desc_k_sw128(wb, kk * 32), smem_desc_k_sw128(ab, kk * 32), idesc,
-                          (kb > g.kb0 || kk > 0) ? 1u : 0u);
-          tc_commit_w(&bs.a_empty[as]);
-          tc_commit_w(&bs.w_empty[ws]);
-        }
-        if (!ok) break;
-        if ((threadIdx.x & 31) == 0) LOOP_STAMP(gs, 6);
-        tc_commit_w(&bs.acc_full);
-        ++acc_n;
-        ++units_before;
-      }
-    } else if (si.kind == LK_ATTN) {
+    if (si.kind == LK_ATTN) {
       const int step0 = si.step == 0;
       const int U = attn_units(a, step0);
       for (int u = blockIdx.x; u < U && ok; u += gridDim.x) {
         const AUnit t = attn_unit(a, u, step0);
-        ++units_before;
         if (t.nb == 0) continue;
         if (!__all_sync(kFull, lwait(&bs.q_full, qn & 1u, a, kErrTimeoutMma))) {
           ok = false;
@@ -825,11 +791,12 @@ __device__ __forceinline__ void add4(float4 &d, const float4 &x) {
 
 // Reduce + epilogue of tokens [t0, t1) of m-tile g.m (warps 4-7).  `stage` receives
 // the m-tile's partial tiles for the slice, split-major (split s, slice token j, 128
-// rows as 32 quads of 4 rows), from cp.async copies every thread has issued; every
+// rows as 32 quads of 4 rows), from one bulk copy per split completing on `staged`; every
 // output adds its splits in a fixed order, so the result does not depend on timing.
 // One warp per SM sub-partition runs this, so the items of a thread are unrolled with
 // independent registers (no shuffles or divergent branches) to overlap their latencies,
-// and their global operands load while the copies are in flight.
+// and their global operands load while the copies are in flight.  A wait that runs out
+// (bounded by the call's limit) leaves the error word set by the caller's next wait.
 //
 // Residual kinds (TOUT: bias; O, DOWN: residual), item (token, quad q = lane), a warp
 // per token: update h and, with a following norm, store bf16 h*(1+g) and the token's
@@ -843,13 +810,14 @@ __device__ __forceinline__ void add4(float4 &d, const float4 &x) {
 constexpr int kRedItems = 4;
 __device__ void reduce_unit(const LoopArgs &a, const StageInfo &si, const LoopGemm &p, const GUnit &g, int t0,
                             int t1, int out_off, int et, const float4 *stage, const float *rstd_s, const int *pos_s,
-                            int gs) {
+                            uint64_t *staged, uint32_t staged_parity, int gs) {
   (void)gs;  // timeline stamps only
   // the call's pointers and sizes in registers: read through `a` after every store
   // (which may alias it, as far as the compiler can tell) they would be reloaded
   const int kind = si.kind, layer = si.layer;
   const int lane = et & 31, ks = p.ksplit, T = t1 - t0;
-  const int rb = a.box_rows, ss_ld = a.ss_ld, R = a.R;
+  const int rb = a.box_rows, ss_ld = a.ss_ld, R = a.R, B = a.B, H = a.H;
+  const int step0 = si.step == 0, qps = q_tiles(a, step0);
   const size_t rep_w = (size_t)a.rep_rows * kWidth, rep_m = (size_t)a.rep_rows * kMlp;
   float *const hbuf = a.h;
   bf16 *const xn = a.xn, *const act = a.act, *const qb = a.q, *const kbuf = a.ks, *const vbuf = a.vs;
@@ -873,8 +841,7 @@ __device__ void reduce_unit(const LoopArgs &a, const StageInfo &si, const LoopGe
       }
     };
     load_ops(et);
-    cp_async_wait<0>();
-    epi_bar();  // every thread's staging copies have landed
+    lwait(staged, staged_parity, a, kErrTimeoutEpilogue);  // the slices have landed
     for (int it0 = et; it0 < items; it0 += 128 * kRedItems) {
       if (it0 != et) load_ops(it0);
       float4 lo4[kRedItems], hi4[kRedItems];
@@ -916,10 +883,26 @@ __device__ void reduce_unit(const LoopArgs &a, const StageInfo &si, const LoopGe
           }
         }
         const int d0 = ((g.m & 1) * 8 + gq) * 8 + e0;
-        bf16 *dst = hd < kHeads ? qb + (size_t)orow * kQDim + hd * kHeadDim + d0
-                                : (hd == kHeads ? kbuf : vbuf) + ((size_t)layer * R + orow) * kHeadDim + d0;
-        *reinterpret_cast<uint2 *>(dst) = pack4(lo[0], lo[1], lo[2], lo[3]);
-        *reinterpret_cast<uint2 *>(dst + kHeadDim / 2) = pack4(hi[0], hi[1], hi[2], hi[3]);
+        if (hd < kHeads) {
+          // query row qi = jq * 8 + head of sample b (jq: the state token at step 0, then
+          // the actions): tile b * qps + qi / 128, stored as [8-dim chunk][row][8 dims]
+          int b, jq;
+          if (orow < B) {
+            b = orow;
+            jq = 0;
+          } else {
+            b = (orow - B) / H;
+            jq = (orow - B) % H + (step0 ? 1 : 0);
+          }
+          const int qi = jq * kHeads + hd;
+          bf16 *tile = qb + (size_t)(b * qps + (qi >> 7)) * 128 * kHeadDim + (size_t)(qi & 127) * 8 + (d0 & 7);
+          *reinterpret_cast<uint2 *>(tile + (size_t)(d0 >> 3) * 128 * 8) = pack4(lo[0], lo[1], lo[2], lo[3]);
+          *reinterpret_cast<uint2 *>(tile + (size_t)((d0 + kHeadDim / 2) >> 3) * 128 * 8) = pack4(hi[0], hi[1], hi[2], hi[3]);
+        } else {
+          bf16 *dst = (hd == kHeads ? kbuf : vbuf) + ((size_t)layer * R + orow) * kHeadDim + d0;
+          *reinterpret_cast<uint2 *>(dst) = pack4(lo[0], lo[1], lo[2], lo[3]);
+          *reinterpret_cast<uint2 *>(dst + kHeadDim / 2) = pack4(hi[0], hi[1], hi[2], hi[3]);
+        }
       }
     }
     return;
@@ -942,8 +925,7 @@ __device__ void reduce_unit(const LoopArgs &a, const StageInfo &si, const LoopGe
     }
   };
   load_ops(et);
-  cp_async_wait<0>();
-  epi_bar();  // every thread's staging copies have landed
+  lwait(staged, staged_parity, a, kErrTimeoutEpilogue);  // the slices have landed
   for (int it0 = et; it0 < items; it0 += 128 * kRedItems) {
     if (it0 != et) load_ops(it0);
     float4 v4[kRedItems];
@@ -1090,7 +1072,10 @@ __device__ void role_epi(const LoopArgs &a, uint8_t *smem, Bars &bs, uint32_t tm
   const int total = total_stages(a);
   const int warp = et >> 5, lane = et & 31;
   const uint32_t t_lane = (uint32_t)(warp * 32) << 16;
-  uint32_t acc_n = 0, sj = 0, pj = 0, pvj = 0, tmem_units = 0;
+  uint32_t acc_n = 0, sj = 0, pj = 0, pvj = 0, tmem_units = 0, red_n = 0, wi = 0, ai = 0;
+  const uint32_t sbase = smem_u32(smem);
+  const int nas = a_slots(a);
+  const uint32_t asb = a_slot_bytes(a);
   bool ok = true;
   float *yrow = reinterpret_cast<float *>(smem + kOffRow);
   auto open = [&](int gs) -> bool {
@@ -1112,18 +1097,61 @@ __device__ void role_epi(const LoopArgs &a, uint8_t *smem, Bars &bs, uint32_t tm
       const int NT = a.box_rows;
       // U <= grid (at most 64 m-tiles, at least 128 CTAs): every unit of an m-tile
       // runs on its own CTA, so waiting for the m-tile's partials cannot wait on itself
+      // D[128 weight rows, NT tokens] += W[128, 16] X[NT, 16]^T: A is the weight K-block,
+      // B the activation K-block, both K-major with the 128-byte swizzle
+      const uint32_t idesc = idesc_bf16_f32(128, NT);
+      const int nch = NT * 4 <= 256 ? 4 : 256 / NT;  // accumulator chains in TMEM 256..511
       for (int u = blockIdx.x; u < U && ok; u += gridDim.x) {
         const GUnit g = gemm_unit(p, u);
-        ok = __all_sync(kFull, lwait(&bs.acc_full, acc_n & 1u, a, kErrTimeoutEpilogue));
-        if (!ok) break;
+        const int nk = g.kb1 - g.kb0;
+        // MMA issue from the four warps (a tcgen05.mma costs its issuing warp a fixed
+        // time): warp w takes K-blocks w, w + nch, .. of the unit into chain w, then every
+        // warp commits acc_full (four arrivals) and the readout adds the chains in order.
+        // The previous unit's TMEM reads finished before the barrier that ended it.
+        tc_fence_after();
+        bool good = true;
+        for (int i = warp; i < nk && warp < nch && good; i += nch) {
+          const uint32_t wk = wi + (uint32_t)i, ak = ai + (uint32_t)i;
+          const int ws = wk % kWSlots, as = ak % nas;
+          good = __all_sync(kFull, lwait(&bs.w_full[ws], (wk / kWSlots) & 1u, a, kErrTimeoutEpilogue)) &&
+                 __all_sync(kFull, lwait(&bs.a_full[as], (ak / nas) & 1u, a, kErrTimeoutEpilogue));
+          if (!good) break;
+          tc_fence_after();
+          const uint32_t wb = sbase + kOffW + ws * kWSlotBytes, ab = sbase + kOffA + as * asb;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            tc_mma_bf16_w(tmem + kTmemAcc + (uint32_t)(warp * NT), smem_desc_k_sw128(wb, kk * 32),
+                          smem_desc_k_sw128(ab, kk * 32), idesc, (i >= nch || kk > 0) ? 1u : 0u);
+          tc_commit_w(&bs.a_empty[as]);
+          tc_commit_w(&bs.w_empty[ws]);
+        }
+        wi += (uint32_t)nk;
+        ai += (uint32_t)nk;
+        tc_commit_w(&bs.acc_full);
+        if (!good && lane == 0) atomicOr(&bs.epi_err, 1u);
+        good = __all_sync(kFull, lwait(&bs.acc_full, acc_n & 1u, a, kErrTimeoutEpilogue));
+        if (!good && lane == 0) atomicOr(&bs.epi_err, 1u);
+        epi_bar();
+        if (*(volatile uint32_t *)&bs.epi_err) {  // the same decision in all four warps
+          ok = false;
+          break;
+        }
         ++acc_n;
         tc_fence_after();
         LOOP_STAMP(gs, 1);
-        // partial tile, token-major: row et of the m-tile for the stored tokens
+        // partial tile, token-major: row et of the m-tile for the stored tokens (the sum
+        // of the unit's chains, in chain order)
+        const int used = nk < nch ? nk : nch;
         float *mine = a.gpart + (size_t)u * 128 * NT;
         for (int c0 = r_lo & ~15; c0 < r_hi; c0 += 16) {
           float v[16];
           tmem_ld_x16(tmem + t_lane + kTmemAcc + (uint32_t)c0, v);
+          for (int c = 1; c < used; ++c) {
+            float w[16];
+            tmem_ld_x16(tmem + t_lane + kTmemAcc + (uint32_t)(c * NT + c0), w);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) v[i] += w[i];
+          }
 #pragma unroll
           for (int i = 0; i < 16; ++i) __stcg(mine + (size_t)(c0 + i) * 128 + et, v[i]);
         }
@@ -1158,15 +1186,25 @@ __device__ void role_epi(const LoopArgs &a, uint8_t *smem, Bars &bs, uint32_t tm
           ok = bs.last != 0;
           if (!ok) break;
           {
-            const int per_split = (t1 - t0) * 32;  // 16-byte chunks of one split's slice
-            const float4 *src = reinterpret_cast<const float4 *>(a.gpart + (size_t)g.m * p.ksplit * NT * 128) + t0 * 32;
-            uint32_t dst = smem_u32(smem + kOffX);
-            for (int sp = 0; sp < p.ksplit; ++sp, src += (size_t)NT * 32, dst += (uint32_t)per_split * 16u)
-              for (int c = et; c < per_split; c += 128) cp_async16(dst + (uint32_t)c * 16u, src + c, true);
-            cp_async_commit();
+            // one bulk copy per split's slice (contiguous in the token-major partial tile),
+            // split sp issued by lane sp / 4 of warp sp % 4: each copy costs its issuing
+            // thread a fixed time, so the issues run in four warps at once
+            const uint32_t slice_bytes = (uint32_t)(t1 - t0) * 512u;
+            if (et == 0) {
+              mbar_arrive_expect_tx(&bs.red_full, slice_bytes * (uint32_t)p.ksplit);
+              bs.red_fills = red_n + 1;
+            }
+            const int sp = lane * 4 + warp;
+            if (sp < p.ksplit) {
+              fence_proxy_async_global();  // the partials were stored through the generic proxy
+              bulk_load(smem_u32(smem + kOffX + (uint32_t)sp * slice_bytes),
+                        a.gpart + ((size_t)(g.m * p.ksplit + sp) * NT + t0) * 128, slice_bytes, &bs.red_full);
+            }
           }
           LOOP_STAMP(gs, 7);
-          reduce_unit(a, si, p, g, t0, t1, out_off, et, reinterpret_cast<const float4 *>(smem + kOffX), rstd_s, pos_s, gs);
+          reduce_unit(a, si, p, g, t0, t1, out_off, et, reinterpret_cast<const float4 *>(smem + kOffX), rstd_s, pos_s,
+                      &bs.red_full, red_n & 1u, gs);
+          ++red_n;
           LOOP_STAMP(gs, 10);
           fence_proxy_async_global();  // outputs are read by bulk copies in the next stage
         }
@@ -1195,11 +1233,13 @@ __device__ void role_epi(const LoopArgs &a, uint8_t *smem, Bars &bs, uint32_t tm
         const int jq = qi / kHeads, head = qi % kHeads;
         int tok = 0;
         if (row_ok) tok = step0 ? (jq == 0 ? qb : a.B + qb * a.H + jq - 1) : a.B + qb * a.H + jq;
+        // q of query tile qt is stored as [8-dim chunk][128 rows] (reduce_unit): chunk e of
+        // this thread's row, for consecutive rows of a warp, is 512 contiguous bytes
         uint4 qq[32];
         {
-          const uint4 *src = reinterpret_cast<const uint4 *>(a.q + (size_t)tok * kQDim + head * kHeadDim);
+          const uint4 *src = reinterpret_cast<const uint4 *>(a.q) + (size_t)qt * (kHeadDim / 8) * 128 + et;
 #pragma unroll
-          for (int e = 0; e < 32; ++e) qq[e] = row_ok ? src[e] : make_uint4(0, 0, 0, 0);
+          for (int e = 0; e < 32; ++e) qq[e] = row_ok ? __ldcg(src + (size_t)e * 128) : make_uint4(0, 0, 0, 0);
         }
         const AUnit t = attn_unit(a, u, step0);
         const bool state_q = step0 && jq == 0;
@@ -1470,6 +1510,10 @@ __device__ void role_epi(const LoopArgs &a, uint8_t *smem, Bars &bs, uint32_t tm
       }
     }
   }
+  // every GEMM MMA this warp issued has completed before the CTA may free TMEM or exit
+  tc_commit_w(&bs.epi_fin);
+  dwait(&bs.epi_fin, 0, a);
+  __syncwarp();
 }
 
 __global__ void __launch_bounds__(kThreads, 1) k_loop(const __grid_constant__ LoopArgs a) {
@@ -1488,7 +1532,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_loop(const __grid_constant__ Lo
       mbar_init(&bs.a_empty[i], 1);
       bs.a_fills[i] = 0;
     }
-    mbar_init(&bs.acc_full, 1);
+    mbar_init(&bs.acc_full, 4);  // one tcgen05.commit per epilogue warp
     bs.tmem_done = 0;
     for (int i = 0; i < kKVBufs; ++i) {
       mbar_init(&bs.k_full[i], 32);  // one cp.async-completion arrival per loader lane (+ TMA bytes)
@@ -1504,6 +1548,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_loop(const __grid_constant__ Lo
     }
     mbar_init(&bs.q_full, 128);
     mbar_init(&bs.mma_fin, 1);
+    mbar_init(&bs.red_full, 1);
+    mbar_init(&bs.epi_fin, 4);
+    bs.red_fills = 0;
+    bs.epi_err = 0;
     bs.x_done = 0;
     bs.ready = 0;
     bs.last = 0;
@@ -1544,6 +1592,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_loop(const __grid_constant__ Lo
     if (warp == 3)
       for (int i = 0; i < kKVBufs; ++i)
         if (bs.v_fills[i]) dwait(&bs.v_full[i], (bs.v_fills[i] - 1) & 1u, a);
+    if (warp == 4 && bs.red_fills) dwait(&bs.red_full, (bs.red_fills - 1) & 1u, a);
   }
   tc_fence_before();
   __syncthreads();

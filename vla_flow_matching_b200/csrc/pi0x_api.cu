@@ -344,7 +344,9 @@ int ensure_workspace(pi0x_handle *h, int B, int P, int N) {
   // xn, att, act and u hold kLoopReps replicas for the persistent loop (bf16 mode)
   const size_t reps = h->bf16 ? kLoopReps : 1;
   add(reps * es * Rp * kWidth);
-  add(es * Rp * kQDim);
+  // q: the persistent loop stores it per 128-row query tile (up to one partial tile per sample more)
+  const size_t q_elems = Rp * kQDim + (h->bf16 ? (size_t)128 * nB * kHeadDim : 0);
+  add(es * q_elems);
   add(es * (size_t)L * Rp * kHeadDim);
   add(es * (size_t)L * Rp * kHeadDim);
   add(reps * es * Rp * kQDim);
@@ -378,7 +380,7 @@ int ensure_workspace(pi0x_handle *h, int B, int P, int N) {
   ws.ss_ld = (int)Rp;
   ws.rope_tab = (float *)ws.arena.take(4 * rope_floats);
   ws.xn = ws.arena.take(reps * es * Rp * kWidth);
-  ws.q = ws.arena.take(es * Rp * kQDim);
+  ws.q = ws.arena.take(es * q_elems);
   ws.ks = ws.arena.take(es * (size_t)L * Rp * kHeadDim);
   ws.vs = ws.arena.take(es * (size_t)L * Rp * kHeadDim);
   ws.att = ws.arena.take(reps * es * Rp * kQDim);
