@@ -221,15 +221,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     // a buffer is free again once S (K) or P.V (V) of the block it held has completed
     uint64_t *empty = is_v ? pv_done : k_empty;
     const uint32_t ring = sbase + (is_v ? kSmemV0 : kSmemK0);
-    if (lane == 0) {  // (the prefix map is unused, and zero, when there is no prefix key)
+    // (the prefix map is unused, and zero, when there is no prefix key).  Every lane that
+    // may issue a tensor copy acquires the maps itself: the fence orders the executing
+    // thread's tensor-map accesses only.
+    if (nv > 0) {
+      tma_map_acquire(pmap);
+      tma_map_acquire(pmap64);
+    }
+    tma_map_acquire(smap);
+    tma_map_acquire(smap64);
+    if (lane == 0) {
       if (nv > 0) {
-        tma_map_acquire(pmap);
-        tma_map_acquire(pmap64);
         tma_prefetch_desc(pmap);
         tma_prefetch_desc(pmap64);
       }
-      tma_map_acquire(smap);
-      tma_map_acquire(smap64);
       tma_prefetch_desc(smap);
       tma_prefetch_desc(smap64);
     }

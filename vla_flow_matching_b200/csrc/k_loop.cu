@@ -716,14 +716,16 @@ __device__ void role_loader(const LoopArgs &a, uint8_t *smem, Bars &bs, bool is_
         const AUnit t = attn_unit(a, u, step0);
         if (t.nb == 0) continue;
         if (!maps_ready) {
-          if (lane == 0) {
-            if (a.P > 0) {
-              tma_map_acquire(pmap);
-              tma_map_acquire(pmap32);
-            }
-            tma_map_acquire(smap);
-            tma_map_acquire(smap32);
+          // the maps are rewritten in global memory before every call: each lane that
+          // may issue a tensor copy with them (load_kv_tile) acquires them itself, since
+          // the fence orders the executing thread's tensor-map accesses only
+          if (a.P > 0) {
+            tma_map_acquire(pmap);
+            tma_map_acquire(pmap32);
           }
+          tma_map_acquire(smap);
+          tma_map_acquire(smap32);
+          __syncwarp();
           maps_ready = true;
         }
         const int *vi = a.vidx + (size_t)t.b * a.P;
