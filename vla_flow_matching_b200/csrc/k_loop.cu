@@ -520,20 +520,29 @@ __device__ void role_weights(const LoopArgs &a, uint8_t *smem, Bars &bs, int me)
       const bf16 *src = wt + (size_t)g.m * 128 * p.K;
       if (wnext && me == 0)
         prefetch_l2(wnext + (size_t)g.m * 128 * p.K + (size_t)g.kb0 * 128 * 64, (uint32_t)(g.kb1 - g.kb0) * kWSlotBytes);
-      for (int kb = g.kb0; kb < g.kb1; ++kb, ++wi) {
-        if ((int)(wi & 1u) != me) continue;  // the other issuing lane's fill
-        const int slot = wi % kWSlots;
-        const uint32_t n = wi / kWSlots;
-        if (n > 0 && !lwait(&bs.w_empty[slot], (n - 1) & 1u, a, kErrTimeoutProducer)) {
-          ok = false;
-          break;
+      // rounds of two K-blocks, one per lane, the two lanes in step (as the activation
+      // loader's four): a lane that waited alone in a diverged warp could hold back the
+      // other lane's fill that its own wait depends on
+      const int nk = g.kb1 - g.kb0;
+      for (int i0 = 0; i0 < nk && ok; i0 += 2) {
+        const int i = i0 + me;
+        bool good = true;
+        if (i < nk) {
+          const uint32_t f = wi + (uint32_t)i;
+          const int slot = f % kWSlots;
+          const uint32_t n = f / kWSlots;
+          if (n > 0) good = lwait(&bs.w_empty[slot], (n - 1) & 1u, a, kErrTimeoutProducer);
+          if (good) {
+            mbar_arrive_expect_tx(&bs.w_full[slot], kWSlotBytes);
+            bulk_load(smem_u32(smem + kOffW + slot * kWSlotBytes), src + (size_t)(g.kb0 + i) * 128 * 64, kWSlotBytes,
+                      &bs.w_full[slot]);
+            bs.w_fills[slot] = n + 1;
+          }
         }
-        mbar_arrive_expect_tx(&bs.w_full[slot], kWSlotBytes);
-        bulk_load(smem_u32(smem + kOffW + slot * kWSlotBytes), src + (size_t)kb * 128 * 64, kWSlotBytes,
-                  &bs.w_full[slot]);
-        bs.w_fills[slot] = n + 1;
-        if (kb + 1 >= g.kb1) LOOP_STAMP(gs, 5);
+        ok = __all_sync(0x3u, good);
       }
+      wi += (uint32_t)nk;
+      LOOP_STAMP(gs, 5);
     }
   }
 }
@@ -1141,9 +1150,9 @@ __device__ void role_epi(const LoopArgs &a, uint8_t *smem, Bars &bs, uint32_t tm
         ++acc_n;
         tc_fence_after();
         LOOP_STAMP(gs, 1);
+        const int used = nk < nch ? nk : nch;
         // partial tile, token-major: row et of the m-tile for the stored tokens (the sum
         // of the unit's chains, in chain order)
-        const int used = nk < nch ? nk : nch;
         float *mine = a.gpart + (size_t)u * 128 * NT;
         for (int c0 = r_lo & ~15; c0 < r_hi; c0 += 16) {
           float v[16];
