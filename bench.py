@@ -268,8 +268,11 @@ def roofline_of(wl, kernel_ms, call_ms):
 
 
 # DRAM bytes (read + write) per launch of the dominant kernel from an ncu capture of
-# the same build, keyed by (workload, kernel class); None when not captured.
-TRAFFIC = {}
+# the same build, keyed by (workload, kernel class); None when not captured.  full_b1:
+# k_loop over one Euler step (the full_b1_1step profiling case) read 734,413,056 B and
+# wrote 12,787,968 B; every step streams all weights (629 MB, more than L2), so the
+# ten-step launch moves ten times that.
+TRAFFIC = {("full_b1", "loop"): 10 * (734413056 + 12787968)}
 
 
 def measure(wl, args, sampler, inp, rank, dist, clocks_on):
@@ -332,7 +335,8 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="full_b1", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--workload", default="full_b1",
+                    choices=sorted(synth.WORKLOADS) + sorted(synth.PROFILE_WORKLOADS))
     ap.add_argument("--precision", default="bf16", choices=["bf16", "fp32"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-by-workload", action="store_true",
@@ -351,7 +355,7 @@ def main():
               f"python -m torch.distributed.run --nproc-per-node {args.gpus} bench.py --gpus {args.gpus}",
               file=sys.stderr)
         return 2
-    wl = synth.WORKLOADS[args.workload]
+    wl = {**synth.WORKLOADS, **synth.PROFILE_WORKLOADS}[args.workload]
     if args.impl == "reference":
         return run_reference(args, wl)
 

@@ -100,6 +100,13 @@ WORKLOADS: Dict[str, Workload] = {
                           mask_a=600),
 }
 
+#: Profiling case, not a benchmark config: one Euler step of full_b1.  Every step
+#: streams all of the expert's weights (629 MB against a 126 MB L2), so DRAM counters
+#: taken on it scale to full_b1's ten steps by the step count.
+PROFILE_WORKLOADS: Dict[str, Workload] = {
+    "full_b1_1step": dataclasses.replace(WORKLOADS["full_b1"], name="full_b1_1step", num_steps=1),
+}
+
 #: Tiny dims for the float64 brute force (pure-Python loops stay fast).
 TINY_BRUTE_DIMS = ExpertDims(width=16, depth=2, mlp_dim=32, num_heads=2,
                              num_kv_heads=1, head_dim=8, horizon=3,
