@@ -215,8 +215,8 @@ constexpr int kLoopNormSlots = 8;    // fused-norm partial sums: one slot per 12
 constexpr int kLoopKeyBlock = 32;    // attention key block of the loop kernel
 constexpr int kLoopMinGrid = 128;    // enough CTAs to split every GEMM's K over most SMs
 constexpr int kLoopReps = 1;         // replicas of each tiled activation operand
-constexpr int kLoopMaxMtiles = 64;
-constexpr int kLoopMaxSplits = 8;    // key-range splits of a query tile (the COMBINE registers)   // m-tiles of the widest GEMM (gate/up: 8192 / 128)
+constexpr int kLoopMaxMtiles = 64;   // m-tiles of the widest GEMM (gate/up: 8192 / 128)
+constexpr int kLoopMaxSplits = 8;    // key-range splits of a query tile (the COMBINE registers)
 
 __host__ __device__ inline int loop_layer_stages(int attn_splits) { return attn_splits > 1 ? 6 : 5; }
 __host__ __device__ inline int loop_stages_per_step(int L, int attn_splits) {
