@@ -1394,9 +1394,11 @@ __device__ void role_epi(const LoopArgs &a, uint8_t *smem, Bars &bs, uint32_t tm
             }
           }
         } else {
-          // partial O of unit u = (b * qps + ti) * splits + split as [u][4-dim chunk][row]:
-          // the 32 rows of a warp store 512 contiguous bytes per chunk
-          float4 *pbase = reinterpret_cast<float4 *>(a.part_o) + (size_t)u * (kHeadDim / 4) * 128 + et;
+          // partial O of unit u = (b * qps + ti) * splits + split, normalised by its own l
+          // and rounded to bf16 (as the attention output it becomes is), as [u][8-dim
+          // chunk][row]: the 32 rows of a warp store 512 contiguous bytes per chunk, and
+          // the unit's release waits for half the bytes an fp32 partial would take
+          uint4 *pbase = reinterpret_cast<uint4 *>(a.part_o) + (size_t)u * (kHeadDim / 8) * 128 + et;
           for (int c0 = 0; c0 < kHeadDim; c0 += 32) {
             float v[32];
             if (t.nb > 0) {
@@ -1407,9 +1409,9 @@ __device__ void role_epi(const LoopArgs &a, uint8_t *smem, Bars &bs, uint32_t tm
             }
             if (row_ok) {
 #pragma unroll
-              for (int e = 0; e < 8; ++e)
-                __stcg(pbase + (size_t)(c0 / 4 + e) * 128,
-                       make_float4(v[4 * e] * inv_l, v[4 * e + 1] * inv_l, v[4 * e + 2] * inv_l, v[4 * e + 3] * inv_l));
+              for (int e = 0; e < 32; ++e) v[e] *= inv_l;
+#pragma unroll
+              for (int e = 0; e < 4; ++e) __stcg(pbase + (size_t)(c0 / 8 + e) * 128, pack8(v + 8 * e));
             }
           }
           if (row_ok) {
@@ -1453,16 +1455,14 @@ __device__ void role_epi(const LoopArgs &a, uint8_t *smem, Bars &bs, uint32_t tm
             ls[sp] = ml.y;
           }
         }
-        // unit (qt, sp) holds chunk k of its row r at part_o float4 (unit * 64 + k) * 128 + r
-        const float4 *src = reinterpret_cast<const float4 *>(a.part_o) + ((size_t)qt * S * (kHeadDim / 4) + dg * 2) * 128 +
-                            rg * 32 + lane;
-        float4 x[kLoopMaxSplits][2];
+        // unit (qt, sp) holds 8-dim chunk k of its row r (bf16) at part_o uint4
+        // (unit * 32 + k) * 128 + r
+        const uint4 *src = reinterpret_cast<const uint4 *>(a.part_o) + ((size_t)qt * S * (kHeadDim / 8) + dg) * 128 +
+                           rg * 32 + lane;
+        uint4 x[kLoopMaxSplits];
 #pragma unroll
-        for (int sp = 0; sp < kLoopMaxSplits; ++sp)
-#pragma unroll
-          for (int e = 0; e < 2; ++e)
-            x[sp][e] = sp < S ? __ldcg(src + ((size_t)sp * (kHeadDim / 4) + e) * 128)  // (every unit stores its rows)
-                              : make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int sp = 0; sp < kLoopMaxSplits; ++sp)  // (every unit stores its rows)
+          x[sp] = sp < S ? __ldcg(src + (size_t)sp * (kHeadDim / 8) * 128) : make_uint4(0, 0, 0, 0);
         float M = -INFINITY;
 #pragma unroll
         for (int sp = 0; sp < kLoopMaxSplits; ++sp)
@@ -1474,12 +1474,12 @@ __device__ void role_epi(const LoopArgs &a, uint8_t *smem, Bars &bs, uint32_t tm
           if (!(sp < S && ls[sp] > 0.f)) continue;
           const float wgt = ls[sp] * ex2_approx(ms[sp] - M);
           den += wgt;
+          const uint32_t w4[4] = {x[sp].x, x[sp].y, x[sp].z, x[sp].w};
 #pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            o[4 * e] = fmaf(wgt, x[sp][e].x, o[4 * e]);
-            o[4 * e + 1] = fmaf(wgt, x[sp][e].y, o[4 * e + 1]);
-            o[4 * e + 2] = fmaf(wgt, x[sp][e].z, o[4 * e + 2]);
-            o[4 * e + 3] = fmaf(wgt, x[sp][e].w, o[4 * e + 3]);
+          for (int e = 0; e < 4; ++e) {
+            const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w4[e]));
+            o[2 * e] = fmaf(wgt, f.x, o[2 * e]);
+            o[2 * e + 1] = fmaf(wgt, f.y, o[2 * e + 1]);
           }
         }
         const int j = qi / kHeads, hd = qi % kHeads;
