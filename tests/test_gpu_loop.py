@@ -71,6 +71,43 @@ def test_loop_two_samples_ragged_prefix(masked, hole):
     s.close()
 
 
+def test_loop_full_128_row_tile():
+    """B=2 at horizon 63: 128 rows, the largest tile the loop takes (N = 128 tokens per
+    MMA, two accumulator chains per GEMM unit, an 8-slot activation ring, the largest
+    split-K slices); against the oracle, the multi-kernel path and itself."""
+    wl = small_wl(B=2, P=40, masked=20, horizon=63, depth=2, steps=2)
+    inp = synth.make_inputs(wl)
+    s = _sampler(wl.dims, wl.seed)
+    assert s.uses_loop(2) and not s.uses_loop(3)
+    a = run_gpu(s, inp)
+    assert np.array_equal(run_gpu(s, inp), a)
+    check(a, oracle_x0(inp), 0, "128-row loop")
+    s.debug_set_loop(False)
+    b = run_gpu(s, inp)
+    assert np.abs(a.astype(np.float64) - b).max() <= BF16_MAX
+    s.close()
+
+
+def test_loop_empty_prefix():
+    """No prefix keys at all: attention over the suffix only (state and action keys)."""
+    wl = small_wl(B=1, P=0, kind="all", depth=2, steps=2)
+    inp = synth.make_inputs(wl)
+    s = _sampler(wl.dims, wl.seed)
+    assert s.uses_loop(1)
+    check(run_gpu(s, inp), oracle_x0(inp), 0, "P=0 loop")
+    s.close()
+
+
+def test_loop_four_ragged_samples_short_horizon():
+    """B=4 at horizon 20 (84 rows, N = 96 tokens): ragged valid prefixes per sample."""
+    wl = small_wl(B=4, P=90, masked=35, horizon=20, depth=2, steps=3)
+    inp = synth.make_inputs(wl)
+    s = _sampler(wl.dims, wl.seed)
+    assert s.uses_loop(4)
+    check(run_gpu(s, inp), oracle_x0(inp), 0, "B=4 loop")
+    s.close()
+
+
 @pytest.mark.parametrize("stage", [1, 9], ids=["step0_mlp_out", "step0_layer1"])
 def test_stalled_stage_times_out_and_next_call_is_exact(stage):
     """Stage 1 is the action-time MLP output GEMM of step 0; stage 9 lies in layer 1
