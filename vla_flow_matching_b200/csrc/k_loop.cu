@@ -226,17 +226,21 @@ __device__ __forceinline__ void x_release(Bars &bs) {
   atomicAdd(&bs.x_done, 1u);
 }
 
-__device__ __forceinline__ void tmem_ld_x16(uint32_t taddr, float (&v)[16]) {
-  uint32_t r[16];
+// TMEM load of 32 lanes x 16 fp32 columns without its wait: issue several, then one
+// tc_wait_ld_regs64 over the registers they write (named there, so that no use of
+// them moves above the wait).
+__device__ __forceinline__ void tmem_ld_x16_nw(uint32_t taddr, uint32_t *r) {
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
       "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
       : "r"(taddr));
-  tc_wait_ld();
-#pragma unroll
-  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+__device__ __forceinline__ void tc_wait_ld_regs64(uint32_t (&r)[64]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), "+r"(r[30]), "+r"(r[31]), "+r"(r[32]), "+r"(r[33]), "+r"(r[34]), "+r"(r[35]), "+r"(r[36]), "+r"(r[37]), "+r"(r[38]), "+r"(r[39]), "+r"(r[40]), "+r"(r[41]), "+r"(r[42]), "+r"(r[43]), "+r"(r[44]), "+r"(r[45]), "+r"(r[46]), "+r"(r[47]), "+r"(r[48]), "+r"(r[49]), "+r"(r[50]), "+r"(r[51]), "+r"(r[52]), "+r"(r[53]), "+r"(r[54]), "+r"(r[55]), "+r"(r[56]), "+r"(r[57]), "+r"(r[58]), "+r"(r[59]), "+r"(r[60]), "+r"(r[61]), "+r"(r[62]), "+r"(r[63])
+               :
+               : "memory");
 }
 
 // Store of 8 bf16 at offset `off` of every replica of a tiled activation buffer.
@@ -1155,14 +1159,27 @@ __device__ void role_epi(const LoopArgs &a, uint8_t *smem, Bars &bs, uint32_t tm
         // of the unit's chains, in chain order)
         float *mine = a.gpart + (size_t)u * 128 * NT;
         for (int c0 = r_lo & ~15; c0 < r_hi; c0 += 16) {
-          float v[16];
-          tmem_ld_x16(tmem + t_lane + kTmemAcc + (uint32_t)c0, v);
-          for (int c = 1; c < used; ++c) {
-            float w[16];
-            tmem_ld_x16(tmem + t_lane + kTmemAcc + (uint32_t)(c * NT + c0), w);
+          // the group's columns of every chain, loaded together under one wait
+          uint32_t r[64];
 #pragma unroll
-            for (int i = 0; i < 16; ++i) v[i] += w[i];
+          for (int c = 0; c < 4; ++c) {
+            if (c < used) {
+              tmem_ld_x16_nw(tmem + t_lane + kTmemAcc + (uint32_t)(c * NT + c0), r + 16 * c);
+            } else {
+#pragma unroll
+              for (int i = 0; i < 16; ++i) r[16 * c + i] = 0u;
+            }
           }
+          tc_wait_ld_regs64(r);
+          float v[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+#pragma unroll
+          for (int c = 1; c < 4; ++c)
+            if (c < used) {
+#pragma unroll
+              for (int i = 0; i < 16; ++i) v[i] += __uint_as_float(r[16 * c + i]);
+            }
 #pragma unroll
           for (int i = 0; i < 16; ++i) __stcg(mine + (size_t)(c0 + i) * 128 + et, v[i]);
         }
@@ -1399,19 +1416,19 @@ __device__ void role_epi(const LoopArgs &a, uint8_t *smem, Bars &bs, uint32_t tm
           // chunk][row]: the 32 rows of a warp store 512 contiguous bytes per chunk, and
           // the unit's release waits for half the bytes an fp32 partial would take
           uint4 *pbase = reinterpret_cast<uint4 *>(a.part_o) + (size_t)u * (kHeadDim / 8) * 128 + et;
-          for (int c0 = 0; c0 < kHeadDim; c0 += 32) {
-            float v[32];
+          for (int c0 = 0; c0 < kHeadDim; c0 += 64) {
+            float v[64];
             if (t.nb > 0) {
-              tmem_ld_32x32b_x32(tmem + t_lane + kTmemO + c0, v);
+              tmem_ld_32x32b_x64(tmem + t_lane + kTmemO + c0, v);
             } else {
 #pragma unroll
-              for (int e = 0; e < 32; ++e) v[e] = 0.f;
+              for (int e = 0; e < 64; ++e) v[e] = 0.f;
             }
             if (row_ok) {
 #pragma unroll
-              for (int e = 0; e < 32; ++e) v[e] *= inv_l;
+              for (int e = 0; e < 64; ++e) v[e] *= inv_l;
 #pragma unroll
-              for (int e = 0; e < 4; ++e) __stcg(pbase + (size_t)(c0 / 8 + e) * 128, pack8(v + 8 * e));
+              for (int e = 0; e < 8; ++e) __stcg(pbase + (size_t)(c0 / 8 + e) * 128, pack8(v + 8 * e));
             }
           }
           if (row_ok) {
