@@ -27,7 +27,7 @@
 //
 // Roles (256 threads):
 //   warp 0    weight producer (lanes 0 and 1, alternate K-blocks): streams this CTA's
-//             weight K-blocks of every stage, in program order, into a 5-slot ring of
+//             weight K-blocks of every stage, in program order, into a 6-slot ring of
 //             16 KB.  Weights are inputs, so it runs ahead of the activations across
 //             stage boundaries, bounded only by the ring.
 //   warp 1    tcgen05.mma issuer of attention units (S = Q K^T, O += P V).
@@ -60,7 +60,7 @@
 // Shared memory: region X (128 KB) holds either the activation ring of a GEMM unit
 // or the K/V rings (3 x 16 KB each) and P buffers (2 x 16 KB) of an attention unit,
 // handed from unit to unit through a counter of units whose MMAs have completed; then
-// the weight ring (5 x 16 KB).
+// the weight ring (6 x 16 KB); XOUT keeps its normalised row in region X.
 //
 // Every wait is bounded (LoopArgs::wait_ns) and gives up early once the error word
 // is set; on the way out each role waits for the copies it issued, the MMA warp for
@@ -89,7 +89,7 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr uint32_t kXBytes = 128 * 1024;
-constexpr int kWSlots = 5;
+constexpr int kWSlots = 6;
 constexpr uint32_t kWSlotBytes = 16384;           // one K-block of a 128-row weight m-tile
 constexpr int kKB = kLoopKeyBlock;            // 32 keys per attention block
 constexpr int kKVBufs = 3;
@@ -130,8 +130,10 @@ struct Bars {
   uint32_t epi_err;  // an epilogue warp's wait gave up (read by all four after a barrier)
 };
 constexpr uint32_t kBarBytes = ((sizeof(Bars) + 127) / 128) * 128;
-constexpr uint32_t kOffRow = kOffBar + kBarBytes;   // XOUT: the normalised row (1024 fp32)
-constexpr uint32_t kSmemTotal = kOffRow + 4096 + 1024 /* alignment slack */;
+// GEMM reduce scratch: the slice's per-token rstd and RoPE positions (128 + 128 words).
+// (XOUT's normalised row uses region X, which no copy fills during that stage.)
+constexpr uint32_t kOffScratch = kOffBar + kBarBytes;
+constexpr uint32_t kSmemTotal = kOffScratch + 1024 + 1024 /* alignment slack */;
 static_assert(kSmemTotal <= 232448, "shared memory per CTA");
 
 // TMEM columns: S 0..127 (two buffers x two dim-halves of 32 columns), Q 128..255
@@ -1092,7 +1094,8 @@ __device__ void role_epi(const LoopArgs &a, uint8_t *smem, Bars &bs, uint32_t tm
   const int nas = a_slots(a);
   const uint32_t asb = a_slot_bytes(a);
   bool ok = true;
-  float *yrow = reinterpret_cast<float *>(smem + kOffRow);
+  float *yrow = reinterpret_cast<float *>(smem + kOffX);         // XOUT's normalised row
+  float *scratch = reinterpret_cast<float *>(smem + kOffScratch);  // GEMM reduce
   auto open = [&](int gs) -> bool {
     const bool good = gate(bs, gs, a);
     LOOP_STAMP(gs, 0);
@@ -1196,8 +1199,8 @@ __device__ void role_epi(const LoopArgs &a, uint8_t *smem, Bars &bs, uint32_t tm
         red_slice(r_lo, r_hi, p.ksplit, g.s, t0, t1);
         if (t0 < t1) {
           // per-token rstd / RoPE position of the slice while the other splits finish
-          float *rstd_s = yrow;
-          int *pos_s = reinterpret_cast<int *>(yrow + kLoopMaxRows);
+          float *rstd_s = scratch;
+          int *pos_s = reinterpret_cast<int *>(scratch + kLoopMaxRows);
           if (si.kind == LK_QKV || si.kind == LK_GU) {
             const float *ssn = si.kind == LK_QKV ? a.ss_a : a.ss_m;
             for (int j = et; j < t1 - t0; j += 128) {
@@ -1531,6 +1534,7 @@ __device__ void role_epi(const LoopArgs &a, uint8_t *smem, Bars &bs, uint32_t tm
       if (!ok) break;
       const int nch = (a.A + 15) / 16;
       for (int u = blockIdx.x; u < xout_units(a); u += nc) xout_unit(a, bs, yrow, u / nch, u % nch, si.step, et);
+      fence_proxy_async_smem();  // region X is next filled by bulk / tensor copies
       epi_bar();
       if (et == 0) {
         LOOP_STAMP(gs, 2);
