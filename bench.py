@@ -272,7 +272,7 @@ def roofline_of(wl, kernel_ms, call_ms):
 # k_loop over one Euler step (the full_b1_1step profiling case) read 734,413,056 B and
 # wrote 12,787,968 B; every step streams all weights (629 MB, more than L2), so the
 # ten-step launch moves ten times that.
-TRAFFIC = {("full_b1", "loop"): 10 * (734413056 + 12787968)}
+TRAFFIC = {("full_b1", "loop"): 10 * (709838336 + 7940096)}
 
 
 def measure(wl, args, sampler, inp, rank, dist, clocks_on):
