@@ -13,7 +13,7 @@
 // invariant to the order of the keys.  Masked prefix positions are never read (the
 // page adds -2.38e38 to their logits, whose exp is exactly 0 in fp32).
 //
-// Warp roles (224 threads):
+// Warp roles (256 threads):
 //  * warps 0-3: one query row per thread.  Q goes to TMEM (the A operand of
 //    S = Q K^T); per key block the thread reads its S row from TMEM, forms
 //    P = 2^(s - m) with an online softmax, writes P (bf16) to shared memory, and
@@ -22,9 +22,10 @@
 //    block whose 64 slots are consecutive rows of one tensor is one 64-row TMA box
 //    per 64 dims; otherwise each such run of 8 slots is an 8-row box, and other runs
 //    are copied row by row with cp.async.
-//  * warp 6: tcgen05.mma issuer (the whole warp runs the loop, one elected lane
-//    issues): S(j+1) before PV(j), so the softmax of block j+1 overlaps the P.V of
-//    block j.
+//  * warp 6 / warp 7: tcgen05.mma issuers of S = Q K^T / of O += P V (the whole warp
+//    runs the loop, one elected lane issues).  An MMA costs its issuing warp a fixed
+//    time, so the two streams (16 and 4 MMAs per block) are issued side by side; S
+//    runs up to two blocks ahead of the softmax (two S buffers).
 // All hand-offs are mbarriers (TMA transaction bytes, cp.async completion, tcgen05
 // commits, thread arrivals) and every wait is bounded.  O / l at the end
 // normalises.  With split-KV (small batches) every split writes O/l and (m, l) and
@@ -62,7 +63,7 @@ constexpr uint32_t kTmemQ = 128;
 constexpr uint32_t kTmemO = 256;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleSlack = 8.0f;  // log2 units
-constexpr int kThreads = 224;
+constexpr int kThreads = 256;
 constexpr unsigned kFull = 0xffffffffu;
 }  // namespace
 
@@ -193,7 +194,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int i = 0; i < kPBufs; ++i) mbar_init(&p_full[i], 128);
     mbar_init(q_full, 128);
-    mbar_init(mma_done, 1);
+    mbar_init(mma_done, 2);  // one commit per MMA-issuing warp
     fence_mbar_init();
   }
   if (warp == 0) {
@@ -248,8 +249,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     cp_async_commit();  // nothing may still land in shared memory once the CTA exits
     cp_async_wait<0>();
-  } else if (warp == 6) {
-    // ------------------------------------------------------------ MMA issuer
+  } else if (warp == 6 || warp == 7) {
+    // ------------------------------------------------------------ MMA issuers
     // The whole warp runs the loop (waits and descriptors stay warp-uniform); one
     // elected lane issues each MMA and commit.
     if (nb > 0) {
@@ -294,14 +295,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_commit_w(&pv_done[vbuf]);  // V buffer and P buffer free, O updated
         return true;
       };
-      ok = __all_sync(kFull, mbar_wait(q_full, 0, err, kErrTimeoutMma));
-      tc_fence_after();
-      if (ok) ok = issue_s(0);
-      for (int j = 0; j < nb && ok; ++j) {
-        if (j + 1 < nb) ok = issue_s(j + 1);
-        if (ok) ok = issue_pv(j);
+      if (warp == 6) {
+        ok = __all_sync(kFull, mbar_wait(q_full, 0, err, kErrTimeoutMma));
+        tc_fence_after();
+        for (int j = 0; j < nb && ok; ++j) ok = issue_s(j);
+      } else {
+        for (int j = 0; j < nb && ok; ++j) ok = issue_pv(j);
       }
-      // every MMA issued (also after a failed wait) has finished before TMEM is freed
+      // every MMA issued by either warp (also after a failed wait) has finished before
+      // TMEM is freed
       tc_commit_w(mma_done);
       mbar_wait(mma_done, 0, err, kErrTimeoutMma);
     }
